@@ -1,0 +1,163 @@
+"""ctypes binding of the C ABI in include/svdq.h (argument marshalling only).
+
+Every function has the name of its C entry point and takes torch tensors
+(or None for NULL) plus an optional CUDA stream; it passes their device
+pointers to the shared library and raises ``SvdqError`` on any status other
+than SVDQ_OK.  No arithmetic of the layer happens here.  If the compiled
+library is missing, importing this module fails loudly: there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsvdq_b200.so")
+
+SVDQ_OK = 0
+SVDQ_ERR_INVALID_ARG = 1
+SVDQ_ERR_UNSUPPORTED_SHAPE = 2
+SVDQ_ERR_UNSUPPORTED_DEVICE = 3
+SVDQ_ERR_CUDA = 4
+SVDQ_ERR_TIMEOUT = 5
+
+SVDQ_NVFP4 = 0
+SVDQ_INT4 = 1
+PRECISIONS = {"nvfp4": SVDQ_NVFP4, "int4": SVDQ_INT4}
+GROUP_SIZES = {"nvfp4": 16, "int4": 64}
+
+# Every entry point declared in include/svdq.h.
+EXPORTS = (
+    "svdq_status_string", "svdq_abi_version", "svdq_buffer_sizes", "svdq_pack_weight",
+    "svdq_quantize_act", "svdq_gemm_w4a4", "svdq_device_status",
+    "svdq_debug_set_wait_limit_ns", "svdq_debug_timeout_probe", "svdq_debug_override_capability",
+)
+
+
+class SvdqError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+
+
+class svdq_sizes(ctypes.Structure):
+    _fields_ = [("codes_bytes", ctypes.c_size_t), ("scales_bytes", ctypes.c_size_t),
+                ("lowrank_bytes", ctypes.c_size_t)]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"the CUDA library {LIB_PATH} is not built; run __graft_entry__.build() "
+                          "(there is no CPU fallback)")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I, I64, U64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_uint64
+    lib.svdq_status_string.argtypes = [I]
+    lib.svdq_status_string.restype = ctypes.c_char_p
+    lib.svdq_abi_version.argtypes = []
+    lib.svdq_abi_version.restype = I
+    lib.svdq_buffer_sizes.argtypes = [I, I64, I64, I, ctypes.POINTER(svdq_sizes)]
+    lib.svdq_buffer_sizes.restype = I
+    lib.svdq_pack_weight.argtypes = [I, I, P, I64, I64, P, P, P, I, P, P, P, P, P, P, P]
+    lib.svdq_pack_weight.restype = I
+    lib.svdq_quantize_act.argtypes = [I, I, P, I64, I64, P, P, I, P, P, I, P, P, P, P]
+    lib.svdq_quantize_act.restype = I
+    lib.svdq_gemm_w4a4.argtypes = [I, I, P, P, P, I64, P, P, P, I64, I64, P, P, I, P, P, P]
+    lib.svdq_gemm_w4a4.restype = I
+    lib.svdq_device_status.argtypes = [I, ctypes.POINTER(ctypes.c_int)]
+    lib.svdq_device_status.restype = I
+    lib.svdq_debug_set_wait_limit_ns.argtypes = [U64]
+    lib.svdq_debug_set_wait_limit_ns.restype = I
+    lib.svdq_debug_timeout_probe.argtypes = [P]
+    lib.svdq_debug_timeout_probe.restype = I
+    lib.svdq_debug_override_capability.argtypes = [I, I]
+    lib.svdq_debug_override_capability.restype = None
+    return lib
+
+
+lib = _load()
+
+
+def status_string(status: int) -> str:
+    return lib.svdq_status_string(int(status)).decode()
+
+
+def _ptr(t) -> int | None:
+    """Device pointer of a tensor (None -> NULL); raw ints pass through."""
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        import torch
+
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(status: int, where: str) -> None:
+    if status != SVDQ_OK:
+        raise SvdqError(status, where)
+
+
+def _prec(p) -> int:
+    return PRECISIONS[p] if isinstance(p, str) else int(p)
+
+
+def svdq_abi_version() -> int:
+    return int(lib.svdq_abi_version())
+
+
+def svdq_buffer_sizes(precision, rows: int, K: int, rank: int) -> dict:
+    out = svdq_sizes()
+    _check(lib.svdq_buffer_sizes(_prec(precision), int(rows), int(K), int(rank), ctypes.byref(out)),
+           "svdq_buffer_sizes")
+    return {"codes_bytes": out.codes_bytes, "scales_bytes": out.scales_bytes, "lowrank_bytes": out.lowrank_bytes}
+
+
+def svdq_pack_weight(precision, group_size, R, N, K, lam, L_down, L_up, rank, w_codes, w_scales,
+                     w_tensor_scale, inv_lambda, L_down_t, L_up_t, stream=None) -> None:
+    _check(lib.svdq_pack_weight(_prec(precision), int(group_size), _ptr(R), int(N), int(K), _ptr(lam),
+                                _ptr(L_down), _ptr(L_up), int(rank), _ptr(w_codes), _ptr(w_scales),
+                                _ptr(w_tensor_scale), _ptr(inv_lambda), _ptr(L_down_t), _ptr(L_up_t),
+                                _stream(stream)), "svdq_pack_weight")
+
+
+def svdq_quantize_act(precision, group_size, x, M, K, inv_lambda, x_tensor_scale, compute_scale,
+                      w_tensor_scale, L_down_t, rank, x_codes, x_scales, lowrank_act, stream=None) -> None:
+    _check(lib.svdq_quantize_act(_prec(precision), int(group_size), _ptr(x), int(M), int(K), _ptr(inv_lambda),
+                                 _ptr(x_tensor_scale), int(bool(compute_scale)), _ptr(w_tensor_scale),
+                                 _ptr(L_down_t), int(rank), _ptr(x_codes), _ptr(x_scales), _ptr(lowrank_act),
+                                 _stream(stream)), "svdq_quantize_act")
+
+
+def svdq_gemm_w4a4(precision, group_size, x_codes, x_scales, x_tensor_scale, M, w_codes, w_scales,
+                   w_tensor_scale, N, K, lowrank_act, L_up_t, rank, bias, y, stream=None) -> None:
+    _check(lib.svdq_gemm_w4a4(_prec(precision), int(group_size), _ptr(x_codes), _ptr(x_scales),
+                              _ptr(x_tensor_scale), int(M), _ptr(w_codes), _ptr(w_scales), _ptr(w_tensor_scale),
+                              int(N), int(K), _ptr(lowrank_act), _ptr(L_up_t), int(rank), _ptr(bias), _ptr(y),
+                              _stream(stream)), "svdq_gemm_w4a4")
+
+
+def svdq_device_status(clear: bool = True) -> tuple[int, int]:
+    """(status, site) after synchronising the device; does not raise."""
+    site = ctypes.c_int(0)
+    st = lib.svdq_device_status(int(bool(clear)), ctypes.byref(site))
+    return int(st), int(site.value)
+
+
+def svdq_debug_set_wait_limit_ns(ns: int) -> None:
+    _check(lib.svdq_debug_set_wait_limit_ns(int(ns)), "svdq_debug_set_wait_limit_ns")
+
+
+def svdq_debug_timeout_probe(stream=None) -> None:
+    _check(lib.svdq_debug_timeout_probe(_stream(stream)), "svdq_debug_timeout_probe")
+
+
+def svdq_debug_override_capability(major: int, minor: int = 0) -> None:
+    lib.svdq_debug_override_capability(int(major), int(minor))

@@ -1,0 +1,239 @@
+// gemm_nvfp4.cuh -- block-scaled FP4 GEMM of the SVDQ W4A4 layer (sm_100a).
+//
+//   acc[m, n]  = sum_k (q_x[m,k] e_x[m,k/16]) (q_w[n,k] e_w[n,k/16])   FP4 x FP4, fp32 in TMEM
+//   acc[m, n] += sum_j L'[m, j] L_up[j, n]       rank-r branch, bf16 MMA into the same accumulator
+//   y[m, n]    = bf16( S_x S_w acc[m, n] + b[n] )
+// where L' = ((x/lambda) . L_down) / (S_x S_w) comes from the quantizer.  The
+// "NVFP4 runtime kernel with SVDQ low-rank correction" of the Diffusers docs
+// page "Nunchaku Lite" ("Supported quantization types" table).
+//
+// One CTA computes a 128 x 256 tile: warp 0 issues TMA loads (codes with
+// 128-byte swizzle, scale blocks with bulk copies) into a 4-stage ring, warp 1
+// copies the scale blocks to TMEM and issues tcgen05.mma (kind::mxf4nvf4,
+// K = 64 per instruction, then kind::f16 for the rank-r chunks), warps 2..5
+// drain the fp32 accumulator from TMEM and store bf16.
+#pragma once
+#include "sm100_ptx.cuh"
+
+namespace svdq {
+namespace gm {
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK_BYTES = 128;                 // 256 FP4 values of K per row per stage
+constexpr int kStages = 4;
+constexpr int A_BYTES = BM * BK_BYTES;        // 16 KB (also holds a 128 x 64 bf16 rank-r tile)
+constexpr int B_BYTES = BN * BK_BYTES;        // 32 KB (also holds a 256 x 64 bf16 L_up tile)
+constexpr int SFA_BYTES = 4 * 512;            // 4 scale blocks: 128 rows x 16 groups
+constexpr int SFB_BYTES = 8 * 512;            // 2 row blocks x 4 scale blocks
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+constexpr int kThreads = 192;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t ACC_COL = 0;               // 256 fp32 columns
+constexpr uint32_t SFA_COL = 256;             // 4 k-steps x 4 columns
+constexpr uint32_t SFB_COL = 272;             // 4 k-steps x 8 columns
+constexpr size_t SMEM_BYTES = 1024 + (size_t)kStages * STAGE_BYTES + 256;
+}  // namespace gm
+
+struct GemmArgs {
+    const uint8_t* x_scales;
+    const uint8_t* w_scales;
+    const float* x_scale;
+    const float* w_scale;
+    const __nv_bfloat16* bias;   // may be null
+    __nv_bfloat16* y;
+    int M, N, K, rank;
+    int kg4;                     // K / 64: scale blocks per 128 rows
+    int n_sf_blocks;             // ceil(N / 128): 128-row blocks present in w_scales
+};
+
+enum : uint32_t { kSiteGmEmpty = 16, kSiteGmFull = 17, kSiteGmAcc = 18, kSiteGmDrain = 19 };
+
+__global__ void __launch_bounds__(gm::kThreads, 1)
+    gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_xc, const __grid_constant__ CUtensorMap tm_wc,
+                      const __grid_constant__ CUtensorMap tm_L, const __grid_constant__ CUtensorMap tm_Lup,
+                      GemmArgs a) {
+    using namespace gm;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)kStages * STAGE_BYTES);
+    uint64_t* empty = full + kStages;
+    uint64_t* accb = empty + kStages;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accb + 1);
+    __shared__ int s_issued, s_consumed, s_failed;
+
+    const uint32_t warp = warp_id(), lane = lane_id();
+    const int m_tile = blockIdx.x, n_tile = blockIdx.y;
+    const int m0 = m_tile * BM, n0 = n_tile * BN;
+    const int n_kb = (a.K + 255) / 256;
+    const int n_lr = a.rank > 0 ? (a.rank + 63) / 64 : 0;
+    const int total = n_kb + n_lr;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(accb, 1);
+        s_issued = 0;
+        s_consumed = 0;
+        s_failed = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tensormap(&tm_xc);
+        prefetch_tensormap(&tm_wc);
+        if (a.rank > 0) {
+            prefetch_tensormap(&tm_L);
+            prefetch_tensormap(&tm_Lup);
+        }
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            int it = 0;
+            for (; it < total; ++it) {
+                const int s = it % kStages;
+                const uint32_t ph = (uint32_t)(it / kStages) & 1u;
+                if (!mbar_wait(&empty[s], ph ^ 1u, kSiteGmEmpty)) {
+                    s_failed = 1;
+                    break;
+                }
+                uint8_t* sa = smem + (size_t)s * STAGE_BYTES;
+                uint8_t* sb = sa + A_BYTES;
+                if (it < n_kb) {
+                    const int kb = it;
+                    const int natoms = min(4, a.kg4 - 4 * kb);
+                    const uint32_t sf_bytes = (uint32_t)natoms * 512u;
+                    const int nb0 = 2 * n_tile;
+                    const int nbv = (nb0 < a.n_sf_blocks ? 1 : 0) + (nb0 + 1 < a.n_sf_blocks ? 1 : 0);
+                    mbar_arrive_expect_tx(&full[s], A_BYTES + B_BYTES + sf_bytes * (1u + (uint32_t)nbv));
+                    tma_load_2d(sa, &tm_xc, &full[s], kb * BK_BYTES, m0);
+                    tma_load_2d(sb, &tm_wc, &full[s], kb * BK_BYTES, n0);
+                    uint8_t* sfa = sb + B_BYTES;
+                    uint8_t* sfb = sfa + SFA_BYTES;
+                    bulk_load(sfa, a.x_scales + ((int64_t)m_tile * a.kg4 + 4 * kb) * 512, sf_bytes, &full[s]);
+                    for (int rb = 0; rb < nbv; ++rb)
+                        bulk_load(sfb + rb * 2048, a.w_scales + ((int64_t)(nb0 + rb) * a.kg4 + 4 * kb) * 512,
+                                  sf_bytes, &full[s]);
+                } else {
+                    const int c = it - n_kb;
+                    mbar_arrive_expect_tx(&full[s], A_BYTES + B_BYTES);
+                    tma_load_2d(sa, &tm_L, &full[s], c * 64, m0);
+                    tma_load_2d(sb, &tm_Lup, &full[s], c * 64, n0);
+                }
+            }
+            s_issued = it;
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc_fp4 = idesc_nvfp4(BN);
+            const uint32_t idesc_lr = idesc_bf16_f32(BN);
+            bool ok = true;
+            int it = 0;
+            for (; it < total; ++it) {
+                const int s = it % kStages;
+                const uint32_t ph = (uint32_t)(it / kStages) & 1u;
+                if (!mbar_wait(&full[s], ph, kSiteGmFull)) {
+                    ok = false;
+                    s_failed = 1;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t sa = smem_u32(smem + (size_t)s * STAGE_BYTES);
+                const uint32_t sb = sa + A_BYTES;
+                if (it < n_kb) {
+                    const uint32_t sfa = sb + B_BYTES;
+                    const uint32_t sfb = sfa + SFA_BYTES;
+                    const int nks = min(4, a.kg4 - 4 * it);
+                    for (int j = 0; j < nks; ++j) {
+                        tmem_cp_32x128b_x4(tmem + SFA_COL + 4u * j, desc_sf_block(sfa + 512u * j));
+                        tmem_cp_32x128b_x4(tmem + SFB_COL + 8u * j, desc_sf_block(sfb + 512u * j));
+                        tmem_cp_32x128b_x4(tmem + SFB_COL + 8u * j + 4u, desc_sf_block(sfb + 2048u + 512u * j));
+                    }
+                    for (int j = 0; j < nks; ++j)
+                        mma_nvfp4(tmem + ACC_COL, desc_sw128(sa + 32u * j), desc_sw128(sb + 32u * j), idesc_fp4,
+                                  tmem + SFA_COL + 4u * j, tmem + SFB_COL + 8u * j, (it > 0 || j > 0) ? 1u : 0u);
+                } else {
+                    const int c = it - n_kb;
+                    const int nks = min(4, (a.rank - 64 * c + 15) / 16);
+                    for (int j = 0; j < nks; ++j)
+                        mma_bf16(tmem + ACC_COL, desc_sw128(sa + 32u * j), desc_sw128(sb + 32u * j), idesc_lr, 1u);
+                }
+                tc_commit(&empty[s]);
+            }
+            s_consumed = it;
+            if (ok) tc_commit(accb);
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const uint32_t q = warp & 3u;
+        const int row = (int)(32u * q + lane);
+        const int64_t grow = (int64_t)m0 + row;
+        const bool ok = mbar_wait(accb, 0, kSiteGmAcc);
+        if (!ok) s_failed = 1;
+        tc_fence_after();
+        const float S = __fmul_rn(*a.x_scale, *a.w_scale);
+        for (int c = 0; c < BN / 32; ++c) {
+            const int n = n0 + 32 * c;
+            if (n >= a.N) break;
+            uint32_t r[32];
+            tmem_ld_32x32b_x32(tmem + ((32u * q) << 16) + ACC_COL + 32u * c, r);
+            tmem_ld_wait();
+            if (!ok || grow >= a.M) continue;
+            const int nvec = (a.N - n >= 32) ? 4 : 2;   // N % 16 == 0: a tail chunk has 16 columns
+            float bv[32];
+            if (a.bias) {
+                const uint4* bp = reinterpret_cast<const uint4*>(a.bias + n);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const uint4 w = (i < nvec) ? __ldg(bp + i) : make_uint4(0u, 0u, 0u, 0u);
+                    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                    for (int p = 0; p < 4; ++p) {
+                        bv[8 * i + 2 * p] = bf16lo_to_f32(ws[p]);
+                        bv[8 * i + 2 * p + 1] = bf16hi_to_f32(ws[p]);
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) bv[i] = 0.0f;
+            }
+            uint32_t packed[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const float o0 = fmaf(__uint_as_float(r[2 * i]), S, bv[2 * i]);
+                const float o1 = fmaf(__uint_as_float(r[2 * i + 1]), S, bv[2 * i + 1]);
+                const __nv_bfloat162 h = __floats2bfloat162_rn(o0, o1);
+                packed[i] = *reinterpret_cast<const uint32_t*>(&h);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(a.y + grow * (int64_t)a.N + n);
+            for (int i = 0; i < nvec; ++i)
+                dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+        }
+    }
+
+    __syncthreads();
+    if (s_failed && warp == 0 && lane == 0) {
+        // on a timeout, let the loads already issued land before the CTA exits
+        for (int it = s_consumed; it < s_issued; ++it)
+            mbar_wait(&full[it % kStages], (uint32_t)(it / kStages) & 1u, kSiteGmDrain);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+}  // namespace svdq

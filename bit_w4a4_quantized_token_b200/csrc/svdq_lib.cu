@@ -1,0 +1,470 @@
+// svdq_lib.cu -- host side of the C ABI declared in include/svdq.h: argument
+// validation, the device-capability check, TMA descriptor construction and
+// kernel launches.  All kernels live in the headers included below; this is
+// the library's single translation unit.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "svdq.h"
+#include "sm100_ptx.cuh"
+#include "quant_nvfp4.cuh"
+#include "gemm_nvfp4.cuh"
+#include "int4.cuh"
+
+namespace svdq {
+namespace {
+
+constexpr int kAbiVersion = 1;
+
+// ------------------------------------------------------------- validation
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+svdq_status check_precision(svdq_precision p, int group_size) {
+    if (p == SVDQ_NVFP4) return group_size == 16 ? SVDQ_OK : SVDQ_ERR_INVALID_ARG;
+    if (p == SVDQ_INT4) return group_size == 64 ? SVDQ_OK : SVDQ_ERR_INVALID_ARG;
+    return SVDQ_ERR_INVALID_ARG;
+}
+
+svdq_status check_rank(int rank) {
+    return (rank >= 0 && rank <= 256 && rank % 16 == 0) ? SVDQ_OK : SVDQ_ERR_INVALID_ARG;
+}
+
+svdq_status check_dims(int64_t rows, int64_t K) {
+    if (rows < 1 || rows >= (int64_t(1) << 31)) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+    if (K < 64 || K >= (int64_t(1) << 31) || K % 64 != 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+    return SVDQ_OK;
+}
+
+svdq_status check_ptr(const void* p) {
+    if (p == nullptr || !aligned16(p)) return SVDQ_ERR_INVALID_ARG;
+    return SVDQ_OK;
+}
+
+svdq_status check_opt_ptr(const void* p) { return (p == nullptr || aligned16(p)) ? SVDQ_OK : SVDQ_ERR_INVALID_ARG; }
+
+#define SVDQ_TRY(expr)                          \
+    do {                                        \
+        const svdq_status _st = (expr);         \
+        if (_st != SVDQ_OK) return _st;         \
+    } while (0)
+
+int64_t round_up(int64_t v, int64_t m) { return (v + m - 1) / m * m; }
+
+// ------------------------------------------------------------ the device
+std::mutex g_mutex;
+int g_override_major = -1, g_override_minor = 0;
+constexpr int kMaxDevices = 64;
+bool g_device_ready[kMaxDevices];
+
+svdq_status cuda_fail() {
+    cudaGetLastError();  // clear a sticky-free error so later calls start clean
+    return SVDQ_ERR_CUDA;
+}
+
+// Rejects anything but compute capability 10.0 before any launch, and sets
+// the kernels' shared-memory limits once per device.
+svdq_status check_device() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return SVDQ_ERR_UNSUPPORTED_DEVICE;
+    }
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+        cudaGetLastError();
+        return SVDQ_ERR_UNSUPPORTED_DEVICE;
+    }
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (g_override_major >= 0) {
+        major = g_override_major;
+        minor = g_override_minor;
+    }
+    if (major != 10 || minor != 0) return SVDQ_ERR_UNSUPPORTED_DEVICE;
+    if (dev < 0 || dev >= kMaxDevices) return SVDQ_ERR_UNSUPPORTED_DEVICE;
+    if (!g_device_ready[dev]) {
+        if (cudaFuncSetAttribute(gemm_nvfp4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)gm::SMEM_BYTES) != cudaSuccess ||
+            cudaFuncSetAttribute(quantize_act_nvfp4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 227 * 1024) != cudaSuccess ||
+            int4_prepare_device() != cudaSuccess)
+            return cuda_fail();
+        g_device_ready[dev] = true;
+    }
+    return SVDQ_OK;
+}
+
+// ------------------------------------------------------------ tensor maps
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+        else
+            cudaGetLastError();
+    });
+    return fn;
+}
+
+// 2-D row-major tensor [outer, inner] with 128-byte swizzled boxes.
+bool make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
+              uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {inner, outer};
+    const cuuint64_t strides[1] = {row_bytes};
+    const cuuint32_t box[2] = {box_inner, box_outer};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int g_num_sms = 0;
+int num_sms() {
+    if (g_num_sms == 0) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev);
+        if (g_num_sms <= 0) g_num_sms = 148;
+    }
+    return g_num_sms;
+}
+
+// ---------------------------------------------------------- nvfp4 paths
+svdq_status tensor_scale_prepass(const void* src, const float* inv_lambda, int64_t rows, int64_t K, float* out,
+                                 cudaStream_t st) {
+    if (cudaMemsetAsync(out, 0, sizeof(float), st) != cudaSuccess) return cuda_fail();
+    const int64_t nvec = rows * K / 8;
+    const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>((nvec + 255) / 256, 8LL * num_sms()));
+    amax_kernel<<<blocks, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(src), inv_lambda, rows, K,
+                                        reinterpret_cast<unsigned int*>(out));
+    finalize_tensor_scale_kernel<<<1, 1, 0, st>>>(out);
+    return cudaGetLastError() == cudaSuccess ? SVDQ_OK : SVDQ_ERR_CUDA;
+}
+
+svdq_status fold_lowrank(const float* lambda, const void* L_down, const void* L_up, int64_t N, int64_t K, int rank,
+                         float* inv_lambda, void* L_down_t, void* L_up_t, cudaStream_t st) {
+    const int64_t work = std::max<int64_t>(K, std::max<int64_t>(K * rank, N * rank));
+    const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>((work + 255) / 256, 8LL * num_sms()));
+    fold_lowrank_kernel<<<blocks, 256, 0, st>>>(lambda, reinterpret_cast<const __nv_bfloat16*>(L_down),
+                                                reinterpret_cast<const __nv_bfloat16*>(L_up), K, N, rank, inv_lambda,
+                                                reinterpret_cast<__nv_bfloat16*>(L_down_t),
+                                                reinterpret_cast<__nv_bfloat16*>(L_up_t));
+    return cudaGetLastError() == cudaSuccess ? SVDQ_OK : SVDQ_ERR_CUDA;
+}
+
+svdq_status pack_weight_nvfp4(const void* R, int64_t N, int64_t K, void* w_codes, void* w_scales,
+                              float* w_tensor_scale, cudaStream_t st) {
+    SVDQ_TRY(tensor_scale_prepass(R, nullptr, N, K, w_tensor_scale, st));
+    const int64_t rows_pad = round_up(N, 128);
+    const int64_t work = rows_pad * (K / 16);
+    quantize_rows_nvfp4_kernel<<<(unsigned)((work + 255) / 256), 256, 0, st>>>(
+        reinterpret_cast<const __nv_bfloat16*>(R), N, rows_pad, K, w_tensor_scale,
+        reinterpret_cast<uint8_t*>(w_codes), reinterpret_cast<uint8_t*>(w_scales));
+    return cudaGetLastError() == cudaSuccess ? SVDQ_OK : SVDQ_ERR_CUDA;
+}
+
+// Cluster width for the activation quantizer: enough CTAs to cover the SMs
+// in one wave, a power of two dividing 128 (rows are split evenly for the
+// reduction), at most 8 (portable) and at most the number of column chunks.
+int choose_cluster(int64_t row_blocks, int chunks, int smem_bytes) {
+    int c = 1;
+    while (c < 8 && row_blocks * (c * 2) <= num_sms() && c * 2 <= chunks) c *= 2;
+    // make sure that many clusters can be resident at once; shrink otherwise
+    while (c > 1) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)c, (unsigned)row_blocks, 1);
+        cfg.blockDim = dim3(qa::kThreads, 1, 1);
+        cfg.dynamicSmemBytes = (size_t)smem_bytes;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = (unsigned)c;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int nclusters = 0;
+        if (cudaOccupancyMaxActiveClusters(&nclusters, quantize_act_nvfp4_kernel, &cfg) != cudaSuccess) {
+            cudaGetLastError();
+            nclusters = 0;
+        }
+        if ((int64_t)nclusters >= row_blocks) break;
+        c /= 2;
+    }
+    return c;
+}
+
+svdq_status quantize_act_nvfp4(const void* x, int64_t M, int64_t K, const float* inv_lambda, float* x_scale,
+                               int compute_scale, const float* w_scale, const void* L_down_t, int rank,
+                               void* x_codes, void* x_scales, void* lowrank, cudaStream_t st) {
+    if (compute_scale) SVDQ_TRY(tensor_scale_prepass(x, inv_lambda, M, K, x_scale, st));
+    CUtensorMap tm_x, tm_ld;
+    if (!make_map(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, 64, 128))
+        return SVDQ_ERR_CUDA;
+    if (rank > 0) {
+        if (!make_map(&tm_ld, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L_down_t, (uint64_t)K, (uint64_t)rank,
+                      (uint64_t)K * 2, 64, (uint32_t)rank))
+            return SVDQ_ERR_CUDA;
+    } else {
+        tm_ld = tm_x;
+    }
+    QuantActArgs a;
+    a.inv_lambda = inv_lambda;
+    a.x_scale = x_scale;
+    a.w_scale = w_scale;
+    a.x_codes = reinterpret_cast<uint8_t*>(x_codes);
+    a.x_scales = reinterpret_cast<uint8_t*>(x_scales);
+    a.lowrank = reinterpret_cast<__nv_bfloat16*>(lowrank);
+    a.M = (int)M;
+    a.K = (int)K;
+    a.rank = rank;
+    a.chunks = (int)(K / 64);
+    const uint32_t ld_pad = (uint32_t)round_up((int64_t)rank * 128, 1024);
+    a.stage_bytes = (uint32_t)qa::kXBytes + ld_pad;
+    const size_t fixed = 1024 + qa::kMaxStages * qa::kCols * 4 + (2 * qa::kMaxStages + 1) * 8 + 16;
+    int stages = (int)std::min<size_t>(qa::kMaxStages, (226 * 1024 - fixed) / a.stage_bytes);
+    const size_t red_bytes = (size_t)qa::kRows * (rank + 1) * 4;
+    if (stages < 2 || (size_t)stages * a.stage_bytes < red_bytes) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+    a.stages = stages;
+    uint32_t tcols = 32;
+    while ((int)tcols < rank) tcols *= 2;
+    a.tmem_cols = tcols;
+    const size_t smem = fixed + (size_t)stages * a.stage_bytes;
+    const int64_t row_blocks = (M + qa::kRows - 1) / qa::kRows;
+    if (row_blocks > 65535) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+    a.cluster = choose_cluster(row_blocks, a.chunks, (int)smem);
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)a.cluster, (unsigned)row_blocks, 1);
+    cfg.blockDim = dim3(qa::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)a.cluster;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, quantize_act_nvfp4_kernel, tm_x, tm_ld, a) != cudaSuccess) return cuda_fail();
+    return SVDQ_OK;
+}
+
+svdq_status gemm_nvfp4(const void* x_codes, const void* x_scales, const float* x_scale, int64_t M,
+                       const void* w_codes, const void* w_scales, const float* w_scale, int64_t N, int64_t K,
+                       const void* lowrank, const void* L_up_t, int rank, const void* bias, void* y, cudaStream_t st) {
+    CUtensorMap tm_xc, tm_wc, tm_L, tm_Lup;
+    if (!make_map(&tm_xc, CU_TENSOR_MAP_DATA_TYPE_UINT8, x_codes, (uint64_t)K / 2, (uint64_t)M, (uint64_t)K / 2,
+                  gm::BK_BYTES, gm::BM) ||
+        !make_map(&tm_wc, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_codes, (uint64_t)K / 2, (uint64_t)N, (uint64_t)K / 2,
+                  gm::BK_BYTES, gm::BN))
+        return SVDQ_ERR_CUDA;
+    if (rank > 0) {
+        if (!make_map(&tm_L, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, lowrank, (uint64_t)rank, (uint64_t)M,
+                      (uint64_t)rank * 2, 64, gm::BM) ||
+            !make_map(&tm_Lup, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L_up_t, (uint64_t)rank, (uint64_t)N,
+                      (uint64_t)rank * 2, 64, gm::BN))
+            return SVDQ_ERR_CUDA;
+    } else {
+        tm_L = tm_xc;
+        tm_Lup = tm_wc;
+    }
+    GemmArgs a;
+    a.x_scales = reinterpret_cast<const uint8_t*>(x_scales);
+    a.w_scales = reinterpret_cast<const uint8_t*>(w_scales);
+    a.x_scale = x_scale;
+    a.w_scale = w_scale;
+    a.bias = reinterpret_cast<const __nv_bfloat16*>(bias);
+    a.y = reinterpret_cast<__nv_bfloat16*>(y);
+    a.M = (int)M;
+    a.N = (int)N;
+    a.K = (int)K;
+    a.rank = rank;
+    a.kg4 = (int)(K / 64);
+    a.n_sf_blocks = (int)((N + 127) / 128);
+    const int64_t mt = (M + gm::BM - 1) / gm::BM, nt = (N + gm::BN - 1) / gm::BN;
+    if (nt > 65535) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+    gemm_nvfp4_kernel<<<dim3((unsigned)mt, (unsigned)nt, 1), gm::kThreads, gm::SMEM_BYTES, st>>>(tm_xc, tm_wc, tm_L,
+                                                                                             tm_Lup, a);
+    return cudaGetLastError() == cudaSuccess ? SVDQ_OK : SVDQ_ERR_CUDA;
+}
+
+// Kernel that waits on a barrier nobody completes: exercises the bounded wait.
+__global__ void timeout_probe_kernel() {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) mbar_wait(&bar, 0, 0xEE);
+    __syncthreads();
+}
+
+}  // namespace
+}  // namespace svdq
+
+using namespace svdq;
+
+extern "C" {
+
+const char* svdq_status_string(svdq_status s) {
+    switch (s) {
+        case SVDQ_OK: return "ok";
+        case SVDQ_ERR_INVALID_ARG: return "invalid argument";
+        case SVDQ_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+        case SVDQ_ERR_UNSUPPORTED_DEVICE: return "unsupported device (needs compute capability 10.0, sm_100a)";
+        case SVDQ_ERR_CUDA: return "CUDA error";
+        case SVDQ_ERR_TIMEOUT: return "a kernel timed out waiting on a barrier";
+    }
+    return "unknown status";
+}
+
+int svdq_abi_version(void) { return kAbiVersion; }
+
+svdq_status svdq_buffer_sizes(svdq_precision p, int64_t rows, int64_t K, int rank, svdq_sizes* out) {
+    if (!out) return SVDQ_ERR_INVALID_ARG;
+    if (p != SVDQ_NVFP4 && p != SVDQ_INT4) return SVDQ_ERR_INVALID_ARG;
+    SVDQ_TRY(check_rank(rank));
+    SVDQ_TRY(check_dims(rows, K));
+    const int64_t rows_pad = round_up(rows, 128);
+    out->codes_bytes = (size_t)(rows * K / 2);
+    out->scales_bytes = p == SVDQ_NVFP4 ? (size_t)(rows_pad * K / 16) : (size_t)(2 * rows_pad * K / 64);
+    out->lowrank_bytes = (size_t)(2 * rows * rank);
+    return SVDQ_OK;
+}
+
+svdq_status svdq_pack_weight(svdq_precision p, int group_size, const void* R, int64_t N, int64_t K,
+                             const float* lambda, const void* L_down, const void* L_up, int rank, void* w_codes,
+                             void* w_scales, float* w_tensor_scale, float* inv_lambda, void* L_down_t, void* L_up_t,
+                             svdq_stream_t stream) {
+    SVDQ_TRY(check_precision(p, group_size));
+    SVDQ_TRY(check_rank(rank));
+    SVDQ_TRY(check_dims(N, K));
+    if (N % 16 != 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+    SVDQ_TRY(check_ptr(R));
+    SVDQ_TRY(check_ptr(lambda));
+    SVDQ_TRY(check_ptr(w_codes));
+    SVDQ_TRY(check_ptr(w_scales));
+    SVDQ_TRY(check_ptr(inv_lambda));
+    if (p == SVDQ_NVFP4) SVDQ_TRY(check_ptr(w_tensor_scale));
+    if (rank > 0) {
+        SVDQ_TRY(check_ptr(L_down));
+        SVDQ_TRY(check_ptr(L_up));
+        SVDQ_TRY(check_ptr(L_down_t));
+        SVDQ_TRY(check_ptr(L_up_t));
+    }
+    SVDQ_TRY(check_device());
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    SVDQ_TRY(fold_lowrank(lambda, L_down, L_up, N, K, rank, inv_lambda, L_down_t, L_up_t, st));
+    if (p == SVDQ_NVFP4) return pack_weight_nvfp4(R, N, K, w_codes, w_scales, w_tensor_scale, st);
+    return int4_quantize_rows(R, nullptr, N, K, w_codes, w_scales, st);
+}
+
+svdq_status svdq_quantize_act(svdq_precision p, int group_size, const void* x, int64_t M, int64_t K,
+                              const float* inv_lambda, float* x_tensor_scale, int compute_scale,
+                              const float* w_tensor_scale, const void* L_down_t, int rank, void* x_codes,
+                              void* x_scales, void* lowrank_act, svdq_stream_t stream) {
+    SVDQ_TRY(check_precision(p, group_size));
+    SVDQ_TRY(check_rank(rank));
+    SVDQ_TRY(check_dims(M, K));
+    SVDQ_TRY(check_ptr(x));
+    SVDQ_TRY(check_ptr(inv_lambda));
+    SVDQ_TRY(check_ptr(x_codes));
+    SVDQ_TRY(check_ptr(x_scales));
+    if (p == SVDQ_NVFP4) SVDQ_TRY(check_ptr(x_tensor_scale));
+    if (rank > 0) {
+        SVDQ_TRY(check_ptr(L_down_t));
+        SVDQ_TRY(check_ptr(lowrank_act));
+        if (p == SVDQ_NVFP4) SVDQ_TRY(check_ptr(w_tensor_scale));
+    }
+    SVDQ_TRY(check_device());
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (p == SVDQ_NVFP4)
+        return quantize_act_nvfp4(x, M, K, inv_lambda, x_tensor_scale, compute_scale, w_tensor_scale, L_down_t, rank,
+                                  x_codes, x_scales, lowrank_act, st);
+    return int4_quantize_act(x, M, K, inv_lambda, L_down_t, rank, x_codes, x_scales, lowrank_act, st);
+}
+
+svdq_status svdq_gemm_w4a4(svdq_precision p, int group_size, const void* x_codes, const void* x_scales,
+                           const float* x_tensor_scale, int64_t M, const void* w_codes, const void* w_scales,
+                           const float* w_tensor_scale, int64_t N, int64_t K, const void* lowrank_act,
+                           const void* L_up_t, int rank, const void* bias, void* y, svdq_stream_t stream) {
+    SVDQ_TRY(check_precision(p, group_size));
+    SVDQ_TRY(check_rank(rank));
+    SVDQ_TRY(check_dims(M, K));
+    SVDQ_TRY(check_dims(N, K));
+    if (N % 16 != 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+    SVDQ_TRY(check_ptr(x_codes));
+    SVDQ_TRY(check_ptr(x_scales));
+    SVDQ_TRY(check_ptr(w_codes));
+    SVDQ_TRY(check_ptr(w_scales));
+    SVDQ_TRY(check_ptr(y));
+    SVDQ_TRY(check_opt_ptr(bias));
+    if (p == SVDQ_NVFP4) {
+        SVDQ_TRY(check_ptr(x_tensor_scale));
+        SVDQ_TRY(check_ptr(w_tensor_scale));
+    }
+    if (rank > 0) {
+        SVDQ_TRY(check_ptr(lowrank_act));
+        SVDQ_TRY(check_ptr(L_up_t));
+    }
+    SVDQ_TRY(check_device());
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (p == SVDQ_NVFP4)
+        return gemm_nvfp4(x_codes, x_scales, x_tensor_scale, M, w_codes, w_scales, w_tensor_scale, N, K, lowrank_act,
+                          L_up_t, rank, bias, y, st);
+    return int4_gemm(x_codes, x_scales, M, w_codes, w_scales, N, K, lowrank_act, L_up_t, rank, bias, y, st);
+}
+
+svdq_status svdq_device_status(int clear, int* site) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return SVDQ_ERR_UNSUPPORTED_DEVICE;
+    }
+    if (cudaDeviceSynchronize() != cudaSuccess) return cuda_fail();
+    unsigned int word = 0;
+    if (cudaMemcpyFromSymbol(&word, g_status_word, sizeof(word)) != cudaSuccess) return cuda_fail();
+    if (site) *site = (int)((word >> 8) & 0xFFu);
+    if (clear && word) {
+        const unsigned int zero = 0;
+        if (cudaMemcpyToSymbol(g_status_word, &zero, sizeof(zero)) != cudaSuccess) return cuda_fail();
+    }
+    return (word & 1u) ? SVDQ_ERR_TIMEOUT : SVDQ_OK;
+}
+
+svdq_status svdq_debug_set_wait_limit_ns(uint64_t ns) {
+    SVDQ_TRY(check_device());
+    const unsigned long long v = ns ? (unsigned long long)ns : 2000000000ull;
+    if (cudaMemcpyToSymbol(g_wait_limit_ns, &v, sizeof(v)) != cudaSuccess) return cuda_fail();
+    return SVDQ_OK;
+}
+
+svdq_status svdq_debug_timeout_probe(svdq_stream_t stream) {
+    SVDQ_TRY(check_device());
+    timeout_probe_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>();
+    return cudaGetLastError() == cudaSuccess ? SVDQ_OK : SVDQ_ERR_CUDA;
+}
+
+void svdq_debug_override_capability(int major, int minor) {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    g_override_major = major;
+    g_override_minor = minor;
+}
+
+}  // extern "C"

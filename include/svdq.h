@@ -1,0 +1,169 @@
+/*
+ * svdq.h -- C ABI of the B200 (sm_100a) SVDQuant W4A4 linear layer.
+ *
+ * The layer (the `svdq_w4a4` scheme of the Diffusers docs page "Nunchaku Lite",
+ * section "Supported quantization types": "NVFP4 runtime kernel with SVDQ
+ * low-rank correction", nvfp4 with group 16, or "INT4 W4A4 kernel with SVDQ
+ * low-rank correction", int4 with group 64; the SVDQuant paper linked from
+ * that page defines the split W . diag(lambda) = L_down . L_up + R):
+ *
+ *     y = dequant(Q4(x/lambda)) . dequant(Q4(R))^T + ((x/lambda) . L_down) . L_up + b
+ *
+ * A forward pass is two calls on one stream, with no host synchronisation:
+ *     svdq_quantize_act   x -> 4-bit codes + group scales (+ rank-r activations)
+ *     svdq_gemm_w4a4      block-scaled 4-bit GEMM + rank-r up-projection + bias
+ * The weight side is packed once, offline, by svdq_pack_weight.
+ *
+ * Conventions for every call below
+ *  - Pointers named "device" are device memory of the current CUDA device,
+ *    owned by the caller; the library allocates nothing and keeps no state
+ *    between calls (except the device status word, see svdq_device_status).
+ *  - All device pointers must be 16-byte aligned.
+ *  - bf16 tensors are row-major with the last dimension contiguous.
+ *  - Calls are asynchronous on `stream` (NULL = the legacy default stream).
+ *    Argument errors are returned before anything is launched; a failed
+ *    launch returns SVDQ_ERR_CUDA.  A kernel that waits on a barrier for
+ *    longer than the wait limit (2 s by default) abandons its work, records
+ *    the fact in the device status word, and returns; svdq_device_status()
+ *    reports it as SVDQ_ERR_TIMEOUT.
+ *  - Sizes: 1 <= M, N and K < 2^31; K % 64 == 0; N % 16 == 0;
+ *    rank in {0, 16, 32, ..., 256} (multiples of 16; 0 disables the branch).
+ *  - The device must be compute capability 10.0 (B200 class, sm_100a); any
+ *    other device is rejected with SVDQ_ERR_UNSUPPORTED_DEVICE before a
+ *    launch (the pages' load-time capability check: tutorial page, section
+ *    "3. Hardware notes").
+ *
+ * Packed layouts (owned by this library; svdq_buffer_sizes gives the bytes)
+ *  - codes:  [rows, K/2] bytes; element k of a row is in the low nibble of
+ *            byte k/2 when k is even, in the high nibble when k is odd.
+ *            nvfp4: FP4 E2M1 codes (bit 3 = sign).  int4: two's complement.
+ *  - nvfp4 scales: one UE4M3 byte per (row, group of 16), rows padded to a
+ *            multiple of 128 with zero bytes, in the tensor-core scale-factor
+ *            layout: with Kg4 = K/64, the byte of (row r, group g) is at
+ *              ((r/128)*Kg4 + g/4)*512 + (r%32)*16 + ((r%128)/32)*4 + g%4.
+ *  - int4 scales: one bf16 per (row, group of 64), group-major:
+ *            scales[g * rows_pad + r] with rows_pad = rows rounded up to 128
+ *            (padding rows are zero).
+ *  - tensor scale (nvfp4 only): one fp32 S; a value is code * scale * S.
+ *  - rank-r activations ("lowrank_act"): bf16 [M, rank].  nvfp4 stores
+ *            ((x/lambda) . L_down) / (S_x * S_w) so the GEMM can add it into the
+ *            unscaled FP4 accumulator; int4 stores (x/lambda) . L_down.
+ *  - folded weights: inv_lambda fp32 [K] = 1/lambda (IEEE round-to-nearest);
+ *            L_down_t bf16 [rank, K] = bf16(L_down[k,j] / lambda[k]) transposed;
+ *            L_up_t bf16 [N, rank] = L_up transposed.
+ */
+#ifndef SVDQ_H_
+#define SVDQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st* svdq_stream_t;
+
+typedef enum {
+    SVDQ_OK = 0,
+    SVDQ_ERR_INVALID_ARG = 1,        /* null pointer, misalignment, bad precision/group/rank */
+    SVDQ_ERR_UNSUPPORTED_SHAPE = 2,  /* sizes outside the limits above */
+    SVDQ_ERR_UNSUPPORTED_DEVICE = 3, /* no CUDA device, or not compute capability 10.0 */
+    SVDQ_ERR_CUDA = 4,               /* a CUDA runtime/driver call or launch failed */
+    SVDQ_ERR_TIMEOUT = 5             /* a kernel gave up waiting on a barrier */
+} svdq_status;
+
+typedef enum {
+    SVDQ_NVFP4 = 0, /* FP4 E2M1 codes, UE4M3 scale per 16, fp32 tensor scale */
+    SVDQ_INT4 = 1   /* signed int4 codes, bf16 scale per 64 */
+} svdq_precision;
+
+/* Byte sizes of the packed buffers for `rows` rows of K columns. */
+typedef struct {
+    size_t codes_bytes;    /* rows * K / 2 */
+    size_t scales_bytes;   /* nvfp4: rows_pad * K / 16;  int4: 2 * rows_pad * K / 64 */
+    size_t lowrank_bytes;  /* 2 * rows * rank (bf16 rank-r activations) */
+} svdq_sizes;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* svdq_status_string(svdq_status status);
+
+/* Version of this ABI (increments on any incompatible change). */
+int svdq_abi_version(void);
+
+/* Pure host function: fills *out for the given precision and sizes.
+ * Errors: INVALID_ARG (out NULL, unknown precision, bad rank),
+ *         UNSUPPORTED_SHAPE (rows < 1, K not a multiple of 64). */
+svdq_status svdq_buffer_sizes(svdq_precision precision, int64_t rows, int64_t K, int rank, svdq_sizes* out);
+
+/* Offline packing of the weight side (run once per layer).
+ *   R          device bf16 [N, K]    residual weight (out x in)
+ *   lambda     device fp32 [K]       smoothing divisors, > 0 and finite
+ *   L_down     device bf16 [K, rank] (may be NULL when rank == 0)
+ *   L_up       device bf16 [rank, N] (may be NULL when rank == 0)
+ * Outputs (device, caller-allocated):
+ *   w_codes [N, K/2]; w_scales (scales_bytes for N rows); w_tensor_scale fp32[1]
+ *   (nvfp4: S_w = amax|R| / 2688, or 1 when R == 0; int4: may be NULL);
+ *   inv_lambda fp32 [K]; L_down_t bf16 [rank, K]; L_up_t bf16 [N, rank].
+ * group_size must be 16 for SVDQ_NVFP4 and 64 for SVDQ_INT4. */
+svdq_status svdq_pack_weight(svdq_precision precision, int group_size,
+                             const void* R, int64_t N, int64_t K,
+                             const float* lambda, const void* L_down, const void* L_up, int rank,
+                             void* w_codes, void* w_scales, float* w_tensor_scale,
+                             float* inv_lambda, void* L_down_t, void* L_up_t,
+                             svdq_stream_t stream);
+
+/* Activation quantizer, fused with the rank-r down-projection.
+ *   x              device bf16 [M, K]
+ *   inv_lambda     device fp32 [K] (from svdq_pack_weight)
+ *   x_tensor_scale device fp32 [1] (nvfp4 only): read as S_x when
+ *                  compute_scale == 0 (must be > 0 and finite); when
+ *                  compute_scale != 0 it is overwritten with
+ *                  S_x = amax|x/lambda| / 2688 (1 when x == 0) first.
+ *   w_tensor_scale device fp32 [1] (nvfp4 with rank > 0): S_w
+ *   L_down_t       device bf16 [rank, K] (NULL when rank == 0)
+ * Outputs: x_codes [M, K/2]; x_scales (scales_bytes for M rows, padding rows
+ *   written as zeros); lowrank_act bf16 [M, rank] (NULL when rank == 0). */
+svdq_status svdq_quantize_act(svdq_precision precision, int group_size,
+                              const void* x, int64_t M, int64_t K, const float* inv_lambda,
+                              float* x_tensor_scale, int compute_scale,
+                              const float* w_tensor_scale, const void* L_down_t, int rank,
+                              void* x_codes, void* x_scales, void* lowrank_act,
+                              svdq_stream_t stream);
+
+/* The W4A4 GEMM with the rank-r up-projection and bias fused in.
+ *   y[m, n] = bf16( S_x S_w sum_k xq[m,k] wq[n,k] + sum_j L[m,j] L_up[j,n] + b[n] )   (nvfp4)
+ *   y[m, n] = bf16( sum_g sx[m,g] sw[n,g] sum_{k in g} qx qw + sum_j L[m,j] L_up[j,n] + b[n] )  (int4)
+ * Inputs are the outputs of the two calls above; bias is device bf16 [N] or
+ * NULL; lowrank_act / L_up_t may be NULL when rank == 0.
+ * Output: y device bf16 [M, N]. */
+svdq_status svdq_gemm_w4a4(svdq_precision precision, int group_size,
+                           const void* x_codes, const void* x_scales, const float* x_tensor_scale, int64_t M,
+                           const void* w_codes, const void* w_scales, const float* w_tensor_scale,
+                           int64_t N, int64_t K,
+                           const void* lowrank_act, const void* L_up_t, int rank,
+                           const void* bias, void* y, svdq_stream_t stream);
+
+/* Synchronises the current device, then reads the device status word.
+ * Returns SVDQ_OK, SVDQ_ERR_TIMEOUT (a kernel abandoned a wait; *site, if not
+ * NULL, receives the id of the first wait that did) or SVDQ_ERR_CUDA.
+ * clear != 0 resets the word afterwards. */
+svdq_status svdq_device_status(int clear, int* site);
+
+/* Test hooks (not for production use).
+ *  svdq_debug_set_wait_limit_ns: changes the barrier wait limit (0 restores 2 s).
+ *  svdq_debug_timeout_probe: launches one small kernel that waits on a barrier
+ *    nothing ever completes, so it must give up after the wait limit; the
+ *    status word then reads SVDQ_ERR_TIMEOUT.  Used to test failure detection.
+ *  svdq_debug_override_capability: pretend the device has compute capability
+ *    major.minor (major = -1 removes the override), to test the device check. */
+svdq_status svdq_debug_set_wait_limit_ns(uint64_t ns);
+svdq_status svdq_debug_timeout_probe(svdq_stream_t stream);
+void svdq_debug_override_capability(int major, int minor);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SVDQ_H_ */
