@@ -28,7 +28,7 @@ GROUP_SIZES = {"nvfp4": 16, "int4": 64}
 
 # Every entry point declared in include/svdq.h.
 EXPORTS = (
-    "svdq_status_string", "svdq_abi_version", "svdq_buffer_sizes", "svdq_pack_weight",
+    "svdq_status_string", "svdq_abi_version", "svdq_last_error", "svdq_buffer_sizes", "svdq_pack_weight",
     "svdq_quantize_act", "svdq_gemm_w4a4", "svdq_device_status",
     "svdq_debug_set_wait_limit_ns", "svdq_debug_timeout_probe", "svdq_debug_override_capability",
 )
@@ -37,7 +37,10 @@ EXPORTS = (
 class SvdqError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
-        super().__init__(f"{where}: {status_string(status)} (status {status})")
+        detail = ""
+        if status == SVDQ_ERR_CUDA:
+            detail = f" [{lib.svdq_last_error().decode()}]"
+        super().__init__(f"{where}: {status_string(status)} (status {status}){detail}")
 
 
 class svdq_sizes(ctypes.Structure):
@@ -55,6 +58,8 @@ def _load():
     lib.svdq_status_string.restype = ctypes.c_char_p
     lib.svdq_abi_version.argtypes = []
     lib.svdq_abi_version.restype = I
+    lib.svdq_last_error.argtypes = []
+    lib.svdq_last_error.restype = ctypes.c_char_p
     lib.svdq_buffer_sizes.argtypes = [I, I64, I64, I, ctypes.POINTER(svdq_sizes)]
     lib.svdq_buffer_sizes.restype = I
     lib.svdq_pack_weight.argtypes = [I, I, P, I64, I64, P, P, P, I, P, P, P, P, P, P, P]

@@ -1,7 +1,8 @@
 // gemm_nvfp4.cuh -- block-scaled FP4 GEMM of the SVDQ W4A4 layer (sm_100a).
 //
 //   acc[m, n]  = sum_k (q_x[m,k] e_x[m,k/16]) (q_w[n,k] e_w[n,k/16])   FP4 x FP4, fp32 in TMEM
-//   acc[m, n] += sum_j L'[m, j] L_up[j, n]       rank-r branch, bf16 MMA into the same accumulator
+//   acc[m, n] += sum_j L'[m, j] L_up[j, n]       rank-r branch: bf16 MMAs of the hi and lo
+//                                                parts of L' into the same accumulator
 //   y[m, n]    = bf16( S_x S_w acc[m, n] + b[n] )
 // where L' = ((x/lambda) . L_down) / (S_x S_w) comes from the quantizer.  The
 // "NVFP4 runtime kernel with SVDQ low-rank correction" of the Diffusers docs
@@ -65,7 +66,7 @@ __global__ void __launch_bounds__(gm::kThreads, 1)
     const int m_tile = blockIdx.x, n_tile = blockIdx.y;
     const int m0 = m_tile * BM, n0 = n_tile * BN;
     const int n_kb = (a.K + 255) / 256;
-    const int n_lr = a.rank > 0 ? (a.rank + 63) / 64 : 0;
+    const int n_lr = a.rank > 0 ? 2 * ((a.rank + 63) / 64) : 0;   // hi and lo part of each 64-column chunk
     const int total = n_kb + n_lr;
 
     if (threadIdx.x == 0) {
@@ -125,9 +126,9 @@ __global__ void __launch_bounds__(gm::kThreads, 1)
                         bulk_load(sfb + rb * 2048, a.w_scales + ((int64_t)(nb0 + rb) * a.kg4 + 4 * kb) * 512,
                                   sf_bytes, &full[s]);
                 } else {
-                    const int c = it - n_kb;
+                    const int c = (it - n_kb) >> 1, part = (it - n_kb) & 1;
                     mbar_arrive_expect_tx(&full[s], A_BYTES + B_BYTES);
-                    tma_load_2d(sa, &tm_L, &full[s], c * 64, m0);
+                    tma_load_3d(sa, &tm_L, &full[s], c * 64, m0, part);
                     tma_load_2d(sb, &tm_Lup, &full[s], c * 64, n0);
                 }
             }
@@ -164,7 +165,7 @@ __global__ void __launch_bounds__(gm::kThreads, 1)
                         mma_nvfp4(tmem + ACC_COL, desc_sw128(sa + 32u * j), desc_sw128(sb + 32u * j), idesc_fp4,
                                   tmem + SFA_COL + 4u * j, tmem + SFB_COL + 8u * j, (it > 0 || j > 0) ? 1u : 0u);
                 } else {
-                    const int c = it - n_kb;
+                    const int c = (it - n_kb) >> 1;
                     const int nks = min(4, (a.rank - 64 * c + 15) / 16);
                     for (int j = 0; j < nks; ++j)
                         mma_bf16(tmem + ACC_COL, desc_sw128(sa + 32u * j), desc_sw128(sb + 32u * j), idesc_lr, 1u);

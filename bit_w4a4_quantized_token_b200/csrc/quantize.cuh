@@ -1,11 +1,11 @@
-// quant_nvfp4.cuh -- NVFP4 quantizers of the SVDQ W4A4 layer (sm_100a).
+// quantize.cuh -- the quantizers of the SVDQ W4A4 layer (sm_100a).
 //
-//  * the tensor-scale pre-pass (amax, then S = amax / 2688),
-//  * the weight packer (R -> E2M1 codes + UE4M3 group scales; 1/lambda folded
-//    into L_down, L_up transposed),
+//  * the NVFP4 tensor-scale pre-pass (amax, then S = amax / 2688),
+//  * the weight packer (R -> 4-bit codes + group scales; 1/lambda folded into
+//    L_down as an fp32 value carried by a bf16 hi/lo pair, L_up transposed),
 //  * the activation quantizer fused with the rank-r down-projection
 //    (x/lambda -> codes + scales, and (x/lambda) . L_down on the tensor cores
-//    from the same shared-memory tile).
+//    from the same shared-memory tile), for nvfp4 and int4.
 //
 // Group rule (Diffusers docs "Nunchaku Lite", "Supported quantization types":
 // nvfp4, group 16): for a group of 16 smoothed values v with a = max|v|,
@@ -42,6 +42,37 @@ __device__ __forceinline__ uint32_t quant_group16(const float (&v)[16], float S,
     for (int i = 0; i < 8; ++i) q[i] = __fmul_rn(v[8 + i], inv);
     hi = cvt_e2m1x8(q);
     return eb;
+}
+
+// Splits v into hi = bf16(v) and lo = bf16(v - hi): hi + lo carries v to
+// about 2^-17 relative, so two bf16 MMAs reproduce an fp32 operand.
+__device__ __forceinline__ void split_bf16(float v, __nv_bfloat16& hi, __nv_bfloat16& lo) {
+    hi = __float2bfloat16_rn(v);
+    lo = __float2bfloat16_rn(__fsub_rn(v, __bfloat162float(hi)));
+}
+
+// int4 group of 64 (Diffusers docs "Nunchaku Lite", "Supported quantization
+// types": int4, group 64): s = bf16(a / 7), q = clamp(rint(v * (1/s)), -8, 7).
+// Returns the bf16 scale bits; codes as eight words of two's-complement nibbles.
+__device__ __forceinline__ uint32_t quant_group64_int4(const float (&v)[64], uint32_t (&cw)[8]) {
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 64; ++i) amax = fmaxf(amax, fabsf(v[i]));
+    const __nv_bfloat16 sb = __float2bfloat16_rn(__fdiv_rn(amax, 7.0f));
+    const float sf = __bfloat162float(sb);
+    const float inv = (sf == 0.0f) ? 0.0f : __frcp_rn(sf);
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+        uint32_t word = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            int q = __float2int_rn(__fmul_rn(v[8 * w + i], inv));
+            q = max(-8, min(7, q));
+            word |= ((uint32_t)q & 15u) << (4 * i);
+        }
+        cw[w] = word;
+    }
+    return (uint32_t)__bfloat16_as_ushort(sb);
 }
 
 // ---------------------------------------------------------------- pre-pass
@@ -119,7 +150,41 @@ __global__ void __launch_bounds__(256) quantize_rows_nvfp4_kernel(const __nv_bfl
     scales[sf_offset(r, g, K / 64)] = (uint8_t)eb;
 }
 
-// inv_lambda = 1/lambda; L_down_t[j, k] = bf16(L_down[k, j] / lambda[k]);
+// int4 weight packing: one thread per (row, group of 64) over rows_pad rows;
+// the bf16 scales are group-major (scales[g * rows_pad + r]).
+__global__ void __launch_bounds__(256) quantize_rows_int4_kernel(const __nv_bfloat16* __restrict__ R, int64_t rows,
+                                                                 int64_t rows_pad, int64_t K,
+                                                                 uint8_t* __restrict__ codes,
+                                                                 uint16_t* __restrict__ scales) {
+    const int64_t kg = K / 64;
+    const int64_t gid = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    if (gid >= rows_pad * kg) return;
+    const int64_t r = gid % rows_pad, g = gid / rows_pad;   // consecutive threads: consecutive rows
+    uint32_t sb = 0;
+    if (r < rows) {
+        const uint4* src = reinterpret_cast<const uint4*>(R + r * K + g * 64);
+        float v[64];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const uint4 w = __ldg(src + c);
+            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+                v[8 * c + 2 * p] = bf16lo_to_f32(ws[p]);
+                v[8 * c + 2 * p + 1] = bf16hi_to_f32(ws[p]);
+            }
+        }
+        uint32_t cw[8];
+        sb = quant_group64_int4(v, cw);
+        uint4* dst = reinterpret_cast<uint4*>(codes + r * (K / 2) + g * 32);
+        dst[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+        dst[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+    }
+    scales[g * rows_pad + r] = (uint16_t)sb;
+}
+
+// inv_lambda = 1/lambda; with v = fl32(L_down[k, j] / lambda[k]):
+// L_down_t[0, j, k] = bf16(v) and L_down_t[1, j, k] = bf16(v - bf16(v));
 // L_up_t[n, j] = L_up[j, n].
 __global__ void __launch_bounds__(256) fold_lowrank_kernel(const float* __restrict__ lambda,
                                                            const __nv_bfloat16* __restrict__ L_down,
@@ -132,8 +197,10 @@ __global__ void __launch_bounds__(256) fold_lowrank_kernel(const float* __restri
     for (int64_t k = t0; k < K; k += stride) inv_lambda[k] = __frcp_rn(lambda[k]);
     for (int64_t i = t0; i < K * rank; i += stride) {  // i = j * K + k (coalesced stores)
         const int64_t j = i / K, k = i % K;
-        const float v = __bfloat162float(L_down[k * rank + j]);
-        L_down_t[i] = __float2bfloat16_rn(__fdiv_rn(v, lambda[k]));
+        const float v = __fdiv_rn(__bfloat162float(L_down[k * rank + j]), lambda[k]);
+        const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+        L_down_t[i] = hi;
+        L_down_t[K * rank + i] = __float2bfloat16_rn(__fsub_rn(v, __bfloat162float(hi)));
     }
     for (int64_t i = t0; i < N * rank; i += stride) {  // i = n * rank + j
         const int64_t n = i / rank, j = i % rank;
@@ -152,18 +219,20 @@ constexpr int kMaxStages = 8;
 
 struct QuantActArgs {
     const float* inv_lambda;   // [K]
-    const float* x_scale;      // S_x
-    const float* w_scale;      // S_w (rank > 0)
+    const float* x_scale;      // S_x (nvfp4)
+    const float* w_scale;      // S_w (nvfp4 with rank > 0)
     uint8_t* x_codes;          // [M, K/2]
-    uint8_t* x_scales;         // scale layout
-    __nv_bfloat16* lowrank;    // [M, rank]
+    uint8_t* x_scales;         // nvfp4: scale-factor layout; int4: bf16 [K/64, rows_pad]
+    __nv_bfloat16* lowrank;    // [2, M, rank]: hi and lo bf16 parts
     int M, K, rank;
+    int rows_pad;              // M rounded up to 128
     int chunks;                // K / 64
     int cluster;               // CTAs of one cluster split K for one 128-row block
     int stages;
-    uint32_t stage_bytes;      // 16 KB x tile + L_down_t tile (rank x 128 B, padded to 1 KB)
+    uint32_t stage_bytes;      // 16 KB x tile + two L_down_t tiles (hi, lo: rank x 128 B each)
     uint32_t tmem_cols;
 };
+
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {
     uint32_t r;
@@ -186,13 +255,18 @@ __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
 
 enum : uint32_t { kSiteQaEmpty = 1, kSiteQaFullMma = 2, kSiteQaFullWork = 3, kSiteQaAcc = 4, kSiteQaDrain = 5 };
 
+constexpr int kPrecNvfp4 = 0, kPrecInt4 = 1;
+
 // Grid (cluster, ceil(M/128)); cluster dims (cluster, 1, 1).  CTA `q` of a
 // cluster handles chunks [q*T/c, (q+1)*T/c) of the T = K/64 column chunks of
 // its 128-row block; the clusters' partial rank-r sums are reduced through
-// distributed shared memory in a fixed order (deterministic).
+// distributed shared memory in a fixed order (deterministic).  The rank-r
+// down-projection runs on the tensor cores: x (bf16, exact) times the hi and
+// lo bf16 parts of L_down / lambda, fp32 accumulate in TMEM.
+template <int PREC>
 __global__ void __launch_bounds__(qa::kThreads, 1)
-    quantize_act_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_ld,
-                              QuantActArgs a) {
+    quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_ld,
+                        QuantActArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int nst = a.stages;
@@ -237,7 +311,8 @@ __global__ void __launch_bounds__(qa::kThreads, 1)
     if (warp == 0) {
         // ---------------------------------------------------------- producer
         if (lane == 0) {
-            const uint32_t bytes = qa::kXBytes + (has_lr ? (uint32_t)a.rank * 128u : 0u) + qa::kCols * 4u;
+            const uint32_t ld_tile = (uint32_t)a.rank * 128u;
+            const uint32_t bytes = qa::kXBytes + (has_lr ? 2u * ld_tile : 0u) + qa::kCols * 4u;
             int it = 0;
             for (; it < n_it; ++it) {
                 const int s = it % nst;
@@ -250,7 +325,10 @@ __global__ void __launch_bounds__(qa::kThreads, 1)
                 uint8_t* st = smem + (size_t)s * a.stage_bytes;
                 mbar_arrive_expect_tx(&full[s], bytes);
                 tma_load_2d(st, &tm_x, &full[s], kc * qa::kCols, m0);
-                if (has_lr) tma_load_2d(st + qa::kXBytes, &tm_ld, &full[s], kc * qa::kCols, 0);
+                if (has_lr) {
+                    tma_load_3d(st + qa::kXBytes, &tm_ld, &full[s], kc * qa::kCols, 0, 0);
+                    tma_load_3d(st + qa::kXBytes + ld_tile, &tm_ld, &full[s], kc * qa::kCols, 0, 1);
+                }
                 bulk_load(invl + s * qa::kCols, a.inv_lambda + (int64_t)kc * qa::kCols, qa::kCols * 4, &full[s]);
             }
             s_issued = it;
@@ -272,9 +350,12 @@ __global__ void __launch_bounds__(qa::kThreads, 1)
                 const uint32_t xa = smem_u32(smem + (size_t)s * a.stage_bytes);
                 const uint32_t lb = xa + qa::kXBytes;
 #pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    mma_bf16(tmem, desc_sw128(xa + 32u * j), desc_sw128(lb + 32u * j), idesc,
-                             (it > 0 || j > 0) ? 1u : 0u);
+                for (int part = 0; part < 2; ++part)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        mma_bf16(tmem, desc_sw128(xa + 32u * j),
+                                 desc_sw128(lb + (uint32_t)part * (uint32_t)a.rank * 128u + 32u * j), idesc,
+                                 (it > 0 || part > 0 || j > 0) ? 1u : 0u);
                 tc_commit(&empty[s]);
             }
             if (ok) tc_commit(accb);
@@ -284,8 +365,11 @@ __global__ void __launch_bounds__(qa::kThreads, 1)
         const uint32_t q = warp & 3u;
         const int row = (int)(32u * q + lane);
         const int64_t grow = (int64_t)m0 + row;
-        const float S = *a.x_scale;
-        const float six_s = __fmul_rn(6.0f, S);
+        float S = 1.0f, six_s = 6.0f;
+        if (PREC == kPrecNvfp4) {
+            S = *a.x_scale;
+            six_s = __fmul_rn(6.0f, S);
+        }
         bool ok = true;
         for (int it = 0; it < n_it; ++it) {
             const int s = it % nst;
@@ -299,41 +383,46 @@ __global__ void __launch_bounds__(qa::kThreads, 1)
             uint4 raw[8];
 #pragma unroll
             for (int c = 0; c < 8; ++c) raw[c] = *reinterpret_cast<const uint4*>(xr + ((c ^ (row & 7)) << 4));
-            float il[64];
+            float v[64];
             const float4* ilp = reinterpret_cast<const float4*>(invl + s * qa::kCols);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const float4 t = ilp[i];
-                il[4 * i] = t.x;
-                il[4 * i + 1] = t.y;
-                il[4 * i + 2] = t.z;
-                il[4 * i + 3] = t.w;
+            for (int c = 0; c < 8; ++c) {
+                const float4 l0 = ilp[2 * c], l1 = ilp[2 * c + 1];
+                const uint32_t ws[4] = {raw[c].x, raw[c].y, raw[c].z, raw[c].w};
+                v[8 * c + 0] = __fmul_rn(bf16lo_to_f32(ws[0]), l0.x);
+                v[8 * c + 1] = __fmul_rn(bf16hi_to_f32(ws[0]), l0.y);
+                v[8 * c + 2] = __fmul_rn(bf16lo_to_f32(ws[1]), l0.z);
+                v[8 * c + 3] = __fmul_rn(bf16hi_to_f32(ws[1]), l0.w);
+                v[8 * c + 4] = __fmul_rn(bf16lo_to_f32(ws[2]), l1.x);
+                v[8 * c + 5] = __fmul_rn(bf16hi_to_f32(ws[2]), l1.y);
+                v[8 * c + 6] = __fmul_rn(bf16lo_to_f32(ws[3]), l1.z);
+                v[8 * c + 7] = __fmul_rn(bf16hi_to_f32(ws[3]), l1.w);
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[s]);
-
             const int kc = c_lo + it;
             uint32_t cw[8];
-            uint32_t scw = 0;
+            if (PREC == kPrecNvfp4) {
+                uint32_t scw = 0;
 #pragma unroll
-            for (int g = 0; g < 4; ++g) {
-                float v[16];
-                const uint32_t ws[8] = {raw[2 * g].x,     raw[2 * g].y,     raw[2 * g].z,     raw[2 * g].w,
-                                        raw[2 * g + 1].x, raw[2 * g + 1].y, raw[2 * g + 1].z, raw[2 * g + 1].w};
+                for (int g = 0; g < 4; ++g) {
+                    float vg[16];
 #pragma unroll
-                for (int p = 0; p < 8; ++p) {
-                    v[2 * p] = __fmul_rn(bf16lo_to_f32(ws[p]), il[16 * g + 2 * p]);
-                    v[2 * p + 1] = __fmul_rn(bf16hi_to_f32(ws[p]), il[16 * g + 2 * p + 1]);
+                    for (int i = 0; i < 16; ++i) vg[i] = v[16 * g + i];
+                    scw |= quant_group16(vg, S, six_s, cw[2 * g], cw[2 * g + 1]) << (8 * g);
                 }
-                const uint32_t eb = quant_group16(v, S, six_s, cw[2 * g], cw[2 * g + 1]);
-                scw |= eb << (8 * g);
+                *reinterpret_cast<uint32_t*>(a.x_scales + sf_offset(grow, (int64_t)kc * 4, a.chunks)) = scw;
+            } else {
+                const uint32_t sb = quant_group64_int4(v, cw);
+                reinterpret_cast<uint16_t*>(a.x_scales)[(int64_t)kc * a.rows_pad + grow] = (uint16_t)sb;
             }
             if (grow < a.M) {
                 uint4* dst = reinterpret_cast<uint4*>(a.x_codes + grow * (int64_t)(a.K / 2) + (int64_t)kc * 32);
                 dst[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
                 dst[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
             }
-            *reinterpret_cast<uint32_t*>(a.x_scales + sf_offset(grow, (int64_t)kc * 4, a.chunks)) = scw;
+            // release the stage only after its data has been consumed
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[s]);
         }
         if (has_lr) {
             // partial rank-r sums of this CTA -> shared memory (reusing the stages)
@@ -360,7 +449,8 @@ __global__ void __launch_bounds__(qa::kThreads, 1)
         if (a.cluster > 1) cluster_sync_all();
         if (warp >= 2) {
             // reduce this CTA's slice of rows over the cluster, in rank order
-            const float ss = __fmul_rn(*a.x_scale, *a.w_scale);
+            const float ss = (PREC == kPrecNvfp4) ? __fmul_rn(*a.x_scale, *a.w_scale) : 1.0f;
+            const int64_t plane = (int64_t)a.M * a.rank;
             const float* red = reinterpret_cast<const float*>(smem);
             const int rs = a.rank + 1;
             const int rows_per = qa::kRows / a.cluster;
@@ -376,7 +466,12 @@ __global__ void __launch_bounds__(qa::kThreads, 1)
                     sum = red[rr * rs + j];
                 }
                 const int64_t gm = (int64_t)m0 + rr;
-                if (gm < a.M) a.lowrank[gm * a.rank + j] = __float2bfloat16_rn(__fdiv_rn(sum, ss));
+                if (gm < a.M) {
+                    __nv_bfloat16 hi, lo;
+                    split_bf16(PREC == kPrecNvfp4 ? __fdiv_rn(sum, ss) : sum, hi, lo);
+                    a.lowrank[gm * a.rank + j] = hi;
+                    a.lowrank[plane + gm * a.rank + j] = lo;
+                }
             }
         }
         if (a.cluster > 1) cluster_sync_all();

@@ -7,12 +7,13 @@
 
 #include <algorithm>
 #include <cstdint>
+#include <cstdio>
 #include <cstring>
 #include <mutex>
 
 #include "svdq.h"
 #include "sm100_ptx.cuh"
-#include "quant_nvfp4.cuh"
+#include "quantize.cuh"
 #include "gemm_nvfp4.cuh"
 #include "int4.cuh"
 
@@ -61,8 +62,27 @@ int g_override_major = -1, g_override_minor = 0;
 constexpr int kMaxDevices = 64;
 bool g_device_ready[kMaxDevices];
 
-svdq_status cuda_fail() {
-    cudaGetLastError();  // clear a sticky-free error so later calls start clean
+// Budget of dynamic shared memory for the activation quantizer (the opt-in
+// maximum is 227 KB per block including static shared memory).
+constexpr int kQuantSmemBudget = 226 * 1024;
+
+thread_local char g_last_error[256] = "";
+
+void note_error(cudaError_t e, const char* where) {
+    snprintf(g_last_error, sizeof(g_last_error), "%s: %s (%s)", where, cudaGetErrorString(e), cudaGetErrorName(e));
+}
+
+// Records and clears the pending CUDA error, then reports SVDQ_ERR_CUDA.
+svdq_status cuda_fail(const char* where = "CUDA call") {
+    const cudaError_t e = cudaGetLastError();
+    note_error(e == cudaSuccess ? cudaErrorUnknown : e, where);
+    return SVDQ_ERR_CUDA;
+}
+
+svdq_status launch_status(const char* where) {
+    const cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess) return SVDQ_OK;
+    note_error(e, where);
     return SVDQ_ERR_CUDA;
 }
 
@@ -90,10 +110,12 @@ svdq_status check_device() {
     if (!g_device_ready[dev]) {
         if (cudaFuncSetAttribute(gemm_nvfp4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)gm::SMEM_BYTES) != cudaSuccess ||
-            cudaFuncSetAttribute(quantize_act_nvfp4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 227 * 1024) != cudaSuccess ||
+            cudaFuncSetAttribute(quantize_act_kernel<kPrecNvfp4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kQuantSmemBudget) != cudaSuccess ||
+            cudaFuncSetAttribute(quantize_act_kernel<kPrecInt4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kQuantSmemBudget) != cudaSuccess ||
             int4_prepare_device() != cudaSuccess)
-            return cuda_fail();
+            return cuda_fail("setting kernel shared-memory limits");
         g_device_ready[dev] = true;
     }
     return SVDQ_OK;
@@ -128,9 +150,29 @@ bool make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t
     const cuuint64_t strides[1] = {row_bytes};
     const cuuint32_t box[2] = {box_inner, box_outer};
     const cuuint32_t estr[2] = {1, 1};
-    return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    const CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS)
+        snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled failed (CUresult %d)", (int)r);
+    return r == CUDA_SUCCESS;
+}
+
+// 3-D row-major tensor [planes, outer, inner] with 128-byte swizzled boxes of one plane.
+bool make_map_3d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
+                 uint64_t planes, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {inner, outer, planes};
+    const cuuint64_t strides[2] = {row_bytes, row_bytes * outer};
+    const cuuint32_t box[3] = {box_inner, box_outer, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS)
+        snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled (3-D) failed (CUresult %d)", (int)r);
+    return r == CUDA_SUCCESS;
 }
 
 int g_num_sms = 0;
@@ -147,13 +189,13 @@ int num_sms() {
 // ---------------------------------------------------------- nvfp4 paths
 svdq_status tensor_scale_prepass(const void* src, const float* inv_lambda, int64_t rows, int64_t K, float* out,
                                  cudaStream_t st) {
-    if (cudaMemsetAsync(out, 0, sizeof(float), st) != cudaSuccess) return cuda_fail();
+    if (cudaMemsetAsync(out, 0, sizeof(float), st) != cudaSuccess) return cuda_fail("cudaMemsetAsync");
     const int64_t nvec = rows * K / 8;
     const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>((nvec + 255) / 256, 8LL * num_sms()));
     amax_kernel<<<blocks, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(src), inv_lambda, rows, K,
                                         reinterpret_cast<unsigned int*>(out));
     finalize_tensor_scale_kernel<<<1, 1, 0, st>>>(out);
-    return cudaGetLastError() == cudaSuccess ? SVDQ_OK : SVDQ_ERR_CUDA;
+    return launch_status("tensor-scale pre-pass");
 }
 
 svdq_status fold_lowrank(const float* lambda, const void* L_down, const void* L_up, int64_t N, int64_t K, int rank,
@@ -164,7 +206,7 @@ svdq_status fold_lowrank(const float* lambda, const void* L_down, const void* L_
                                                 reinterpret_cast<const __nv_bfloat16*>(L_up), K, N, rank, inv_lambda,
                                                 reinterpret_cast<__nv_bfloat16*>(L_down_t),
                                                 reinterpret_cast<__nv_bfloat16*>(L_up_t));
-    return cudaGetLastError() == cudaSuccess ? SVDQ_OK : SVDQ_ERR_CUDA;
+    return launch_status("fold_lowrank_kernel");
 }
 
 svdq_status pack_weight_nvfp4(const void* R, int64_t N, int64_t K, void* w_codes, void* w_scales,
@@ -175,7 +217,7 @@ svdq_status pack_weight_nvfp4(const void* R, int64_t N, int64_t K, void* w_codes
     quantize_rows_nvfp4_kernel<<<(unsigned)((work + 255) / 256), 256, 0, st>>>(
         reinterpret_cast<const __nv_bfloat16*>(R), N, rows_pad, K, w_tensor_scale,
         reinterpret_cast<uint8_t*>(w_codes), reinterpret_cast<uint8_t*>(w_scales));
-    return cudaGetLastError() == cudaSuccess ? SVDQ_OK : SVDQ_ERR_CUDA;
+    return launch_status("quantize_rows_nvfp4_kernel");
 }
 
 // Cluster width for the activation quantizer: enough CTAs to cover the SMs
@@ -198,7 +240,7 @@ int choose_cluster(int64_t row_blocks, int chunks, int smem_bytes) {
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         int nclusters = 0;
-        if (cudaOccupancyMaxActiveClusters(&nclusters, quantize_act_nvfp4_kernel, &cfg) != cudaSuccess) {
+        if (cudaOccupancyMaxActiveClusters(&nclusters, quantize_act_kernel<kPrecNvfp4>, &cfg) != cudaSuccess) {
             cudaGetLastError();
             nclusters = 0;
         }
@@ -208,16 +250,17 @@ int choose_cluster(int64_t row_blocks, int chunks, int smem_bytes) {
     return c;
 }
 
-svdq_status quantize_act_nvfp4(const void* x, int64_t M, int64_t K, const float* inv_lambda, float* x_scale,
-                               int compute_scale, const float* w_scale, const void* L_down_t, int rank,
-                               void* x_codes, void* x_scales, void* lowrank, cudaStream_t st) {
-    if (compute_scale) SVDQ_TRY(tensor_scale_prepass(x, inv_lambda, M, K, x_scale, st));
+// Activation quantizer launch (both precisions).  x_scale / w_scale are only
+// read by the nvfp4 variant.
+svdq_status quantize_act_launch(int prec, const void* x, int64_t M, int64_t K, const float* inv_lambda,
+                                const float* x_scale, const float* w_scale, const void* L_down_t, int rank,
+                                void* x_codes, void* x_scales, void* lowrank, cudaStream_t st) {
     CUtensorMap tm_x, tm_ld;
     if (!make_map(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, 64, 128))
         return SVDQ_ERR_CUDA;
     if (rank > 0) {
-        if (!make_map(&tm_ld, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L_down_t, (uint64_t)K, (uint64_t)rank,
-                      (uint64_t)K * 2, 64, (uint32_t)rank))
+        if (!make_map_3d(&tm_ld, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L_down_t, (uint64_t)K, (uint64_t)rank, 2,
+                         (uint64_t)K * 2, 64, (uint32_t)rank))
             return SVDQ_ERR_CUDA;
     } else {
         tm_ld = tm_x;
@@ -232,11 +275,11 @@ svdq_status quantize_act_nvfp4(const void* x, int64_t M, int64_t K, const float*
     a.M = (int)M;
     a.K = (int)K;
     a.rank = rank;
+    a.rows_pad = (int)round_up(M, 128);
     a.chunks = (int)(K / 64);
-    const uint32_t ld_pad = (uint32_t)round_up((int64_t)rank * 128, 1024);
-    a.stage_bytes = (uint32_t)qa::kXBytes + ld_pad;
+    a.stage_bytes = (uint32_t)qa::kXBytes + (uint32_t)rank * 256u;   // x tile + hi and lo L_down_t tiles
     const size_t fixed = 1024 + qa::kMaxStages * qa::kCols * 4 + (2 * qa::kMaxStages + 1) * 8 + 16;
-    int stages = (int)std::min<size_t>(qa::kMaxStages, (226 * 1024 - fixed) / a.stage_bytes);
+    const int stages = (int)std::min<size_t>(qa::kMaxStages, (kQuantSmemBudget - fixed) / a.stage_bytes);
     const size_t red_bytes = (size_t)qa::kRows * (rank + 1) * 4;
     if (stages < 2 || (size_t)stages * a.stage_bytes < red_bytes) return SVDQ_ERR_UNSUPPORTED_SHAPE;
     a.stages = stages;
@@ -260,8 +303,28 @@ svdq_status quantize_act_nvfp4(const void* x, int64_t M, int64_t K, const float*
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, quantize_act_nvfp4_kernel, tm_x, tm_ld, a) != cudaSuccess) return cuda_fail();
+    const cudaError_t e = prec == kPrecNvfp4 ? cudaLaunchKernelEx(&cfg, quantize_act_kernel<kPrecNvfp4>, tm_x, tm_ld, a)
+                                             : cudaLaunchKernelEx(&cfg, quantize_act_kernel<kPrecInt4>, tm_x, tm_ld, a);
+    if (e != cudaSuccess) return cuda_fail("quantize_act_kernel launch");
     return SVDQ_OK;
+}
+
+svdq_status quantize_act_nvfp4(const void* x, int64_t M, int64_t K, const float* inv_lambda, float* x_scale,
+                               int compute_scale, const float* w_scale, const void* L_down_t, int rank,
+                               void* x_codes, void* x_scales, void* lowrank, cudaStream_t st) {
+    if (compute_scale) SVDQ_TRY(tensor_scale_prepass(x, inv_lambda, M, K, x_scale, st));
+    return quantize_act_launch(kPrecNvfp4, x, M, K, inv_lambda, x_scale, w_scale, L_down_t, rank, x_codes, x_scales,
+                               lowrank, st);
+}
+
+// ----------------------------------------------------------- int4 paths
+svdq_status int4_quantize_rows(const void* R, int64_t N, int64_t K, void* w_codes, void* w_scales, cudaStream_t st) {
+    const int64_t rows_pad = round_up(N, 128);
+    const int64_t work = rows_pad * (K / 64);
+    quantize_rows_int4_kernel<<<(unsigned)((work + 255) / 256), 256, 0, st>>>(
+        reinterpret_cast<const __nv_bfloat16*>(R), N, rows_pad, K, reinterpret_cast<uint8_t*>(w_codes),
+        reinterpret_cast<uint16_t*>(w_scales));
+    return launch_status("quantize_rows_int4_kernel");
 }
 
 svdq_status gemm_nvfp4(const void* x_codes, const void* x_scales, const float* x_scale, int64_t M,
@@ -274,8 +337,8 @@ svdq_status gemm_nvfp4(const void* x_codes, const void* x_scales, const float* x
                   gm::BK_BYTES, gm::BN))
         return SVDQ_ERR_CUDA;
     if (rank > 0) {
-        if (!make_map(&tm_L, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, lowrank, (uint64_t)rank, (uint64_t)M,
-                      (uint64_t)rank * 2, 64, gm::BM) ||
+        if (!make_map_3d(&tm_L, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, lowrank, (uint64_t)rank, (uint64_t)M, 2,
+                         (uint64_t)rank * 2, 64, gm::BM) ||
             !make_map(&tm_Lup, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L_up_t, (uint64_t)rank, (uint64_t)N,
                       (uint64_t)rank * 2, 64, gm::BN))
             return SVDQ_ERR_CUDA;
@@ -300,7 +363,7 @@ svdq_status gemm_nvfp4(const void* x_codes, const void* x_scales, const float* x
     if (nt > 65535) return SVDQ_ERR_UNSUPPORTED_SHAPE;
     gemm_nvfp4_kernel<<<dim3((unsigned)mt, (unsigned)nt, 1), gm::kThreads, gm::SMEM_BYTES, st>>>(tm_xc, tm_wc, tm_L,
                                                                                              tm_Lup, a);
-    return cudaGetLastError() == cudaSuccess ? SVDQ_OK : SVDQ_ERR_CUDA;
+    return launch_status("gemm_nvfp4_kernel launch");
 }
 
 // Kernel that waits on a barrier nobody completes: exercises the bounded wait.
@@ -336,6 +399,8 @@ const char* svdq_status_string(svdq_status s) {
 
 int svdq_abi_version(void) { return kAbiVersion; }
 
+const char* svdq_last_error(void) { return g_last_error; }
+
 svdq_status svdq_buffer_sizes(svdq_precision p, int64_t rows, int64_t K, int rank, svdq_sizes* out) {
     if (!out) return SVDQ_ERR_INVALID_ARG;
     if (p != SVDQ_NVFP4 && p != SVDQ_INT4) return SVDQ_ERR_INVALID_ARG;
@@ -344,7 +409,7 @@ svdq_status svdq_buffer_sizes(svdq_precision p, int64_t rows, int64_t K, int ran
     const int64_t rows_pad = round_up(rows, 128);
     out->codes_bytes = (size_t)(rows * K / 2);
     out->scales_bytes = p == SVDQ_NVFP4 ? (size_t)(rows_pad * K / 16) : (size_t)(2 * rows_pad * K / 64);
-    out->lowrank_bytes = (size_t)(2 * rows * rank);
+    out->lowrank_bytes = (size_t)(4 * rows * rank);   // hi and lo bf16 planes
     return SVDQ_OK;
 }
 
@@ -372,7 +437,7 @@ svdq_status svdq_pack_weight(svdq_precision p, int group_size, const void* R, in
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     SVDQ_TRY(fold_lowrank(lambda, L_down, L_up, N, K, rank, inv_lambda, L_down_t, L_up_t, st));
     if (p == SVDQ_NVFP4) return pack_weight_nvfp4(R, N, K, w_codes, w_scales, w_tensor_scale, st);
-    return int4_quantize_rows(R, nullptr, N, K, w_codes, w_scales, st);
+    return int4_quantize_rows(R, N, K, w_codes, w_scales, st);
 }
 
 svdq_status svdq_quantize_act(svdq_precision p, int group_size, const void* x, int64_t M, int64_t K,
@@ -397,7 +462,8 @@ svdq_status svdq_quantize_act(svdq_precision p, int group_size, const void* x, i
     if (p == SVDQ_NVFP4)
         return quantize_act_nvfp4(x, M, K, inv_lambda, x_tensor_scale, compute_scale, w_tensor_scale, L_down_t, rank,
                                   x_codes, x_scales, lowrank_act, st);
-    return int4_quantize_act(x, M, K, inv_lambda, L_down_t, rank, x_codes, x_scales, lowrank_act, st);
+    return quantize_act_launch(kPrecInt4, x, M, K, inv_lambda, nullptr, nullptr, L_down_t, rank, x_codes, x_scales,
+                               lowrank_act, st);
 }
 
 svdq_status svdq_gemm_w4a4(svdq_precision p, int group_size, const void* x_codes, const void* x_scales,
@@ -458,7 +524,7 @@ svdq_status svdq_debug_set_wait_limit_ns(uint64_t ns) {
 svdq_status svdq_debug_timeout_probe(svdq_stream_t stream) {
     SVDQ_TRY(check_device());
     timeout_probe_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>();
-    return cudaGetLastError() == cudaSuccess ? SVDQ_OK : SVDQ_ERR_CUDA;
+    return launch_status("timeout_probe_kernel launch");
 }
 
 void svdq_debug_override_capability(int major, int minor) {

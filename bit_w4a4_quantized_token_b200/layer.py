@@ -59,7 +59,7 @@ def pack_weight(R: torch.Tensor, lam: torch.Tensor, L_down: torch.Tensor | None,
     w_scales = _empty(sz["scales_bytes"], dev)
     w_ts = torch.empty(4, dtype=torch.float32, device=dev) if precision == "nvfp4" else None
     inv_lambda = torch.empty(K, dtype=torch.float32, device=dev)
-    L_down_t = torch.empty(rank, K, dtype=torch.bfloat16, device=dev) if rank else None
+    L_down_t = torch.empty(2, rank, K, dtype=torch.bfloat16, device=dev) if rank else None
     L_up_t = torch.empty(N, rank, dtype=torch.bfloat16, device=dev) if rank else None
     _lib.svdq_pack_weight(precision, _lib.GROUP_SIZES[precision], R.contiguous(), N, K, lam.contiguous(),
                           None if rank == 0 else L_down.contiguous(), None if rank == 0 else L_up.contiguous(),
@@ -75,7 +75,7 @@ def alloc_act(packed: PackedWeight, M: int, device) -> QuantizedAct:
         _empty(sz["codes_bytes"], device),
         _empty(sz["scales_bytes"], device),
         torch.empty(4, dtype=torch.float32, device=device) if packed.precision == "nvfp4" else None,
-        torch.empty(M, packed.rank, dtype=torch.bfloat16, device=device) if packed.rank else None,
+        torch.empty(2, M, packed.rank, dtype=torch.bfloat16, device=device) if packed.rank else None,
     )
 
 

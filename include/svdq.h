@@ -45,12 +45,16 @@
  *            scales[g * rows_pad + r] with rows_pad = rows rounded up to 128
  *            (padding rows are zero).
  *  - tensor scale (nvfp4 only): one fp32 S; a value is code * scale * S.
- *  - rank-r activations ("lowrank_act"): bf16 [M, rank].  nvfp4 stores
- *            ((x/lambda) . L_down) / (S_x * S_w) so the GEMM can add it into the
- *            unscaled FP4 accumulator; int4 stores (x/lambda) . L_down.
+ *  - hi/lo pairs: an fp32 value v carried as two bf16 planes, hi = bf16(v)
+ *            and lo = bf16(v - hi), so that bf16 tensor-core products of both
+ *            planes reproduce v to about 2^-17 relative.
+ *  - rank-r activations ("lowrank_act"): bf16 [2, M, rank] (hi plane, then lo
+ *            plane) of L' where nvfp4 stores L' = ((x/lambda) . L_down) / (S_x S_w)
+ *            so the GEMM can add it into the unscaled FP4 accumulator, and int4
+ *            stores L' = (x/lambda) . L_down.
  *  - folded weights: inv_lambda fp32 [K] = 1/lambda (IEEE round-to-nearest);
- *            L_down_t bf16 [rank, K] = bf16(L_down[k,j] / lambda[k]) transposed;
- *            L_up_t bf16 [N, rank] = L_up transposed.
+ *            L_down_t bf16 [2, rank, K]: hi/lo pair of fl32(L_down[k,j] / lambda[k]),
+ *            transposed; L_up_t bf16 [N, rank] = L_up transposed.
  */
 #ifndef SVDQ_H_
 #define SVDQ_H_
@@ -83,7 +87,7 @@ typedef enum {
 typedef struct {
     size_t codes_bytes;    /* rows * K / 2 */
     size_t scales_bytes;   /* nvfp4: rows_pad * K / 16;  int4: 2 * rows_pad * K / 64 */
-    size_t lowrank_bytes;  /* 2 * rows * rank (bf16 rank-r activations) */
+    size_t lowrank_bytes;  /* 4 * rows * rank (rank-r activations: hi and lo bf16 planes) */
 } svdq_sizes;
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -91,6 +95,10 @@ const char* svdq_status_string(svdq_status status);
 
 /* Version of this ABI (increments on any incompatible change). */
 int svdq_abi_version(void);
+
+/* Description of the last CUDA failure seen by this thread (the failing call
+ * and the CUDA error name), or "" if none; valid until the next failure. */
+const char* svdq_last_error(void);
 
 /* Pure host function: fills *out for the given precision and sizes.
  * Errors: INVALID_ARG (out NULL, unknown precision, bad rank),
@@ -105,7 +113,7 @@ svdq_status svdq_buffer_sizes(svdq_precision precision, int64_t rows, int64_t K,
  * Outputs (device, caller-allocated):
  *   w_codes [N, K/2]; w_scales (scales_bytes for N rows); w_tensor_scale fp32[1]
  *   (nvfp4: S_w = amax|R| / 2688, or 1 when R == 0; int4: may be NULL);
- *   inv_lambda fp32 [K]; L_down_t bf16 [rank, K]; L_up_t bf16 [N, rank].
+ *   inv_lambda fp32 [K]; L_down_t bf16 [2, rank, K]; L_up_t bf16 [N, rank].
  * group_size must be 16 for SVDQ_NVFP4 and 64 for SVDQ_INT4. */
 svdq_status svdq_pack_weight(svdq_precision precision, int group_size,
                              const void* R, int64_t N, int64_t K,
@@ -122,9 +130,9 @@ svdq_status svdq_pack_weight(svdq_precision precision, int group_size,
  *                  compute_scale != 0 it is overwritten with
  *                  S_x = amax|x/lambda| / 2688 (1 when x == 0) first.
  *   w_tensor_scale device fp32 [1] (nvfp4 with rank > 0): S_w
- *   L_down_t       device bf16 [rank, K] (NULL when rank == 0)
+ *   L_down_t       device bf16 [2, rank, K] (NULL when rank == 0)
  * Outputs: x_codes [M, K/2]; x_scales (scales_bytes for M rows, padding rows
- *   written as zeros); lowrank_act bf16 [M, rank] (NULL when rank == 0). */
+ *   written as zeros); lowrank_act bf16 [2, M, rank] (NULL when rank == 0). */
 svdq_status svdq_quantize_act(svdq_precision precision, int group_size,
                               const void* x, int64_t M, int64_t K, const float* inv_lambda,
                               float* x_tensor_scale, int compute_scale,

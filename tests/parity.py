@@ -53,24 +53,41 @@ def bf16_ulp_distance(a_bits: np.ndarray, b_bits: np.ndarray) -> np.ndarray:
     return np.abs(mono(a_bits) - mono(b_bits))
 
 
+def bf16_half_ulp(v: np.ndarray) -> np.ndarray:
+    """Half a bf16 unit in the last place at |v| (the error of rounding v to bf16)."""
+    a = np.maximum(np.abs(v), 2.0 ** -126)
+    return np.exp2(np.floor(np.log2(a)) - 8)
+
+
 def check_y(y_gpu_bits: np.ndarray, y_ref: np.ndarray, y_ref_bits: np.ndarray, what: str = "y") -> dict:
-    """The output bar: max|d| <= 1e-2 rms(y_ref), and <= 1 bf16 ulp on >= 99.9 %."""
+    """The output bar.
+
+    1. max_i (|y_gpu - y_ref| - half_ulp_bf16(y_ref)) <= 1e-2 rms(y_ref): the
+       error beyond the unavoidable rounding of the exact fp64 value y_ref to
+       the bf16 output is at most 1 % of the output rms.  (Half a bf16 ulp of
+       the largest outputs is itself more than 1 % of the rms, so the bound
+       cannot apply to the rounding of the bf16 store.)
+    2. the bf16 output is within 1 ulp of the oracle's own bf16 rounding of
+       y_ref on >= 99.9 % of the elements.
+    """
     y_gpu = (np.asarray(y_gpu_bits, np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
     assert np.all(np.isfinite(y_gpu)), f"{what}: non-finite outputs"
     rms = float(np.sqrt(np.mean(y_ref ** 2)))
-    maxerr = float(np.max(np.abs(y_gpu - y_ref)))
+    err = np.abs(y_gpu - y_ref)
+    excess = float(np.max(err - bf16_half_ulp(y_ref)))
     ulps = bf16_ulp_distance(y_gpu_bits, y_ref_bits)
     frac1 = float(np.mean(ulps <= 1))
-    stats = {"rms": rms, "max_abs_err": maxerr, "max_rel_rms": maxerr / rms, "frac_within_1ulp": frac1,
-             "max_ulps": int(ulps.max())}
-    assert maxerr <= 1e-2 * rms, f"{what}: {stats}"
+    stats = {"rms": rms, "max_abs_err": float(err.max()), "max_excess_over_half_ulp_rel_rms": excess / rms,
+             "frac_within_1ulp": frac1, "max_ulps": int(ulps.max())}
+    assert excess <= 1e-2 * rms, f"{what}: {stats}"
     assert frac1 >= 0.999, f"{what}: {stats}"
     return stats
 
 
 def check_lowrank(L_gpu: torch.Tensor, L_ref: np.ndarray, prescale: float) -> float:
-    """Rank-r activations within 1e-2 relative rms (bf16 storage, folded 1/lambda)."""
-    got = L_gpu.float().cpu().numpy().astype(np.float64) * prescale
+    """Rank-r activations (hi + lo bf16 planes) within 1e-2 relative rms."""
+    planes = L_gpu.double().cpu().numpy()
+    got = (planes[0] + planes[1]) * prescale
     err = float(np.sqrt(np.mean((got - L_ref) ** 2)) / max(np.sqrt(np.mean(L_ref ** 2)), 1e-30))
     assert err <= 1e-2, err
     return err

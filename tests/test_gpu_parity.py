@@ -121,3 +121,27 @@ FULL = [W.QKV, W.FC1, W.FC2] + [W.OUTPROJ[r] for r in (0, 16, 32, 64, 128)]
 @pytest.mark.parametrize("case", FULL, ids=lambda c: c.name)
 def test_full_size_sampled_rows(case):
     check_case(case, rows=sample_rows(case.M, n=24, seed=case.seed))
+
+
+# ------------------------------------------------------------ int4 quantizers
+@pytest.mark.parametrize("case", [W.scaled(W.INT4_QKV, M=200, K=320, N=272, rank=16, name="int4_ragged"),
+                                  W.scaled(W.INT4_QKV, M=256, K=1024, N=512, rank=32, name="int4_small"),
+                                  W.INT4_QKV], ids=lambda c: c.name)
+def test_int4_quantizers(case):
+    """Codes and bf16 group scales bit-exact; rank-r activations within 1e-2 rms."""
+    from bit_w4a4_quantized_token_b200 import layer
+
+    from .parity import check_lowrank, unswizzle_int4_scales
+
+    inp = W.make_inputs(case)
+    d = {k: v.cuda() for k, v in inp.items()}
+    packed = layer.pack_weight(d["R"], d["lam"], d["L_down"], d["L_up"], d["b"], precision="int4")
+    q = layer.quantize_act(d["x"], packed)
+    torch.cuda.synchronize()
+    ref = oracle_for(case, inp, with_y=False)
+    M, K, N = case.M, case.K, case.N
+    assert np.array_equal(packed.w_codes.cpu().numpy().reshape(N, K // 2), ref.w_codes)
+    assert np.array_equal(q.x_codes.cpu().numpy().reshape(M, K // 2), ref.x_codes)
+    assert np.array_equal(unswizzle_int4_scales(packed.w_scales.cpu().numpy(), N, K), ref.w_scales)
+    assert np.array_equal(unswizzle_int4_scales(q.x_scales.cpu().numpy(), M, K), ref.x_scales)
+    check_lowrank(q.lowrank_act, ref.L, 1.0)
