@@ -29,7 +29,7 @@ GROUP_SIZES = {"nvfp4": 16, "int4": 64}
 # Every entry point declared in include/svdq.h.
 EXPORTS = (
     "svdq_status_string", "svdq_abi_version", "svdq_last_error", "svdq_buffer_sizes", "svdq_pack_weight",
-    "svdq_quantize_act", "svdq_gemm_w4a4", "svdq_device_status",
+    "svdq_quantize_act_workspace_bytes", "svdq_quantize_act", "svdq_gemm_w4a4", "svdq_device_status",
     "svdq_debug_set_wait_limit_ns", "svdq_debug_timeout_probe", "svdq_debug_override_capability",
 )
 
@@ -64,7 +64,9 @@ def _load():
     lib.svdq_buffer_sizes.restype = I
     lib.svdq_pack_weight.argtypes = [I, I, P, I64, I64, P, P, P, I, P, P, P, P, P, P, P]
     lib.svdq_pack_weight.restype = I
-    lib.svdq_quantize_act.argtypes = [I, I, P, I64, I64, P, P, I, P, P, I, P, P, P, P]
+    lib.svdq_quantize_act_workspace_bytes.argtypes = [I, I64, I64, I, ctypes.POINTER(ctypes.c_size_t)]
+    lib.svdq_quantize_act_workspace_bytes.restype = I
+    lib.svdq_quantize_act.argtypes = [I, I, P, I64, I64, P, P, I, P, P, I, P, P, P, P, ctypes.c_size_t, P]
     lib.svdq_quantize_act.restype = I
     lib.svdq_gemm_w4a4.argtypes = [I, I, P, P, P, I64, P, P, P, I64, I64, P, P, I, P, P, P]
     lib.svdq_gemm_w4a4.restype = I
@@ -133,12 +135,22 @@ def svdq_pack_weight(precision, group_size, R, N, K, lam, L_down, L_up, rank, w_
                                 _stream(stream)), "svdq_pack_weight")
 
 
+def svdq_quantize_act_workspace_bytes(precision, M: int, K: int, rank: int) -> int:
+    out = ctypes.c_size_t(0)
+    _check(lib.svdq_quantize_act_workspace_bytes(_prec(precision), int(M), int(K), int(rank), ctypes.byref(out)),
+           "svdq_quantize_act_workspace_bytes")
+    return int(out.value)
+
+
 def svdq_quantize_act(precision, group_size, x, M, K, inv_lambda, x_tensor_scale, compute_scale,
-                      w_tensor_scale, L_down_t, rank, x_codes, x_scales, lowrank_act, stream=None) -> None:
+                      w_tensor_scale, L_down_t, rank, x_codes, x_scales, lowrank_act, workspace=None,
+                      workspace_bytes=0, stream=None) -> None:
+    if workspace is not None and not isinstance(workspace, int) and not workspace_bytes:
+        workspace_bytes = workspace.numel() * workspace.element_size()
     _check(lib.svdq_quantize_act(_prec(precision), int(group_size), _ptr(x), int(M), int(K), _ptr(inv_lambda),
                                  _ptr(x_tensor_scale), int(bool(compute_scale)), _ptr(w_tensor_scale),
                                  _ptr(L_down_t), int(rank), _ptr(x_codes), _ptr(x_scales), _ptr(lowrank_act),
-                                 _stream(stream)), "svdq_quantize_act")
+                                 _ptr(workspace), int(workspace_bytes), _stream(stream)), "svdq_quantize_act")
 
 
 def svdq_gemm_w4a4(precision, group_size, x_codes, x_scales, x_tensor_scale, M, w_codes, w_scales,

@@ -8,11 +8,14 @@
 // "NVFP4 runtime kernel with SVDQ low-rank correction" of the Diffusers docs
 // page "Nunchaku Lite" ("Supported quantization types" table).
 //
-// One CTA computes a 128 x 256 tile: warp 0 issues TMA loads (codes with
-// 128-byte swizzle, scale blocks with bulk copies) into a 4-stage ring, warp 1
-// copies the scale blocks to TMEM and issues tcgen05.mma (kind::mxf4nvf4,
-// K = 64 per instruction, then kind::f16 for the rank-r chunks), warps 2..5
-// drain the fp32 accumulator from TMEM and store bf16.
+// Persistent kernel, one CTA per SM, 128 x 256 output tiles taken round-robin.
+// Warp 0 issues TMA loads (codes with 128-byte swizzle, scale blocks with bulk
+// copies) into a ring of stages that runs across tile boundaries; warp 1
+// copies each stage's scale blocks into TMEM and issues tcgen05.mma
+// (kind::mxf4nvf4, K = 64 per instruction; kind::f16 for the rank-r chunks);
+// eight epilogue warps pull the finished accumulator out of TMEM into
+// registers, hand TMEM back to the MMA warp at once, and then scale, add the
+// bias and store bf16 while the next tile's MMAs run.
 #pragma once
 #include "sm100_ptx.cuh"
 
@@ -27,7 +30,8 @@ constexpr int B_BYTES = BN * BK_BYTES;        // 32 KB (also holds a 256 x 64 bf
 constexpr int SFA_BYTES = 4 * 512;            // 4 scale blocks: 128 rows x 16 groups
 constexpr int SFB_BYTES = 8 * 512;            // 2 row blocks x 4 scale blocks
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
-constexpr int kThreads = 192;
+constexpr int kEpiWarps = 8;                  // 2 per TMEM lane quadrant, 128 columns each
+constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COL = 0;               // 256 fp32 columns
 constexpr uint32_t SFA_COL = 256;             // 4 k-steps x 4 columns
@@ -45,9 +49,10 @@ struct GemmArgs {
     int M, N, K, rank;
     int kg4;                     // K / 64: scale blocks per 128 rows
     int n_sf_blocks;             // ceil(N / 128): 128-row blocks present in w_scales
+    int m_tiles, n_tiles;
 };
 
-enum : uint32_t { kSiteGmEmpty = 16, kSiteGmFull = 17, kSiteGmAcc = 18, kSiteGmDrain = 19 };
+enum : uint32_t { kSiteGmEmpty = 16, kSiteGmFull = 17, kSiteGmAcc = 18, kSiteGmDrain = 19, kSiteGmAccEmpty = 20 };
 
 __global__ void __launch_bounds__(gm::kThreads, 1)
     gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_xc, const __grid_constant__ CUtensorMap tm_wc,
@@ -58,23 +63,24 @@ __global__ void __launch_bounds__(gm::kThreads, 1)
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)kStages * STAGE_BYTES);
     uint64_t* empty = full + kStages;
-    uint64_t* accb = empty + kStages;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accb + 1);
+    uint64_t* acc_full = empty + kStages;
+    uint64_t* acc_empty = acc_full + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
     __shared__ int s_issued, s_consumed, s_failed;
 
     const uint32_t warp = warp_id(), lane = lane_id();
-    const int m_tile = blockIdx.x, n_tile = blockIdx.y;
-    const int m0 = m_tile * BM, n0 = n_tile * BN;
     const int n_kb = (a.K + 255) / 256;
     const int n_lr = a.rank > 0 ? 2 * ((a.rank + 63) / 64) : 0;   // hi and lo part of each 64-column chunk
-    const int total = n_kb + n_lr;
+    const int per_tile = n_kb + n_lr;
+    const int total_tiles = a.m_tiles * a.n_tiles;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        mbar_init(accb, 1);
+        mbar_init(acc_full, 1);
+        mbar_init(acc_empty, kEpiWarps);
         s_issued = 0;
         s_consumed = 0;
         s_failed = 0;
@@ -100,36 +106,42 @@ __global__ void __launch_bounds__(gm::kThreads, 1)
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
-            int it = 0;
-            for (; it < total; ++it) {
-                const int s = it % kStages;
-                const uint32_t ph = (uint32_t)(it / kStages) & 1u;
-                if (!mbar_wait(&empty[s], ph ^ 1u, kSiteGmEmpty)) {
-                    s_failed = 1;
-                    break;
-                }
-                uint8_t* sa = smem + (size_t)s * STAGE_BYTES;
-                uint8_t* sb = sa + A_BYTES;
-                if (it < n_kb) {
-                    const int kb = it;
-                    const int natoms = min(4, a.kg4 - 4 * kb);
-                    const uint32_t sf_bytes = (uint32_t)natoms * 512u;
-                    const int nb0 = 2 * n_tile;
-                    const int nbv = (nb0 < a.n_sf_blocks ? 1 : 0) + (nb0 + 1 < a.n_sf_blocks ? 1 : 0);
-                    mbar_arrive_expect_tx(&full[s], A_BYTES + B_BYTES + sf_bytes * (1u + (uint32_t)nbv));
-                    tma_load_2d(sa, &tm_xc, &full[s], kb * BK_BYTES, m0);
-                    tma_load_2d(sb, &tm_wc, &full[s], kb * BK_BYTES, n0);
-                    uint8_t* sfa = sb + B_BYTES;
-                    uint8_t* sfb = sfa + SFA_BYTES;
-                    bulk_load(sfa, a.x_scales + ((int64_t)m_tile * a.kg4 + 4 * kb) * 512, sf_bytes, &full[s]);
-                    for (int rb = 0; rb < nbv; ++rb)
-                        bulk_load(sfb + rb * 2048, a.w_scales + ((int64_t)(nb0 + rb) * a.kg4 + 4 * kb) * 512,
-                                  sf_bytes, &full[s]);
-                } else {
-                    const int c = (it - n_kb) >> 1, part = (it - n_kb) & 1;
-                    mbar_arrive_expect_tx(&full[s], A_BYTES + B_BYTES);
-                    tma_load_3d(sa, &tm_L, &full[s], c * 64, m0, part);
-                    tma_load_2d(sb, &tm_Lup, &full[s], c * 64, n0);
+            int it = 0;   // position in the stage ring, continued across tiles
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+                const int m_tile = tile % a.m_tiles, n_tile = tile / a.m_tiles;
+                const int m0 = m_tile * BM, n0 = n_tile * BN;
+                const int nb0 = 2 * n_tile;
+                const int nbv = (nb0 < a.n_sf_blocks ? 1 : 0) + (nb0 + 1 < a.n_sf_blocks ? 1 : 0);
+                for (int kk = 0; kk < per_tile; ++kk, ++it) {
+                    const int s = it % kStages;
+                    const uint32_t ph = (uint32_t)(it / kStages) & 1u;
+                    if (!mbar_wait(&empty[s], ph ^ 1u, kSiteGmEmpty)) {
+                        s_failed = 1;
+                        ok = false;
+                        break;
+                    }
+                    uint8_t* sa = smem + (size_t)s * STAGE_BYTES;
+                    uint8_t* sb = sa + A_BYTES;
+                    if (kk < n_kb) {
+                        const int kb = kk;
+                        const int natoms = min(4, a.kg4 - 4 * kb);
+                        const uint32_t sf_bytes = (uint32_t)natoms * 512u;
+                        mbar_arrive_expect_tx(&full[s], A_BYTES + B_BYTES + sf_bytes * (1u + (uint32_t)nbv));
+                        tma_load_2d(sa, &tm_xc, &full[s], kb * BK_BYTES, m0);
+                        tma_load_2d(sb, &tm_wc, &full[s], kb * BK_BYTES, n0);
+                        uint8_t* sfa = sb + B_BYTES;
+                        uint8_t* sfb = sfa + SFA_BYTES;
+                        bulk_load(sfa, a.x_scales + ((int64_t)m_tile * a.kg4 + 4 * kb) * 512, sf_bytes, &full[s]);
+                        for (int rb = 0; rb < nbv; ++rb)
+                            bulk_load(sfb + rb * 2048, a.w_scales + ((int64_t)(nb0 + rb) * a.kg4 + 4 * kb) * 512,
+                                      sf_bytes, &full[s]);
+                    } else {
+                        const int c = (kk - n_kb) >> 1, part = (kk - n_kb) & 1;
+                        mbar_arrive_expect_tx(&full[s], A_BYTES + B_BYTES);
+                        tma_load_3d(sa, &tm_L, &full[s], c * 64, m0, part);
+                        tma_load_2d(sb, &tm_Lup, &full[s], c * 64, n0);
+                    }
                 }
             }
             s_issued = it;
@@ -140,86 +152,112 @@ __global__ void __launch_bounds__(gm::kThreads, 1)
             const uint32_t idesc_fp4 = idesc_nvfp4(BN);
             const uint32_t idesc_lr = idesc_bf16_f32(BN);
             bool ok = true;
-            int it = 0;
-            for (; it < total; ++it) {
-                const int s = it % kStages;
-                const uint32_t ph = (uint32_t)(it / kStages) & 1u;
-                if (!mbar_wait(&full[s], ph, kSiteGmFull)) {
-                    ok = false;
+            int it = 0, local = 0;
+            for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x, ++local) {
+                // the epilogue must have pulled the previous tile out of TMEM
+                if (!mbar_wait(acc_empty, ((uint32_t)local & 1u) ^ 1u, kSiteGmAccEmpty)) {
                     s_failed = 1;
                     break;
                 }
                 tc_fence_after();
-                const uint32_t sa = smem_u32(smem + (size_t)s * STAGE_BYTES);
-                const uint32_t sb = sa + A_BYTES;
-                if (it < n_kb) {
-                    const uint32_t sfa = sb + B_BYTES;
-                    const uint32_t sfb = sfa + SFA_BYTES;
-                    const int nks = min(4, a.kg4 - 4 * it);
-                    for (int j = 0; j < nks; ++j) {
-                        tmem_cp_32x128b_x4(tmem + SFA_COL + 4u * j, desc_sf_block(sfa + 512u * j));
-                        tmem_cp_32x128b_x4(tmem + SFB_COL + 8u * j, desc_sf_block(sfb + 512u * j));
-                        tmem_cp_32x128b_x4(tmem + SFB_COL + 8u * j + 4u, desc_sf_block(sfb + 2048u + 512u * j));
+                for (int kk = 0; kk < per_tile; ++kk, ++it) {
+                    const int s = it % kStages;
+                    const uint32_t ph = (uint32_t)(it / kStages) & 1u;
+                    if (!mbar_wait(&full[s], ph, kSiteGmFull)) {
+                        ok = false;
+                        s_failed = 1;
+                        break;
                     }
-                    for (int j = 0; j < nks; ++j)
-                        mma_nvfp4(tmem + ACC_COL, desc_sw128(sa + 32u * j), desc_sw128(sb + 32u * j), idesc_fp4,
-                                  tmem + SFA_COL + 4u * j, tmem + SFB_COL + 8u * j, (it > 0 || j > 0) ? 1u : 0u);
-                } else {
-                    const int c = (it - n_kb) >> 1;
-                    const int nks = min(4, (a.rank - 64 * c + 15) / 16);
-                    for (int j = 0; j < nks; ++j)
-                        mma_bf16(tmem + ACC_COL, desc_sw128(sa + 32u * j), desc_sw128(sb + 32u * j), idesc_lr, 1u);
+                    tc_fence_after();
+                    const uint32_t sa = smem_u32(smem + (size_t)s * STAGE_BYTES);
+                    const uint32_t sb = sa + A_BYTES;
+                    if (kk < n_kb) {
+                        const uint32_t sfa = sb + B_BYTES;
+                        const uint32_t sfb = sfa + SFA_BYTES;
+                        const int nks = min(4, a.kg4 - 4 * kk);
+                        for (int j = 0; j < nks; ++j) {
+                            tmem_cp_32x128b_x4(tmem + SFA_COL + 4u * j, desc_sf_block(sfa + 512u * j));
+                            tmem_cp_32x128b_x4(tmem + SFB_COL + 8u * j, desc_sf_block(sfb + 512u * j));
+                            tmem_cp_32x128b_x4(tmem + SFB_COL + 8u * j + 4u, desc_sf_block(sfb + 2048u + 512u * j));
+                        }
+                        for (int j = 0; j < nks; ++j)
+                            mma_nvfp4(tmem + ACC_COL, desc_sw128(sa + 32u * j), desc_sw128(sb + 32u * j), idesc_fp4,
+                                      tmem + SFA_COL + 4u * j, tmem + SFB_COL + 8u * j, (kk > 0 || j > 0) ? 1u : 0u);
+                    } else {
+                        const int c = (kk - n_kb) >> 1;
+                        const int nks = min(4, (a.rank - 64 * c + 15) / 16);
+                        for (int j = 0; j < nks; ++j)
+                            mma_bf16(tmem + ACC_COL, desc_sw128(sa + 32u * j), desc_sw128(sb + 32u * j), idesc_lr,
+                                     1u);
+                    }
+                    tc_commit(&empty[s]);
                 }
-                tc_commit(&empty[s]);
+                if (ok) tc_commit(acc_full);
             }
             s_consumed = it;
-            if (ok) tc_commit(accb);
         }
     } else {
         // ------------------------------------------------------------ epilogue
-        const uint32_t q = warp & 3u;
+        const uint32_t q = warp & 3u;                 // TMEM lane quadrant this warp may read
+        const int half = (int)(warp - 2) >> 2;        // which 128 of the 256 columns
         const int row = (int)(32u * q + lane);
-        const int64_t grow = (int64_t)m0 + row;
-        const bool ok = mbar_wait(accb, 0, kSiteGmAcc);
-        if (!ok) s_failed = 1;
-        tc_fence_after();
         const float S = __fmul_rn(*a.x_scale, *a.w_scale);
-        for (int c = 0; c < BN / 32; ++c) {
-            const int n = n0 + 32 * c;
-            if (n >= a.N) break;
-            uint32_t r[32];
-            tmem_ld_32x32b_x32(tmem + ((32u * q) << 16) + ACC_COL + 32u * c, r);
+        int local = 0;
+        for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++local) {
+            const int m_tile = tile % a.m_tiles, n_tile = tile / a.m_tiles;
+            const int64_t grow = (int64_t)m_tile * BM + row;
+            const int nbase = n_tile * BN + 128 * half;
+            const bool ok = mbar_wait(acc_full, (uint32_t)local & 1u, kSiteGmAcc);
+            if (!ok) {
+                s_failed = 1;
+                break;
+            }
+            tc_fence_after();
+            uint32_t acc[128];
+            tmem_ld_32x32b_x32(tmem + ((32u * q) << 16) + ACC_COL + 128u * half + 0u,
+                               *reinterpret_cast<uint32_t(*)[32]>(acc + 0));
+            tmem_ld_32x32b_x32(tmem + ((32u * q) << 16) + ACC_COL + 128u * half + 32u,
+                               *reinterpret_cast<uint32_t(*)[32]>(acc + 32));
+            tmem_ld_32x32b_x32(tmem + ((32u * q) << 16) + ACC_COL + 128u * half + 64u,
+                               *reinterpret_cast<uint32_t(*)[32]>(acc + 64));
+            tmem_ld_32x32b_x32(tmem + ((32u * q) << 16) + ACC_COL + 128u * half + 96u,
+                               *reinterpret_cast<uint32_t(*)[32]>(acc + 96));
             tmem_ld_wait();
-            if (!ok || grow >= a.M) continue;
-            const int nvec = (a.N - n >= 32) ? 4 : 2;   // N % 16 == 0: a tail chunk has 16 columns
-            float bv[32];
-            if (a.bias) {
-                const uint4* bp = reinterpret_cast<const uint4*>(a.bias + n);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acc_empty);     // TMEM is free for the next tile
+            if (grow >= a.M) continue;
+            __nv_bfloat16* yrow = a.y + grow * (int64_t)a.N;
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const uint4 w = (i < nvec) ? __ldg(bp + i) : make_uint4(0u, 0u, 0u, 0u);
-                    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+            for (int c = 0; c < 8; ++c) {              // 16 columns at a time
+                const int n = nbase + 16 * c;
+                if (n >= a.N) break;                   // N % 16 == 0
+                float bv[16];
+                if (a.bias) {
+                    const uint4 w0 = __ldg(reinterpret_cast<const uint4*>(a.bias + n));
+                    const uint4 w1 = __ldg(reinterpret_cast<const uint4*>(a.bias + n) + 1);
+                    const uint32_t ws[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
-                    for (int p = 0; p < 4; ++p) {
-                        bv[8 * i + 2 * p] = bf16lo_to_f32(ws[p]);
-                        bv[8 * i + 2 * p + 1] = bf16hi_to_f32(ws[p]);
+                    for (int p = 0; p < 8; ++p) {
+                        bv[2 * p] = bf16lo_to_f32(ws[p]);
+                        bv[2 * p + 1] = bf16hi_to_f32(ws[p]);
                     }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) bv[i] = 0.0f;
                 }
-            } else {
+                uint32_t packed[8];
 #pragma unroll
-                for (int i = 0; i < 32; ++i) bv[i] = 0.0f;
+                for (int i = 0; i < 8; ++i) {
+                    const float o0 = fmaf(__uint_as_float(acc[16 * c + 2 * i]), S, bv[2 * i]);
+                    const float o1 = fmaf(__uint_as_float(acc[16 * c + 2 * i + 1]), S, bv[2 * i + 1]);
+                    const __nv_bfloat162 h = __floats2bfloat162_rn(o0, o1);
+                    packed[i] = *reinterpret_cast<const uint32_t*>(&h);
+                }
+                uint4* dst = reinterpret_cast<uint4*>(yrow + n);
+                dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+                dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
             }
-            uint32_t packed[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const float o0 = fmaf(__uint_as_float(r[2 * i]), S, bv[2 * i]);
-                const float o1 = fmaf(__uint_as_float(r[2 * i + 1]), S, bv[2 * i + 1]);
-                const __nv_bfloat162 h = __floats2bfloat162_rn(o0, o1);
-                packed[i] = *reinterpret_cast<const uint32_t*>(&h);
-            }
-            uint4* dst = reinterpret_cast<uint4*>(a.y + grow * (int64_t)a.N + n);
-            for (int i = 0; i < nvec; ++i)
-                dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
         }
     }
 

@@ -14,6 +14,7 @@
 #include "svdq.h"
 #include "sm100_ptx.cuh"
 #include "quantize.cuh"
+#include "quantize_act.cuh"
 #include "gemm_nvfp4.cuh"
 #include "int4.cuh"
 
@@ -220,41 +221,27 @@ svdq_status pack_weight_nvfp4(const void* R, int64_t N, int64_t K, void* w_codes
     return launch_status("quantize_rows_nvfp4_kernel");
 }
 
-// Cluster width for the activation quantizer: enough CTAs to cover the SMs
-// in one wave, a power of two dividing 128 (rows are split evenly for the
-// reduction), at most 8 (portable) and at most the number of column chunks.
-int choose_cluster(int64_t row_blocks, int chunks, int smem_bytes) {
-    int c = 1;
-    while (c < 8 && row_blocks * (c * 2) <= num_sms() && c * 2 <= chunks) c *= 2;
-    // make sure that many clusters can be resident at once; shrink otherwise
-    while (c > 1) {
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3((unsigned)c, (unsigned)row_blocks, 1);
-        cfg.blockDim = dim3(qa::kThreads, 1, 1);
-        cfg.dynamicSmemBytes = (size_t)smem_bytes;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = (unsigned)c;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        int nclusters = 0;
-        if (cudaOccupancyMaxActiveClusters(&nclusters, quantize_act_kernel<kPrecNvfp4>, &cfg) != cudaSuccess) {
-            cudaGetLastError();
-            nclusters = 0;
-        }
-        if ((int64_t)nclusters >= row_blocks) break;
-        c /= 2;
-    }
-    return c;
+// K-split of the activation quantizer: enough CTAs for about one wave on a
+// B200 (a fixed target, so that the workspace size depends on the shape only).
+int quant_splits(int64_t M, int64_t K) {
+    const int64_t row_blocks = (M + qa::kRows - 1) / qa::kRows;
+    int64_t sp = qa::kSplitTarget / row_blocks;
+    sp = std::min<int64_t>(sp, std::min<int64_t>(K / 64, qa::kMaxSplits));
+    return (int)std::max<int64_t>(sp, 1);
+}
+
+size_t quant_workspace_bytes(int64_t M, int64_t K, int rank) {
+    const int sp = quant_splits(M, K);
+    if (rank == 0 || sp == 1) return 0;
+    const int64_t row_blocks = (M + qa::kRows - 1) / qa::kRows;
+    return (size_t)round_up(row_blocks * 4, 256) + (size_t)row_blocks * sp * qa::kRows * rank * 4;
 }
 
 // Activation quantizer launch (both precisions).  x_scale / w_scale are only
 // read by the nvfp4 variant.
 svdq_status quantize_act_launch(int prec, const void* x, int64_t M, int64_t K, const float* inv_lambda,
                                 const float* x_scale, const float* w_scale, const void* L_down_t, int rank,
-                                void* x_codes, void* x_scales, void* lowrank, cudaStream_t st) {
+                                void* x_codes, void* x_scales, void* lowrank, void* workspace, cudaStream_t st) {
     CUtensorMap tm_x, tm_ld;
     if (!make_map(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, 64, 128))
         return SVDQ_ERR_CUDA;
@@ -265,6 +252,8 @@ svdq_status quantize_act_launch(int prec, const void* x, int64_t M, int64_t K, c
     } else {
         tm_ld = tm_x;
     }
+    const int64_t row_blocks = (M + qa::kRows - 1) / qa::kRows;
+    if (row_blocks > 65535) return SVDQ_ERR_UNSUPPORTED_SHAPE;
     QuantActArgs a;
     a.inv_lambda = inv_lambda;
     a.x_scale = x_scale;
@@ -277,44 +266,34 @@ svdq_status quantize_act_launch(int prec, const void* x, int64_t M, int64_t K, c
     a.rank = rank;
     a.rows_pad = (int)round_up(M, 128);
     a.chunks = (int)(K / 64);
+    a.splits = quant_splits(M, K);
+    a.counters = reinterpret_cast<unsigned int*>(workspace);
+    a.partials = workspace ? reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(workspace) +
+                                                       round_up(row_blocks * 4, 256))
+                           : nullptr;
     a.stage_bytes = (uint32_t)qa::kXBytes + (uint32_t)rank * 256u;   // x tile + hi and lo L_down_t tiles
-    const size_t fixed = 1024 + qa::kMaxStages * qa::kCols * 4 + (2 * qa::kMaxStages + 1) * 8 + 16;
+    const size_t fixed = 1024 + qa::kMaxStages * qa::kCols * 4 + 128 * 4 + (2 * qa::kMaxStages + 1) * 8 + 16;
     const int stages = (int)std::min<size_t>(qa::kMaxStages, (kQuantSmemBudget - fixed) / a.stage_bytes);
-    const size_t red_bytes = (size_t)qa::kRows * (rank + 1) * 4;
-    if (stages < 2 || (size_t)stages * a.stage_bytes < red_bytes) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+    if (stages < 2) return SVDQ_ERR_UNSUPPORTED_SHAPE;
     a.stages = stages;
     uint32_t tcols = 32;
     while ((int)tcols < rank) tcols *= 2;
     a.tmem_cols = tcols;
     const size_t smem = fixed + (size_t)stages * a.stage_bytes;
-    const int64_t row_blocks = (M + qa::kRows - 1) / qa::kRows;
-    if (row_blocks > 65535) return SVDQ_ERR_UNSUPPORTED_SHAPE;
-    a.cluster = choose_cluster(row_blocks, a.chunks, (int)smem);
-
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)a.cluster, (unsigned)row_blocks, 1);
-    cfg.blockDim = dim3(qa::kThreads, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = (unsigned)a.cluster;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    const cudaError_t e = prec == kPrecNvfp4 ? cudaLaunchKernelEx(&cfg, quantize_act_kernel<kPrecNvfp4>, tm_x, tm_ld, a)
-                                             : cudaLaunchKernelEx(&cfg, quantize_act_kernel<kPrecInt4>, tm_x, tm_ld, a);
-    if (e != cudaSuccess) return cuda_fail("quantize_act_kernel launch");
-    return SVDQ_OK;
+    const dim3 grid((unsigned)a.splits, (unsigned)row_blocks, 1);
+    if (prec == kPrecNvfp4)
+        quantize_act_kernel<kPrecNvfp4><<<grid, qa::kThreads, smem, st>>>(tm_x, tm_ld, a);
+    else
+        quantize_act_kernel<kPrecInt4><<<grid, qa::kThreads, smem, st>>>(tm_x, tm_ld, a);
+    return launch_status("quantize_act_kernel launch");
 }
 
 svdq_status quantize_act_nvfp4(const void* x, int64_t M, int64_t K, const float* inv_lambda, float* x_scale,
                                int compute_scale, const float* w_scale, const void* L_down_t, int rank,
-                               void* x_codes, void* x_scales, void* lowrank, cudaStream_t st) {
+                               void* x_codes, void* x_scales, void* lowrank, void* workspace, cudaStream_t st) {
     if (compute_scale) SVDQ_TRY(tensor_scale_prepass(x, inv_lambda, M, K, x_scale, st));
     return quantize_act_launch(kPrecNvfp4, x, M, K, inv_lambda, x_scale, w_scale, L_down_t, rank, x_codes, x_scales,
-                               lowrank, st);
+                               lowrank, workspace, st);
 }
 
 // ----------------------------------------------------------- int4 paths
@@ -360,9 +339,11 @@ svdq_status gemm_nvfp4(const void* x_codes, const void* x_scales, const float* x
     a.kg4 = (int)(K / 64);
     a.n_sf_blocks = (int)((N + 127) / 128);
     const int64_t mt = (M + gm::BM - 1) / gm::BM, nt = (N + gm::BN - 1) / gm::BN;
-    if (nt > 65535) return SVDQ_ERR_UNSUPPORTED_SHAPE;
-    gemm_nvfp4_kernel<<<dim3((unsigned)mt, (unsigned)nt, 1), gm::kThreads, gm::SMEM_BYTES, st>>>(tm_xc, tm_wc, tm_L,
-                                                                                             tm_Lup, a);
+    if (mt * nt > (int64_t(1) << 30)) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+    a.m_tiles = (int)mt;
+    a.n_tiles = (int)nt;
+    const int grid = (int)std::min<int64_t>(mt * nt, num_sms());
+    gemm_nvfp4_kernel<<<grid, gm::kThreads, gm::SMEM_BYTES, st>>>(tm_xc, tm_wc, tm_L, tm_Lup, a);
     return launch_status("gemm_nvfp4_kernel launch");
 }
 
@@ -440,10 +421,20 @@ svdq_status svdq_pack_weight(svdq_precision p, int group_size, const void* R, in
     return int4_quantize_rows(R, N, K, w_codes, w_scales, st);
 }
 
+svdq_status svdq_quantize_act_workspace_bytes(svdq_precision p, int64_t M, int64_t K, int rank, size_t* bytes) {
+    if (!bytes) return SVDQ_ERR_INVALID_ARG;
+    if (p != SVDQ_NVFP4 && p != SVDQ_INT4) return SVDQ_ERR_INVALID_ARG;
+    SVDQ_TRY(check_rank(rank));
+    SVDQ_TRY(check_dims(M, K));
+    *bytes = quant_workspace_bytes(M, K, rank);
+    return SVDQ_OK;
+}
+
 svdq_status svdq_quantize_act(svdq_precision p, int group_size, const void* x, int64_t M, int64_t K,
                               const float* inv_lambda, float* x_tensor_scale, int compute_scale,
                               const float* w_tensor_scale, const void* L_down_t, int rank, void* x_codes,
-                              void* x_scales, void* lowrank_act, svdq_stream_t stream) {
+                              void* x_scales, void* lowrank_act, void* workspace, size_t workspace_bytes,
+                              svdq_stream_t stream) {
     SVDQ_TRY(check_precision(p, group_size));
     SVDQ_TRY(check_rank(rank));
     SVDQ_TRY(check_dims(M, K));
@@ -457,13 +448,20 @@ svdq_status svdq_quantize_act(svdq_precision p, int group_size, const void* x, i
         SVDQ_TRY(check_ptr(lowrank_act));
         if (p == SVDQ_NVFP4) SVDQ_TRY(check_ptr(w_tensor_scale));
     }
+    const size_t ws_needed = quant_workspace_bytes(M, K, rank);
+    if (ws_needed > 0) {
+        SVDQ_TRY(check_ptr(workspace));
+        if (workspace_bytes < ws_needed) return SVDQ_ERR_INVALID_ARG;
+    } else {
+        workspace = nullptr;
+    }
     SVDQ_TRY(check_device());
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (p == SVDQ_NVFP4)
         return quantize_act_nvfp4(x, M, K, inv_lambda, x_tensor_scale, compute_scale, w_tensor_scale, L_down_t, rank,
-                                  x_codes, x_scales, lowrank_act, st);
+                                  x_codes, x_scales, lowrank_act, workspace, st);
     return quantize_act_launch(kPrecInt4, x, M, K, inv_lambda, nullptr, nullptr, L_down_t, rank, x_codes, x_scales,
-                               lowrank_act, st);
+                               lowrank_act, workspace, st);
 }
 
 svdq_status svdq_gemm_w4a4(svdq_precision p, int group_size, const void* x_codes, const void* x_scales,

@@ -47,6 +47,7 @@ class QuantizedAct:
     x_scales: torch.Tensor
     x_tensor_scale: torch.Tensor | None
     lowrank_act: torch.Tensor | None
+    workspace: torch.Tensor | None = None   # zero-filled once; the library keeps it zeroed
 
 
 def pack_weight(R: torch.Tensor, lam: torch.Tensor, L_down: torch.Tensor | None, L_up: torch.Tensor | None,
@@ -70,12 +71,14 @@ def pack_weight(R: torch.Tensor, lam: torch.Tensor, L_down: torch.Tensor | None,
 
 def alloc_act(packed: PackedWeight, M: int, device) -> QuantizedAct:
     sz = _lib.svdq_buffer_sizes(packed.precision, M, packed.K, packed.rank)
+    ws = _lib.svdq_quantize_act_workspace_bytes(packed.precision, M, packed.K, packed.rank)
     return QuantizedAct(
         M,
         _empty(sz["codes_bytes"], device),
         _empty(sz["scales_bytes"], device),
         torch.empty(4, dtype=torch.float32, device=device) if packed.precision == "nvfp4" else None,
         torch.empty(2, M, packed.rank, dtype=torch.bfloat16, device=device) if packed.rank else None,
+        torch.zeros(ws, dtype=torch.uint8, device=device) if ws else None,
     )
 
 
@@ -96,7 +99,7 @@ def quantize_act(x: torch.Tensor, packed: PackedWeight, out: QuantizedAct | None
             q.x_tensor_scale.fill_(float(x_tensor_scale))
     _lib.svdq_quantize_act(packed.precision, packed.group_size, x, M, K, packed.inv_lambda, q.x_tensor_scale,
                            compute, packed.w_tensor_scale, packed.L_down_t, packed.rank, q.x_codes, q.x_scales,
-                           q.lowrank_act, stream)
+                           q.lowrank_act, q.workspace, stream=stream)
     return q
 
 

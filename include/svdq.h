@@ -17,7 +17,8 @@
  * Conventions for every call below
  *  - Pointers named "device" are device memory of the current CUDA device,
  *    owned by the caller; the library allocates nothing and keeps no state
- *    between calls (except the device status word, see svdq_device_status).
+ *    between calls (except the device status word, see svdq_device_status,
+ *    and the zeroed counters of a caller-owned workspace).
  *  - All device pointers must be 16-byte aligned.
  *  - bf16 tensors are row-major with the last dimension contiguous.
  *  - Calls are asynchronous on `stream` (NULL = the legacy default stream).
@@ -122,6 +123,13 @@ svdq_status svdq_pack_weight(svdq_precision precision, int group_size,
                              float* inv_lambda, void* L_down_t, void* L_up_t,
                              svdq_stream_t stream);
 
+/* Bytes of the workspace svdq_quantize_act needs for this shape (0 when it
+ * needs none).  The workspace holds fp32 partial sums of the rank-r product
+ * when K is split across several CTAs, plus one counter per 128-row block.
+ * Pure host function; errors as svdq_buffer_sizes. */
+svdq_status svdq_quantize_act_workspace_bytes(svdq_precision precision, int64_t M, int64_t K, int rank,
+                                              size_t* bytes);
+
 /* Activation quantizer, fused with the rank-r down-projection.
  *   x              device bf16 [M, K]
  *   inv_lambda     device fp32 [K] (from svdq_pack_weight)
@@ -131,6 +139,12 @@ svdq_status svdq_pack_weight(svdq_precision precision, int group_size,
  *                  S_x = amax|x/lambda| / 2688 (1 when x == 0) first.
  *   w_tensor_scale device fp32 [1] (nvfp4 with rank > 0): S_w
  *   L_down_t       device bf16 [2, rank, K] (NULL when rank == 0)
+ *   workspace      device, workspace_bytes long (at least what
+ *                  svdq_quantize_act_workspace_bytes reports; NULL when that is
+ *                  0).  It must be zero-filled once before its first use; every
+ *                  call leaves it zero-filled again.  Calls that share a
+ *                  workspace must not overlap on the GPU.  After a call that
+ *                  ends in SVDQ_ERR_TIMEOUT, zero-fill it again.
  * Outputs: x_codes [M, K/2]; x_scales (scales_bytes for M rows, padding rows
  *   written as zeros); lowrank_act bf16 [2, M, rank] (NULL when rank == 0). */
 svdq_status svdq_quantize_act(svdq_precision precision, int group_size,
@@ -138,6 +152,7 @@ svdq_status svdq_quantize_act(svdq_precision precision, int group_size,
                               float* x_tensor_scale, int compute_scale,
                               const float* w_tensor_scale, const void* L_down_t, int rank,
                               void* x_codes, void* x_scales, void* lowrank_act,
+                              void* workspace, size_t workspace_bytes,
                               svdq_stream_t stream);
 
 /* The W4A4 GEMM with the rank-r up-projection and bias fused in.

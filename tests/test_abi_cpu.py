@@ -116,3 +116,13 @@ def test_capability_check_rejects_other_devices(L):
         assert _gemm_status(L) == L.SVDQ_ERR_UNSUPPORTED_DEVICE
     finally:
         L.svdq_debug_override_capability(-1)
+
+
+def test_quantize_act_workspace_bytes(L):
+    # QKV shape: 36 row blocks x 4 K-splits x 128 rows x rank 32 fp32, plus a 256-byte counter block
+    assert L.svdq_quantize_act_workspace_bytes("nvfp4", 4608, 3072, 32) == 256 + 36 * 4 * 128 * 32 * 4
+    # 144 row blocks fill the GPU without a K split: no workspace
+    assert L.svdq_quantize_act_workspace_bytes("nvfp4", 18432, 3072, 32) == 0
+    assert L.svdq_quantize_act_workspace_bytes("int4", 4608, 3072, 0) == 0
+    # the split never exceeds the number of 64-column chunks
+    assert L.svdq_quantize_act_workspace_bytes("nvfp4", 64, 256, 32) == 256 + 1 * 4 * 128 * 32 * 4
