@@ -29,7 +29,8 @@ GROUP_SIZES = {"nvfp4": 16, "int4": 64}
 # Every entry point declared in include/svdq.h.
 EXPORTS = (
     "svdq_status_string", "svdq_abi_version", "svdq_last_error", "svdq_buffer_sizes", "svdq_pack_weight",
-    "svdq_quantize_act_workspace_bytes", "svdq_quantize_act", "svdq_gemm_w4a4", "svdq_device_status",
+    "svdq_quantize_act_workspace_bytes", "svdq_quantize_act", "svdq_quantize_act_noalloc", "svdq_gemm_w4a4",
+    "svdq_device_status",
     "svdq_debug_set_wait_limit_ns", "svdq_debug_timeout_probe", "svdq_debug_override_capability",
 )
 
@@ -68,6 +69,8 @@ def _load():
     lib.svdq_quantize_act_workspace_bytes.restype = I
     lib.svdq_quantize_act.argtypes = [I, I, P, I64, I64, P, P, I, P, P, I, P, P, P, P, ctypes.c_size_t, P]
     lib.svdq_quantize_act.restype = I
+    lib.svdq_quantize_act_noalloc.argtypes = [I, I, P, I64, I64, P, P, I, P, P, I, P, P, P, P]
+    lib.svdq_quantize_act_noalloc.restype = I
     lib.svdq_gemm_w4a4.argtypes = [I, I, P, P, P, I64, P, P, P, I64, I64, P, P, I, P, P, P]
     lib.svdq_gemm_w4a4.restype = I
     lib.svdq_device_status.argtypes = [I, ctypes.POINTER(ctypes.c_int)]
@@ -151,6 +154,16 @@ def svdq_quantize_act(precision, group_size, x, M, K, inv_lambda, x_tensor_scale
                                  _ptr(x_tensor_scale), int(bool(compute_scale)), _ptr(w_tensor_scale),
                                  _ptr(L_down_t), int(rank), _ptr(x_codes), _ptr(x_scales), _ptr(lowrank_act),
                                  _ptr(workspace), int(workspace_bytes), _stream(stream)), "svdq_quantize_act")
+
+
+def svdq_quantize_act_noalloc(precision, group_size, x, M, K, inv_lambda, x_tensor_scale, compute_scale,
+                              w_tensor_scale, L_down_t, rank, x_codes, x_scales, lowrank_act, stream=None) -> None:
+    """svdq_quantize_act with the library's built-in workspace (for callers that cannot allocate)."""
+    _check(lib.svdq_quantize_act_noalloc(_prec(precision), int(group_size), _ptr(x), int(M), int(K),
+                                         _ptr(inv_lambda), _ptr(x_tensor_scale), int(bool(compute_scale)),
+                                         _ptr(w_tensor_scale), _ptr(L_down_t), int(rank), _ptr(x_codes),
+                                         _ptr(x_scales), _ptr(lowrank_act), _stream(stream)),
+           "svdq_quantize_act_noalloc")
 
 
 def svdq_gemm_w4a4(precision, group_size, x_codes, x_scales, x_tensor_scale, M, w_codes, w_scales,

@@ -359,6 +359,42 @@ __global__ void timeout_probe_kernel() {
     __syncthreads();
 }
 
+// ------------------------------------------------- no-allocation workspace
+// Workspace of svdq_quantize_act_noalloc: a file-scope device array, so that
+// callers without a device allocator need not provide one.  Every GPU that
+// loads the library holds it until the process exits.
+constexpr size_t kNoAllocWorkspaceBytes = size_t(8) << 20;   // 8 MiB
+std::mutex g_noalloc_mutex;
+void* g_noalloc_addr[kMaxDevices];
+
+}  // namespace
+
+static __device__ __align__(256) unsigned char g_noalloc_workspace[kNoAllocWorkspaceBytes];
+
+namespace {
+// Device address of g_noalloc_workspace on the current device, looked up once
+// per device with that device current (the host-side name of the array is
+// only a stand-in and must never be handed to a kernel).
+svdq_status noalloc_workspace_address(void** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        return SVDQ_ERR_UNSUPPORTED_DEVICE;
+    }
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (!g_noalloc_addr[dev]) {
+        void* p = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_workspace);
+        if (e != cudaSuccess || p == nullptr) {
+            note_error(e == cudaSuccess ? cudaErrorUnknown : e, "cudaGetSymbolAddress(no-alloc workspace)");
+            cudaGetLastError();
+            return SVDQ_ERR_CUDA;
+        }
+        g_noalloc_addr[dev] = p;
+    }
+    *out = g_noalloc_addr[dev];
+    return SVDQ_OK;
+}
 }  // namespace
 }  // namespace svdq
 
@@ -462,6 +498,44 @@ svdq_status svdq_quantize_act(svdq_precision p, int group_size, const void* x, i
                                   x_codes, x_scales, lowrank_act, workspace, st);
     return quantize_act_launch(kPrecInt4, x, M, K, inv_lambda, nullptr, nullptr, L_down_t, rank, x_codes, x_scales,
                                lowrank_act, workspace, st);
+}
+
+svdq_status svdq_quantize_act_noalloc(svdq_precision p, int group_size, const void* x, int64_t M, int64_t K,
+                                      const float* inv_lambda, float* x_tensor_scale, int compute_scale,
+                                      const float* w_tensor_scale, const void* L_down_t, int rank, void* x_codes,
+                                      void* x_scales, void* lowrank_act, svdq_stream_t stream) {
+    SVDQ_TRY(check_precision(p, group_size));
+    SVDQ_TRY(check_rank(rank));
+    SVDQ_TRY(check_dims(M, K));
+    SVDQ_TRY(check_ptr(x));
+    SVDQ_TRY(check_ptr(inv_lambda));
+    SVDQ_TRY(check_ptr(x_codes));
+    SVDQ_TRY(check_ptr(x_scales));
+    if (p == SVDQ_NVFP4) SVDQ_TRY(check_ptr(x_tensor_scale));
+    if (rank > 0) {
+        SVDQ_TRY(check_ptr(L_down_t));
+        SVDQ_TRY(check_ptr(lowrank_act));
+        if (p == SVDQ_NVFP4) SVDQ_TRY(check_ptr(w_tensor_scale));
+    }
+    const size_t need = quant_workspace_bytes(M, K, rank);
+    if (need > kNoAllocWorkspaceBytes) {
+        snprintf(g_last_error, sizeof(g_last_error),
+                 "svdq_quantize_act_noalloc: this shape needs %zu bytes of workspace, more than the built-in %zu",
+                 need, kNoAllocWorkspaceBytes);
+        return SVDQ_ERR_UNSUPPORTED_SHAPE;
+    }
+    void* ws = nullptr;
+    if (need > 0) {
+        SVDQ_TRY(check_device());
+        SVDQ_TRY(noalloc_workspace_address(&ws));
+        // the array keeps the previous call's contents: its counters must start at zero
+        const int64_t row_blocks = (M + qa::kRows - 1) / qa::kRows;
+        if (cudaMemsetAsync(ws, 0, (size_t)round_up(row_blocks * 4, 256), reinterpret_cast<cudaStream_t>(stream)) !=
+            cudaSuccess)
+            return cuda_fail("cudaMemsetAsync(no-alloc workspace counters)");
+    }
+    return svdq_quantize_act(p, group_size, x, M, K, inv_lambda, x_tensor_scale, compute_scale, w_tensor_scale,
+                             L_down_t, rank, x_codes, x_scales, lowrank_act, ws, need, stream);
 }
 
 svdq_status svdq_gemm_w4a4(svdq_precision p, int group_size, const void* x_codes, const void* x_scales,

@@ -155,6 +155,31 @@ svdq_status svdq_quantize_act(svdq_precision precision, int group_size,
                               void* workspace, size_t workspace_bytes,
                               svdq_stream_t stream);
 
+/* svdq_quantize_act for callers that cannot allocate device memory: code
+ * that only receives input and output buffers from a host framework and has
+ * no device allocator of its own (plug-in or custom-operator interfaces), and
+ * code that must keep cudaMalloc / cudaFree, which synchronise the whole
+ * device, off a latency-critical path.  (This entry point has no counterpart
+ * on the pages; it is a convenience of this library.)
+ * Arguments, outputs and errors are those of svdq_quantize_act, without the
+ * workspace: the K-split workspace is a library-owned 8 MiB device array
+ * (file-scope, so every GPU that loads the library holds it until the process
+ * exits).  Shapes whose workspace, as reported by
+ * svdq_quantize_act_workspace_bytes, exceeds 8 MiB are rejected with
+ * SVDQ_ERR_UNSUPPORTED_SHAPE, and svdq_last_error() says so.
+ * The first call on each device looks up the array's device address with
+ * that device current; make that first call before any stream capture.
+ * Each call zero-fills the array's counters on `stream` before its launch.
+ * All calls share the one array and it keeps the last call's contents, so
+ * calls that overlap on the GPU (other streams or threads) race on it.
+ * Allocates nothing: no cudaMalloc, cudaFree or allocating library routine. */
+svdq_status svdq_quantize_act_noalloc(svdq_precision precision, int group_size,
+                                      const void* x, int64_t M, int64_t K, const float* inv_lambda,
+                                      float* x_tensor_scale, int compute_scale,
+                                      const float* w_tensor_scale, const void* L_down_t, int rank,
+                                      void* x_codes, void* x_scales, void* lowrank_act,
+                                      svdq_stream_t stream);
+
 /* The W4A4 GEMM with the rank-r up-projection and bias fused in.
  *   y[m, n] = bf16( S_x S_w sum_k xq[m,k] wq[n,k] + sum_j L[m,j] L_up[j,n] + b[n] )   (nvfp4)
  *   y[m, n] = bf16( sum_g sx[m,g] sw[n,g] sum_{k in g} qx qw + sum_j L[m,j] L_up[j,n] + b[n] )  (int4)
