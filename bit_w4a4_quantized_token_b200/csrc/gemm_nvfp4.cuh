@@ -9,11 +9,13 @@
 // page "Nunchaku Lite" ("Supported quantization types" table).
 //
 // Persistent kernel, one CTA per SM, 128 x 256 output tiles taken round-robin.
-// Warp 0 issues TMA loads (codes with 128-byte swizzle, scale blocks with bulk
-// copies) into a ring of stages that runs across tile boundaries; warp 1
-// copies each stage's scale blocks into TMEM and issues tcgen05.mma
-// (kind::mxf4nvf4, K = 64 per instruction; kind::f16 for the rank-r chunks);
-// eight epilogue warps pull the finished accumulator out of TMEM into
+// Three producer warps fill a ring of stages that runs across tile
+// boundaries: warp 0 loads the activation codes (TMA, 128-byte swizzle),
+// warp 1 the weight codes, warp 3 the two operands' scale blocks (bulk
+// copies); one issuing thread cannot keep the tensor core fed on its own.
+// Warp 2 copies each stage's scale blocks into TMEM and issues tcgen05.mma
+// (kind::mxf4nvf4, K = 64 per instruction; kind::f16 for the rank-r chunks).
+// Eight epilogue warps (4..11) pull the finished accumulator out of TMEM into
 // registers, hand TMEM back to the MMA warp at once, and then scale, add the
 // bias and store bf16 while the next tile's MMAs run.
 #pragma once
@@ -31,7 +33,9 @@ constexpr int SFA_BYTES = 4 * 512;            // 4 scale blocks: 128 rows x 16 g
 constexpr int SFB_BYTES = 8 * 512;            // 2 row blocks x 4 scale blocks
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
 constexpr int kEpiWarps = 8;                  // 2 per TMEM lane quadrant, 128 columns each
-constexpr int kThreads = 64 + 32 * kEpiWarps;
+constexpr int kEpiWarp0 = 4;                  // first epilogue warp (a multiple of 4)
+constexpr int kThreads = 32 * (kEpiWarp0 + kEpiWarps);
+constexpr uint32_t kMmaWarp = 2;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COL = 0;               // 256 fp32 columns
 constexpr uint32_t SFA_COL = 256;             // 4 k-steps x 4 columns
@@ -66,7 +70,8 @@ __global__ void __launch_bounds__(gm::kThreads, 1)
     uint64_t* acc_full = empty + kStages;
     uint64_t* acc_empty = acc_full + 1;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
-    __shared__ int s_issued, s_consumed, s_failed;
+    __shared__ int s_failed;
+    __shared__ int s_issued[gm::kStages];   // phases started in each stage (by the A-code producer)
 
     const uint32_t warp = warp_id(), lane = lane_id();
     const int n_kb = (a.K + 255) / 256;
@@ -76,13 +81,12 @@ __global__ void __launch_bounds__(gm::kThreads, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(&full[s], 1);
+            mbar_init(&full[s], 3);               // one arrival per producer warp
             mbar_init(&empty[s], 1);
         }
         mbar_init(acc_full, 1);
         mbar_init(acc_empty, kEpiWarps);
-        s_issued = 0;
-        s_consumed = 0;
+        for (int s = 0; s < kStages; ++s) s_issued[s] = 0;
         s_failed = 0;
         fence_barrier_init();
     }
@@ -94,7 +98,7 @@ __global__ void __launch_bounds__(gm::kThreads, 1)
             prefetch_tensormap(&tm_Lup);
         }
     }
-    if (warp == 1) {
+    if (warp == kMmaWarp) {
         tmem_alloc(tmem_slot, TMEM_COLS);
         tmem_relinquish();
     }
@@ -103,9 +107,10 @@ __global__ void __launch_bounds__(gm::kThreads, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 0) {
-        // ------------------------------------------------------------ producer
+    if (warp == 0 || warp == 1 || warp == 3) {
+        // ----------------------------------------------------------- producers
         if (lane == 0) {
+            const int role = warp == 0 ? 0 : (warp == 1 ? 1 : 2);   // A codes, B codes, scale blocks
             int it = 0;   // position in the stage ring, continued across tiles
             bool ok = true;
             for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
@@ -123,30 +128,43 @@ __global__ void __launch_bounds__(gm::kThreads, 1)
                     }
                     uint8_t* sa = smem + (size_t)s * STAGE_BYTES;
                     uint8_t* sb = sa + A_BYTES;
+                    uint8_t* sfa = sb + B_BYTES;
+                    uint8_t* sfb = sfa + SFA_BYTES;
                     if (kk < n_kb) {
                         const int kb = kk;
-                        const int natoms = min(4, a.kg4 - 4 * kb);
-                        const uint32_t sf_bytes = (uint32_t)natoms * 512u;
-                        mbar_arrive_expect_tx(&full[s], A_BYTES + B_BYTES + sf_bytes * (1u + (uint32_t)nbv));
-                        tma_load_2d(sa, &tm_xc, &full[s], kb * BK_BYTES, m0);
-                        tma_load_2d(sb, &tm_wc, &full[s], kb * BK_BYTES, n0);
-                        uint8_t* sfa = sb + B_BYTES;
-                        uint8_t* sfb = sfa + SFA_BYTES;
-                        bulk_load(sfa, a.x_scales + ((int64_t)m_tile * a.kg4 + 4 * kb) * 512, sf_bytes, &full[s]);
-                        for (int rb = 0; rb < nbv; ++rb)
-                            bulk_load(sfb + rb * 2048, a.w_scales + ((int64_t)(nb0 + rb) * a.kg4 + 4 * kb) * 512,
-                                      sf_bytes, &full[s]);
+                        if (role == 0) {
+                            mbar_arrive_expect_tx(&full[s], A_BYTES);
+                            tma_load_2d(sa, &tm_xc, &full[s], kb * BK_BYTES, m0);
+                            reinterpret_cast<volatile int*>(s_issued)[s] += 1;
+                        } else if (role == 1) {
+                            mbar_arrive_expect_tx(&full[s], B_BYTES);
+                            tma_load_2d(sb, &tm_wc, &full[s], kb * BK_BYTES, n0);
+                        } else {
+                            const int natoms = min(4, a.kg4 - 4 * kb);
+                            const uint32_t sf_bytes = (uint32_t)natoms * 512u;
+                            mbar_arrive_expect_tx(&full[s], sf_bytes * (1u + (uint32_t)nbv));
+                            bulk_load(sfa, a.x_scales + ((int64_t)m_tile * a.kg4 + 4 * kb) * 512, sf_bytes, &full[s]);
+                            for (int rb = 0; rb < nbv; ++rb)
+                                bulk_load(sfb + rb * 2048, a.w_scales + ((int64_t)(nb0 + rb) * a.kg4 + 4 * kb) * 512,
+                                          sf_bytes, &full[s]);
+                        }
                     } else {
                         const int c = (kk - n_kb) >> 1, part = (kk - n_kb) & 1;
-                        mbar_arrive_expect_tx(&full[s], A_BYTES + B_BYTES);
-                        tma_load_3d(sa, &tm_L, &full[s], c * 64, m0, part);
-                        tma_load_2d(sb, &tm_Lup, &full[s], c * 64, n0);
+                        if (role == 0) {
+                            mbar_arrive_expect_tx(&full[s], A_BYTES);
+                            tma_load_3d(sa, &tm_L, &full[s], c * 64, m0, part);
+                            reinterpret_cast<volatile int*>(s_issued)[s] += 1;
+                        } else if (role == 1) {
+                            mbar_arrive_expect_tx(&full[s], B_BYTES);
+                            tma_load_2d(sb, &tm_Lup, &full[s], c * 64, n0);
+                        } else {
+                            mbar_arrive(&full[s]);
+                        }
                     }
                 }
             }
-            s_issued = it;
         }
-    } else if (warp == 1) {
+    } else if (warp == kMmaWarp) {
         // ---------------------------------------------------------- MMA issuer
         if (lane == 0) {
             const uint32_t idesc_fp4 = idesc_nvfp4(BN);
@@ -194,12 +212,11 @@ __global__ void __launch_bounds__(gm::kThreads, 1)
                 }
                 if (ok) tc_commit(acc_full);
             }
-            s_consumed = it;
         }
-    } else {
+    } else if (warp >= (uint32_t)kEpiWarp0) {
         // ------------------------------------------------------------ epilogue
         const uint32_t q = warp & 3u;                 // TMEM lane quadrant this warp may read
-        const int half = (int)(warp - 2) >> 2;        // which 128 of the 256 columns
+        const int half = (int)(warp - kEpiWarp0) >> 2;   // which 128 of the 256 columns
         const int row = (int)(32u * q + lane);
         const float S = __fmul_rn(*a.x_scale, *a.w_scale);
         int local = 0;
@@ -264,12 +281,14 @@ __global__ void __launch_bounds__(gm::kThreads, 1)
     __syncthreads();
     if (s_failed && warp == 0 && lane == 0) {
         // on a timeout, let the loads already issued land before the CTA exits
-        for (int it = s_consumed; it < s_issued; ++it)
-            mbar_wait(&full[it % kStages], (uint32_t)(it / kStages) & 1u, kSiteGmDrain);
+        for (int s = 0; s < kStages; ++s) {
+            const int n = reinterpret_cast<volatile int*>(s_issued)[s];
+            if (n > 0) mbar_wait(&full[s], (uint32_t)(n - 1) & 1u, kSiteGmDrain);
+        }
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 1) {
+    if (warp == kMmaWarp) {
         tc_fence_after();
         tmem_dealloc(tmem, TMEM_COLS);
     }

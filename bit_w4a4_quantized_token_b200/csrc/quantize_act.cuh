@@ -2,12 +2,14 @@
 // the rank-r down-projection (sm_100a).
 //
 // One CTA owns a 128-row block of x and a contiguous range of 64-column
-// chunks.  Warp 0 streams each chunk (a 128 x 64 bf16 tile, 128-byte
-// swizzled) plus the matching hi/lo tiles of L_down / lambda and 64 values of
-// 1/lambda into a ring of shared-memory stages with TMA.  Sixteen quantizer
-// warps turn the tile into 4-bit codes and group scales (one thread per row
-// and group of 16 columns).  Warp 1 issues tcgen05.mma on the same tile:
-// x (bf16, exact) times the hi and lo parts of L_down / lambda, fp32 in TMEM.
+// chunks.  Three producer warps (0, 2, 3; chunks taken in turn, since one
+// issuing thread cannot stream fast enough) load each chunk -- a 128 x 64
+// bf16 tile, 128-byte swizzled -- and the matching hi/lo tiles of
+// L_down / lambda into a ring of shared-memory stages with TMA; 1/lambda for
+// the CTA's columns is loaded once.  Sixteen quantizer warps (4..19) turn the
+// tile into 4-bit codes and group scales (one thread per row and group of 16
+// columns).  Warp 1 issues tcgen05.mma on the same tile: x (bf16, exact)
+// times the hi and lo parts of L_down / lambda, fp32 in TMEM.
 // When K is split over several CTAs, each writes its fp32 partial of the
 // rank-r product to a workspace and the last CTA of the row block (found with
 // a counter it resets afterwards) adds the partials in split order, so the
@@ -22,7 +24,9 @@ constexpr int kRows = 128;              // rows per CTA (= TMEM lanes of the MMA
 constexpr int kCols = 64;               // columns per stage (128 B of bf16)
 constexpr int kXBytes = kRows * kCols * 2;
 constexpr int kWorkerWarps = 16;
-constexpr int kThreads = 64 + 32 * kWorkerWarps;   // warp 0 TMA, warp 1 MMA + TMEM, 16 quantizer warps
+constexpr int kWorker0 = 4;             // first quantizer warp (a multiple of 4: TMEM lane quadrants)
+constexpr int kProducers = 3;           // warps 0, 2, 3
+constexpr int kThreads = 32 * (kWorker0 + kWorkerWarps);   // warp 1: MMA + TMEM
 constexpr int kMaxStages = 8;
 constexpr int kMaxSplits = 16;
 constexpr int kSplitTarget = 148;       // CTAs wanted for one wave (SMs of a B200)
@@ -44,6 +48,7 @@ struct QuantActArgs {
     int chunks;                // K / 64
     int splits;                // CTAs sharing one 128-row block
     int stages;
+    int max_chunks;            // ceil(chunks / splits): 1/lambda values kept in shared memory / 64
     uint32_t stage_bytes;      // x tile + hi and lo L_down_t tiles (rank x 128 B each)
     uint32_t tmem_cols;
 };
@@ -72,13 +77,14 @@ __global__ void __launch_bounds__(qa::kThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int nst = a.stages;
-    float* invl = reinterpret_cast<float*>(smem + (size_t)nst * a.stage_bytes);   // [kMaxStages][64]
-    float* inv_tab = invl + qa::kMaxStages * qa::kCols;                            // [128] 1/(e*S)
+    float* invl = reinterpret_cast<float*>(smem + (size_t)nst * a.stage_bytes);   // [max_chunks * 64]
+    float* inv_tab = invl + a.max_chunks * qa::kCols;                              // [128] 1/(e*S)
     uint64_t* full = reinterpret_cast<uint64_t*>(inv_tab + 128);
     uint64_t* empty = full + qa::kMaxStages;
     uint64_t* accb = empty + qa::kMaxStages;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accb + 1);
-    __shared__ int s_issued, s_failed, s_last;
+    __shared__ int s_failed, s_last;
+    __shared__ int s_issued[qa::kMaxStages];   // loads issued into each stage (phases started)
 
     const uint32_t warp = warp_id(), lane = lane_id();
     const int split = blockIdx.x, rb = blockIdx.y;
@@ -91,10 +97,10 @@ __global__ void __launch_bounds__(qa::kThreads, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < nst; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], qa::kWorkerWarps + (has_lr ? 1u : 0u));
+            mbar_init(&empty[s], qa::kWorkerWarps + (has_lr ? 1u : 0u));   // quantizer warps + MMA commit
         }
         mbar_init(accb, 1);
-        s_issued = 0;
+        for (int s = 0; s < qa::kMaxStages; ++s) s_issued[s] = 0;
         s_failed = 0;
         s_last = 0;
         fence_barrier_init();
@@ -107,24 +113,30 @@ __global__ void __launch_bounds__(qa::kThreads, 1)
         tmem_alloc(tmem_slot, a.tmem_cols);
         tmem_relinquish();
     }
-    if (PREC == kPrecNvfp4 && threadIdx.x >= 64 && threadIdx.x < 64 + 128) {
-        // reciprocals of the 128 possible decoded group scales e * S
-        const int e = threadIdx.x - 64;
-        const float dec = __fmul_rn(e4m3_to_f32((uint32_t)e), *a.x_scale);
-        inv_tab[e] = (dec == 0.0f) ? 0.0f : __frcp_rn(dec);
+    if (warp >= (uint32_t)qa::kWorker0) {
+        const int t = (int)threadIdx.x - 32 * qa::kWorker0;
+        // 1/lambda for this CTA's columns, once
+        const float4* src = reinterpret_cast<const float4*>(a.inv_lambda + (int64_t)c_lo * qa::kCols);
+        for (int i = t; i < n_it * (qa::kCols / 4); i += 32 * qa::kWorkerWarps)
+            reinterpret_cast<float4*>(invl)[i] = __ldg(src + i);
+        if (PREC == kPrecNvfp4 && t < 128) {
+            // reciprocals of the 128 possible decoded group scales e * S
+            const float dec = __fmul_rn(e4m3_to_f32((uint32_t)t), *a.x_scale);
+            inv_tab[t] = (dec == 0.0f) ? 0.0f : __frcp_rn(dec);
+        }
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = has_lr ? *tmem_slot : 0u;
 
-    if (warp == 0) {
-        // ---------------------------------------------------------- producer
+    if (warp == 0 || warp == 2 || warp == 3) {
+        // ---------------------------------------------------------- producers
         if (lane == 0) {
-            const uint32_t ld_tile = (uint32_t)a.rank * 128u;
-            const uint32_t bytes = qa::kXBytes + (has_lr ? 2u * ld_tile : 0u) + qa::kCols * 4u;
-            int it = 0;
-            for (; it < n_it; ++it) {
+            const int pid = warp == 0 ? 0 : (int)warp - 1;     // 0, 1, 2
+            const uint32_t bytes = qa::kXBytes + (has_lr ? 2u * (uint32_t)a.rank * 128u : 0u);
+            int it = pid;
+            for (; it < n_it; it += qa::kProducers) {
                 const int s = it % nst;
                 const uint32_t ph = (uint32_t)(it / nst) & 1u;
                 if (!mbar_wait(&empty[s], ph ^ 1u, kSiteQaEmpty)) {
@@ -135,18 +147,18 @@ __global__ void __launch_bounds__(qa::kThreads, 1)
                 uint8_t* st = smem + (size_t)s * a.stage_bytes;
                 mbar_arrive_expect_tx(&full[s], bytes);
                 tma_load_2d(st, &tm_x, &full[s], kc * qa::kCols, m0);
-                if (has_lr) {
-                    tma_load_3d(st + qa::kXBytes, &tm_ld, &full[s], kc * qa::kCols, 0, 0);
-                    tma_load_3d(st + qa::kXBytes + ld_tile, &tm_ld, &full[s], kc * qa::kCols, 0, 1);
-                }
-                bulk_load(invl + s * qa::kCols, a.inv_lambda + (int64_t)kc * qa::kCols, qa::kCols * 4, &full[s]);
+                if (has_lr) tma_load_3d(st + qa::kXBytes, &tm_ld, &full[s], kc * qa::kCols, 0, 0);   // hi and lo
+                // a stage is refilled only after its previous load was consumed: no concurrent updates
+                reinterpret_cast<volatile int*>(s_issued)[s] += 1;
             }
-            s_issued = it;
         }
     } else if (warp == 1) {
         // --------------------------------------------------- rank-r MMA issuer
         if (has_lr && lane == 0) {
-            const uint32_t idesc = idesc_bf16_f32((uint32_t)a.rank);
+            // B = the hi and lo tiles stacked (2r rows): one MMA per k-step when
+            // 2r <= 256, with hi and lo accumulated in separate column ranges
+            const bool fused = 2 * a.rank <= 256;
+            const uint32_t idesc = idesc_bf16_f32((uint32_t)(fused ? 2 * a.rank : a.rank));
             bool ok = true;
             for (int it = 0; it < n_it; ++it) {
                 const int s = it % nst;
@@ -159,20 +171,27 @@ __global__ void __launch_bounds__(qa::kThreads, 1)
                 tc_fence_after();
                 const uint32_t xa = smem_u32(smem + (size_t)s * a.stage_bytes);
                 const uint32_t lb = xa + qa::kXBytes;
-#pragma unroll
-                for (int part = 0; part < 2; ++part)
+                if (fused) {
 #pragma unroll
                     for (int j = 0; j < 4; ++j)
-                        mma_bf16(tmem, desc_sw128(xa + 32u * j),
-                                 desc_sw128(lb + (uint32_t)part * (uint32_t)a.rank * 128u + 32u * j), idesc,
-                                 (it > 0 || part > 0 || j > 0) ? 1u : 0u);
+                        mma_bf16(tmem, desc_sw128(xa + 32u * j), desc_sw128(lb + 32u * j), idesc,
+                                 (it > 0 || j > 0) ? 1u : 0u);
+                } else {
+#pragma unroll
+                    for (int part = 0; part < 2; ++part)
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            mma_bf16(tmem + (uint32_t)part * (uint32_t)a.rank, desc_sw128(xa + 32u * j),
+                                     desc_sw128(lb + (uint32_t)part * (uint32_t)a.rank * 128u + 32u * j), idesc,
+                                     (it > 0 || j > 0) ? 1u : 0u);
+                }
                 tc_commit(&empty[s]);
             }
             if (ok) tc_commit(accb);
         }
-    } else {
+    } else if (warp >= (uint32_t)qa::kWorker0) {
         // --------------------------------------------------------- quantizers
-        const int t = (int)threadIdx.x - 64;
+        const int t = (int)threadIdx.x - 32 * qa::kWorker0;
         const int row = t >> 2, g = t & 3;            // 4 lanes per row: one group of 16 columns each
         const int64_t grow = (int64_t)m0 + row;
         float S = 1.0f, six_s = 6.0f;
@@ -190,25 +209,17 @@ __global__ void __launch_bounds__(qa::kThreads, 1)
             const uint8_t* xr = smem + (size_t)s * a.stage_bytes + row * 128;
             const uint4 r0 = *reinterpret_cast<const uint4*>(xr + (((2 * g) ^ (row & 7)) << 4));
             const uint4 r1 = *reinterpret_cast<const uint4*>(xr + (((2 * g + 1) ^ (row & 7)) << 4));
-            const float4* il = reinterpret_cast<const float4*>(invl + s * qa::kCols + 16 * g);
+            const float4* il = reinterpret_cast<const float4*>(invl + it * qa::kCols + 16 * g);
             const float4 l0 = il[0], l1 = il[1], l2 = il[2], l3 = il[3];
             float v[16];
-            v[0] = __fmul_rn(bf16lo_to_f32(r0.x), l0.x);
-            v[1] = __fmul_rn(bf16hi_to_f32(r0.x), l0.y);
-            v[2] = __fmul_rn(bf16lo_to_f32(r0.y), l0.z);
-            v[3] = __fmul_rn(bf16hi_to_f32(r0.y), l0.w);
-            v[4] = __fmul_rn(bf16lo_to_f32(r0.z), l1.x);
-            v[5] = __fmul_rn(bf16hi_to_f32(r0.z), l1.y);
-            v[6] = __fmul_rn(bf16lo_to_f32(r0.w), l1.z);
-            v[7] = __fmul_rn(bf16hi_to_f32(r0.w), l1.w);
-            v[8] = __fmul_rn(bf16lo_to_f32(r1.x), l2.x);
-            v[9] = __fmul_rn(bf16hi_to_f32(r1.x), l2.y);
-            v[10] = __fmul_rn(bf16lo_to_f32(r1.y), l2.z);
-            v[11] = __fmul_rn(bf16hi_to_f32(r1.y), l2.w);
-            v[12] = __fmul_rn(bf16lo_to_f32(r1.z), l3.x);
-            v[13] = __fmul_rn(bf16hi_to_f32(r1.z), l3.y);
-            v[14] = __fmul_rn(bf16lo_to_f32(r1.w), l3.z);
-            v[15] = __fmul_rn(bf16hi_to_f32(r1.w), l3.w);
+            fmul2_rn(bf16lo_to_f32(r0.x), bf16hi_to_f32(r0.x), l0.x, l0.y, v[0], v[1]);
+            fmul2_rn(bf16lo_to_f32(r0.y), bf16hi_to_f32(r0.y), l0.z, l0.w, v[2], v[3]);
+            fmul2_rn(bf16lo_to_f32(r0.z), bf16hi_to_f32(r0.z), l1.x, l1.y, v[4], v[5]);
+            fmul2_rn(bf16lo_to_f32(r0.w), bf16hi_to_f32(r0.w), l1.z, l1.w, v[6], v[7]);
+            fmul2_rn(bf16lo_to_f32(r1.x), bf16hi_to_f32(r1.x), l2.x, l2.y, v[8], v[9]);
+            fmul2_rn(bf16lo_to_f32(r1.y), bf16hi_to_f32(r1.y), l2.z, l2.w, v[10], v[11]);
+            fmul2_rn(bf16lo_to_f32(r1.z), bf16hi_to_f32(r1.z), l3.x, l3.y, v[12], v[13]);
+            fmul2_rn(bf16lo_to_f32(r1.w), bf16hi_to_f32(r1.w), l3.z, l3.w, v[14], v[15]);
             const int kc = c_lo + it;
             float amax = 0.0f;
 #pragma unroll
@@ -219,10 +230,10 @@ __global__ void __launch_bounds__(qa::kThreads, 1)
                 const float inv = inv_tab[eb];
                 float q[8];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) q[i] = __fmul_rn(v[i], inv);
+                for (int i = 0; i < 8; i += 2) fmul2_rn(v[i], v[i + 1], inv, inv, q[i], q[i + 1]);
                 c0 = cvt_e2m1x8(q);
 #pragma unroll
-                for (int i = 0; i < 8; ++i) q[i] = __fmul_rn(v[8 + i], inv);
+                for (int i = 0; i < 8; i += 2) fmul2_rn(v[8 + i], v[9 + i], inv, inv, q[i], q[i + 1]);
                 c1 = cvt_e2m1x8(q);
                 // the four scale bytes of this row's chunk are adjacent: gather them in lane g == 0
                 const uint32_t b1 = __shfl_down_sync(0xffffffffu, eb, 1);
@@ -261,8 +272,8 @@ __global__ void __launch_bounds__(qa::kThreads, 1)
     }
 
     // ------------------------------------------------- rank-r result of the CTA
-    if (has_lr && warp >= 2 && warp < 6) {
-        // warps 2..5 cover the four TMEM lane quadrants: one thread per row,
+    if (has_lr && warp >= (uint32_t)qa::kWorker0 && warp < (uint32_t)qa::kWorker0 + 4) {
+        // four warps cover the four TMEM lane quadrants: one thread per row,
         // 16 columns at a time
         const uint32_t q = warp & 3u;
         const int row = (int)(32u * q + lane);
@@ -275,12 +286,14 @@ __global__ void __launch_bounds__(qa::kThreads, 1)
         const int64_t plane = (int64_t)a.M * a.rank;
         float* mine = a.partials + (((int64_t)rb * a.splits + split) * qa::kRows + row) * a.rank;
         for (int c0 = 0; c0 < a.rank; c0 += 16) {
-            uint32_t r16[16];
-            tmem_ld_32x32b_x16(tmem + ((32u * q) << 16) + (uint32_t)c0, r16);
+            uint32_t r16[16], s16[16];
+            tmem_ld_32x32b_x16(tmem + ((32u * q) << 16) + (uint32_t)c0, r16);              // x . hi
+            tmem_ld_32x32b_x16(tmem + ((32u * q) << 16) + (uint32_t)(a.rank + c0), s16);   // x . lo
             tmem_ld_wait();
             float v16[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) v16[i] = ok ? __uint_as_float(r16[i]) : 0.0f;
+            for (int i = 0; i < 16; ++i)
+                v16[i] = ok ? __fadd_rn(__uint_as_float(r16[i]), __uint_as_float(s16[i])) : 0.0f;
             if (a.splits == 1) {
                 if (grow < a.M) store_lowrank_row(a.lowrank + c0, plane, grow, a.rank, v16, 16, ss, scaled);
             } else {
@@ -292,7 +305,7 @@ __global__ void __launch_bounds__(qa::kThreads, 1)
         if (a.splits > 1) {
             __threadfence();
             named_bar_sync(1, 128);
-            if (threadIdx.x == 64) {
+            if (threadIdx.x == 32 * qa::kWorker0) {
                 const unsigned int prev = atomicAdd(a.counters + rb, 1u);
                 s_last = (prev == (unsigned int)(a.splits - 1)) ? 1 : 0;
             }
@@ -317,7 +330,7 @@ __global__ void __launch_bounds__(qa::kThreads, 1)
                     }
                     if (grow < a.M) store_lowrank_row(a.lowrank + c0, plane, grow, a.rank, v16, 16, ss, scaled);
                 }
-                if (threadIdx.x == 64) a.counters[rb] = 0u;   // ready for the next call
+                if (threadIdx.x == 32 * qa::kWorker0) a.counters[rb] = 0u;   // ready for the next call
             }
         }
     }
@@ -325,9 +338,10 @@ __global__ void __launch_bounds__(qa::kThreads, 1)
     __syncthreads();
     // on a timeout, let the copies already issued land before the CTA exits
     if (s_failed && warp == 0 && lane == 0) {
-        const int issued = s_issued;
-        for (int it = (issued > nst ? issued - nst : 0); it < issued; ++it)
-            mbar_wait(&full[it % nst], (uint32_t)(it / nst) & 1u, kSiteQaDrain);
+        for (int s = 0; s < nst; ++s) {
+            const int n = reinterpret_cast<volatile int*>(s_issued)[s];
+            if (n > 0) mbar_wait(&full[s], (uint32_t)(n - 1) & 1u, kSiteQaDrain);
+        }
     }
     tc_fence_before();
     __syncthreads();

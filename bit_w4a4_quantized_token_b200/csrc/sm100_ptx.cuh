@@ -247,6 +247,18 @@ __host__ __device__ constexpr uint32_t idesc_s8_s32(uint32_t n) {
            | ((n >> 3) << 17) | ((128u >> 4) << 24);
 }
 
+// (c0, c1) = (a0 * b0, a1 * b1): one packed fp32 multiply, each lane an IEEE
+// fp32 product rounded to nearest-even (never contracted into an FMA).
+__device__ __forceinline__ void fmul2_rn(float a0, float a1, float b0, float b1, float& c0, float& c1) {
+    asm("{\n\t.reg .b64 ra, rb, rc;\n\t"
+        "mov.b64 ra, {%2, %3};\n\t"
+        "mov.b64 rb, {%4, %5};\n\t"
+        "mul.rn.f32x2 rc, ra, rb;\n\t"
+        "mov.b64 {%0, %1}, rc;\n\t}\n"
+        : "=f"(c0), "=f"(c1)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
 // ------------------------------------------------------------ conversions
 __device__ __forceinline__ float bf16lo_to_f32(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi_to_f32(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }

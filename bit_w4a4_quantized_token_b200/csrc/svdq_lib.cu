@@ -159,14 +159,15 @@ bool make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t
     return r == CUDA_SUCCESS;
 }
 
-// 3-D row-major tensor [planes, outer, inner] with 128-byte swizzled boxes of one plane.
+// 3-D row-major tensor [planes, outer, inner] with 128-byte swizzled boxes of
+// box_planes planes.
 bool make_map_3d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
-                 uint64_t planes, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
+                 uint64_t planes, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, uint32_t box_planes) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t dims[3] = {inner, outer, planes};
     const cuuint64_t strides[2] = {row_bytes, row_bytes * outer};
-    const cuuint32_t box[3] = {box_inner, box_outer, 1};
+    const cuuint32_t box[3] = {box_inner, box_outer, box_planes};
     const cuuint32_t estr[3] = {1, 1, 1};
     const CUresult r = fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -247,7 +248,7 @@ svdq_status quantize_act_launch(int prec, const void* x, int64_t M, int64_t K, c
         return SVDQ_ERR_CUDA;
     if (rank > 0) {
         if (!make_map_3d(&tm_ld, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L_down_t, (uint64_t)K, (uint64_t)rank, 2,
-                         (uint64_t)K * 2, 64, (uint32_t)rank))
+                         (uint64_t)K * 2, 64, (uint32_t)rank, 2))   // hi and lo planes in one box
             return SVDQ_ERR_CUDA;
     } else {
         tm_ld = tm_x;
@@ -272,12 +273,13 @@ svdq_status quantize_act_launch(int prec, const void* x, int64_t M, int64_t K, c
                                                        round_up(row_blocks * 4, 256))
                            : nullptr;
     a.stage_bytes = (uint32_t)qa::kXBytes + (uint32_t)rank * 256u;   // x tile + hi and lo L_down_t tiles
-    const size_t fixed = 1024 + qa::kMaxStages * qa::kCols * 4 + 128 * 4 + (2 * qa::kMaxStages + 1) * 8 + 16;
+    a.max_chunks = (a.chunks + a.splits - 1) / a.splits;
+    const size_t fixed = 1024 + (size_t)a.max_chunks * qa::kCols * 4 + 128 * 4 + (2 * qa::kMaxStages + 1) * 8 + 16;
     const int stages = (int)std::min<size_t>(qa::kMaxStages, (kQuantSmemBudget - fixed) / a.stage_bytes);
-    if (stages < 2) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+    if (stages < 2 || fixed >= (size_t)kQuantSmemBudget) return SVDQ_ERR_UNSUPPORTED_SHAPE;
     a.stages = stages;
     uint32_t tcols = 32;
-    while ((int)tcols < rank) tcols *= 2;
+    while ((int)tcols < 2 * rank) tcols *= 2;   // x . hi and x . lo accumulators
     a.tmem_cols = tcols;
     const size_t smem = fixed + (size_t)stages * a.stage_bytes;
     const dim3 grid((unsigned)a.splits, (unsigned)row_blocks, 1);
@@ -317,7 +319,7 @@ svdq_status gemm_nvfp4(const void* x_codes, const void* x_scales, const float* x
         return SVDQ_ERR_CUDA;
     if (rank > 0) {
         if (!make_map_3d(&tm_L, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, lowrank, (uint64_t)rank, (uint64_t)M, 2,
-                         (uint64_t)rank * 2, 64, gm::BM) ||
+                         (uint64_t)rank * 2, 64, gm::BM, 1) ||
             !make_map(&tm_Lup, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L_up_t, (uint64_t)rank, (uint64_t)N,
                       (uint64_t)rank * 2, 64, gm::BN))
             return SVDQ_ERR_CUDA;
