@@ -115,7 +115,8 @@ svdq_status check_device() {
                                  kQuantSmemBudget) != cudaSuccess ||
             cudaFuncSetAttribute(quantize_act_kernel<kPrecInt4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kQuantSmemBudget) != cudaSuccess ||
-            int4_prepare_device() != cudaSuccess)
+            cudaFuncSetAttribute(gemm_int4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)i4::SMEM_BYTES) != cudaSuccess)
             return cuda_fail("setting kernel shared-memory limits");
         g_device_ready[dev] = true;
     }
@@ -347,6 +348,43 @@ svdq_status gemm_nvfp4(const void* x_codes, const void* x_scales, const float* x
     const int grid = (int)std::min<int64_t>(mt * nt, num_sms());
     gemm_nvfp4_kernel<<<grid, gm::kThreads, gm::SMEM_BYTES, st>>>(tm_xc, tm_wc, tm_L, tm_Lup, a);
     return launch_status("gemm_nvfp4_kernel launch");
+}
+
+svdq_status int4_gemm(const void* x_codes, const void* x_scales, int64_t M, const void* w_codes, const void* w_scales,
+                      int64_t N, int64_t K, const void* lowrank, const void* L_up_t, int rank, const void* bias, void* y,
+                      cudaStream_t st) {
+    CUtensorMap tm_xc, tm_wc, tm_L, tm_Lup;
+    if (!make_map(&tm_xc, CU_TENSOR_MAP_DATA_TYPE_UINT8, x_codes, (uint64_t)K / 2, (uint64_t)M, (uint64_t)K / 2, 128,
+                  i4::BM) ||
+        !make_map(&tm_wc, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_codes, (uint64_t)K / 2, (uint64_t)N, (uint64_t)K / 2, 128,
+                  i4::BN))
+        return SVDQ_ERR_CUDA;
+    if (rank > 0) {
+        if (!make_map_3d(&tm_L, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, lowrank, (uint64_t)rank, (uint64_t)M, 2,
+                         (uint64_t)rank * 2, 64, i4::BM, 1) ||
+            !make_map(&tm_Lup, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L_up_t, (uint64_t)rank, (uint64_t)N,
+                      (uint64_t)rank * 2, 64, i4::BN))
+            return SVDQ_ERR_CUDA;
+    } else {
+        tm_L = tm_xc;
+        tm_Lup = tm_wc;
+    }
+    Int4GemmArgs a;
+    a.x_scales = reinterpret_cast<const uint16_t*>(x_scales);
+    a.w_scales = reinterpret_cast<const uint16_t*>(w_scales);
+    a.bias = reinterpret_cast<const __nv_bfloat16*>(bias);
+    a.y = reinterpret_cast<__nv_bfloat16*>(y);
+    a.M = (int)M;
+    a.N = (int)N;
+    a.K = (int)K;
+    a.rank = rank;
+    a.rows_pad_m = (int)round_up(M, 128);
+    a.rows_pad_n = (int)round_up(N, 128);
+    const int64_t mt = (M + i4::BM - 1) / i4::BM, nt = (N + i4::BN - 1) / i4::BN;
+    if (nt > 65535 || mt > (int64_t(1) << 31) - 1) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+    gemm_int4_kernel<<<dim3((unsigned)mt, (unsigned)nt, 1), i4::kThreads, i4::SMEM_BYTES, st>>>(tm_xc, tm_wc, tm_L,
+                                                                                             tm_Lup, a);
+    return launch_status("gemm_int4_kernel launch");
 }
 
 // Kernel that waits on a barrier nobody completes: exercises the bounded wait.

@@ -145,3 +145,21 @@ def test_int4_quantizers(case):
     assert np.array_equal(unswizzle_int4_scales(packed.w_scales.cpu().numpy(), N, K), ref.w_scales)
     assert np.array_equal(unswizzle_int4_scales(q.x_scales.cpu().numpy(), M, K), ref.x_scales)
     check_lowrank(q.lowrank_act, ref.L, 1.0)
+
+
+# ------------------------------------------------------------ int4 W4A4 GEMM
+INT4_SMALL = [
+    W.scaled(W.INT4_QKV, M=64, K=256, N=256, rank=32, name="int4_tiny"),
+    W.scaled(W.INT4_QKV, M=200, K=320, N=272, rank=16, name="int4_ragged"),   # K tail (5 groups), N tail
+    W.scaled(W.INT4_QKV, M=300, K=1024, N=512, rank=64, name="int4_multi_tile"),
+    W.scaled(W.INT4_QKV, M=129, K=512, N=384, rank=0, name="int4_rank0"),
+]
+
+
+@pytest.mark.parametrize("case", INT4_SMALL, ids=lambda c: c.name)
+def test_int4_small_cases_full(case):
+    check_case(case)
+
+
+def test_int4_full_size_sampled_rows():
+    check_case(W.INT4_QKV, rows=sample_rows(W.INT4_QKV.M, n=24, seed=4))
