@@ -30,6 +30,14 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "SVDQ W4A4 linear TFLOPS (2MNK) and % of B200 dense FP4 tensor peak"
+
+# DRAM bytes (read + write) per launch from one ncu capture of the kernels as
+# they are now (profiles/gemm_nvfp4_qkv.md, profiles/quantize_act_nvfp4_qkv.md).
+# Set an entry to None whenever its kernel changes until it is profiled again.
+PROFILED_DRAM_BYTES = {
+    "gemm_nvfp4_kernel": 25285120 + 31878912,
+    "quantize_act_kernel": 28760832 + 0,
+}
 UNIT = "TFLOPS"
 FP4_OVER_BF16 = 4.0        # nominal dense FP4 : BF16 tensor throughput on B200 (9 : 2.25 PFLOP/s)
 
@@ -237,6 +245,8 @@ def run_cuda(args) -> dict | None:
     e1.record(stream)
     torch.cuda.synchronize(dev)
     t_e2e = max_over_ranks(e0.elapsed_time(e1) / e2e_steps / 1e3, world, dev)
+    # the int4 W4A4 variant on the same QKV shape (group 64, bf16 scales): reported beside the headline
+    int4 = time_int4(args, dev, stream, flush)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -248,7 +258,8 @@ def run_cuda(args) -> dict | None:
     fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16
     gemm_tflops = flops / t_gemm_max / 1e12
     quant_bytes = M * K * 2 + M * K // 2 + M * K // 16 + 4 * M * r + K * 4
-    launches = (2 if not args.dynamic_scale else 4) * args.steps
+    launches = (2 if not args.dynamic_scale else 4) * args.steps   # quantize_act + gemm per step
+    extra = {"int4_qkv": int4}
     return {
         "metric": METRIC,
         "value": round(aggregate(flops, world, t_step), 3),
@@ -271,16 +282,55 @@ def run_cuda(args) -> dict | None:
         "roofline": {"bound": "tensor", "kernel": "gemm_nvfp4_kernel", "achieved": round(gemm_tflops, 2),
                      "peak": round(fp4_peak, 1), "unit": "TFLOP/s", "frac": round(gemm_tflops / fp4_peak, 4),
                      "peak_source": f"{peaks['source']} bf16 burst {peaks['bf16_tflops']} x {FP4_OVER_BF16} (nominal FP4:BF16)",
-                     "traffic": None},
+                     "traffic": PROFILED_DRAM_BYTES.get("gemm_nvfp4_kernel")},
         "quantizer_roofline": {"bound": "hbm", "kernel": "quantize_act_kernel",
                                "achieved": round(quant_bytes / t_quant_max / 1e9, 1), "peak": peaks["hbm_gbs"],
                                "unit": "GB/s", "frac": round(quant_bytes / t_quant_max / 1e9 / peaks["hbm_gbs"], 4),
-                               "traffic": None},
+                               "traffic": PROFILED_DRAM_BYTES.get("quantize_act_kernel")},
         "e2e": {"value": round(aggregate(flops, world, t_e2e), 3), "unit": UNIT,
                 "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2},
         "gpu_launches": launches,
         "clocks": clocks,
+        "extra": extra,
     }
+
+
+def time_int4(args, dev, stream, flush) -> dict:
+    """Device time of the int4 W4A4 layer (quantize + GEMM) on the QKV shape."""
+    import torch
+
+    from bit_w4a4_quantized_token_b200 import _lib, layer
+    from bit_w4a4_quantized_token_b200 import workloads as W
+
+    case = W.INT4_QKV
+    M, K, N, r = case.M, case.K, case.N, case.rank
+    inp = W.make_inputs(case)
+    d = {k: v.to(dev) for k, v in inp.items()}
+    packed = layer.pack_weight(d["R"], d["lam"], d["L_down"], d["L_up"], d["b"], precision="int4")
+    q = layer.alloc_act(packed, M, dev)
+    y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+    steps = max(3, min(args.steps, 10))
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    for i in range(args.warmup + steps):
+        flush.fill_(i & 0xFF)
+        j = i - args.warmup
+        if j >= 0:
+            evs[j][0].record(stream)
+        layer.quantize_act(d["x"], packed, out=q, stream=stream)
+        if j >= 0:
+            evs[j][1].record(stream)
+        layer.gemm(q, packed, y=y, stream=stream)
+        if j >= 0:
+            evs[j][2].record(stream)
+    torch.cuda.synchronize(dev)
+    st, site = _lib.svdq_device_status(clear=True)
+    if st != 0:
+        raise RuntimeError(f"device status {st} at site {site} in the int4 leg")
+    tq = sum(e[0].elapsed_time(e[1]) for e in evs) / steps / 1e3
+    tg = sum(e[1].elapsed_time(e[2]) for e in evs) / steps / 1e3
+    return {"workload": "int4 W4A4 QKV projection M=4608 K=3072 N=9216 rank 32 group 64",
+            "value": round(case.flops / (tq + tg) / 1e12, 2), "unit": "TOPS",
+            "breakdown_us": {"quantize_act": round(tq * 1e6, 2), "gemm_w4a4": round(tg * 1e6, 2)}}
 
 
 # ------------------------------------------------------------------ CPU oracle
