@@ -32,11 +32,11 @@ if ROOT not in sys.path:
 METRIC = "SVDQ W4A4 linear TFLOPS (2MNK) and % of B200 dense FP4 tensor peak"
 
 # DRAM bytes (read + write) per launch from one ncu capture of the kernels as
-# they are now (profiles/gemm_nvfp4_qkv.md, profiles/quantize_act_nvfp4_qkv.md).
+# they are now (profiles/gemm_nvfp4_pair_qkv.md, profiles/quantize_act_nvfp4_qkv.md).
 # Set an entry to None whenever its kernel changes until it is profiled again.
 PROFILED_DRAM_BYTES = {
-    "gemm_nvfp4_kernel": 25285120 + 31878912,
-    "quantize_act_kernel": 28760832 + 0,
+    "gemm_nvfp4_pair_kernel": None,
+    "quantize_act_kernel": None,
 }
 UNIT = "TFLOPS"
 FP4_OVER_BF16 = 4.0        # nominal dense FP4 : BF16 tensor throughput on B200 (9 : 2.25 PFLOP/s)
@@ -279,10 +279,10 @@ def run_cuda(args) -> dict | None:
                    "l2": "flushed before every step (256 MiB write, outside the timed events)",
                    "step": "svdq_quantize_act + svdq_gemm_w4a4", "parallelism": f"replicas x{world} (tokens)"},
         "breakdown_us": {"quantize_act": round(t_quant_max * 1e6, 2), "gemm_w4a4": round(t_gemm_max * 1e6, 2)},
-        "roofline": {"bound": "tensor", "kernel": "gemm_nvfp4_kernel", "achieved": round(gemm_tflops, 2),
+        "roofline": {"bound": "tensor", "kernel": "gemm_nvfp4_pair_kernel", "achieved": round(gemm_tflops, 2),
                      "peak": round(fp4_peak, 1), "unit": "TFLOP/s", "frac": round(gemm_tflops / fp4_peak, 4),
                      "peak_source": f"{peaks['source']} bf16 burst {peaks['bf16_tflops']} x {FP4_OVER_BF16} (nominal FP4:BF16)",
-                     "traffic": PROFILED_DRAM_BYTES.get("gemm_nvfp4_kernel")},
+                     "traffic": PROFILED_DRAM_BYTES.get("gemm_nvfp4_pair_kernel")},
         "quantizer_roofline": {"bound": "hbm", "kernel": "quantize_act_kernel",
                                "achieved": round(quant_bytes / t_quant_max / 1e9, 1), "peak": peaks["hbm_gbs"],
                                "unit": "GB/s", "frac": round(quant_bytes / t_quant_max / 1e9 / peaks["hbm_gbs"], 4),

@@ -32,6 +32,7 @@ EXPORTS = (
     "svdq_quantize_act_workspace_bytes", "svdq_quantize_act", "svdq_quantize_act_noalloc", "svdq_gemm_w4a4",
     "svdq_device_status",
     "svdq_debug_set_wait_limit_ns", "svdq_debug_timeout_probe", "svdq_debug_override_capability",
+    "svdq_debug_force_gemm_tiles",
 )
 
 
@@ -81,6 +82,8 @@ def _load():
     lib.svdq_debug_timeout_probe.restype = I
     lib.svdq_debug_override_capability.argtypes = [I, I]
     lib.svdq_debug_override_capability.restype = None
+    lib.svdq_debug_force_gemm_tiles.argtypes = [I]
+    lib.svdq_debug_force_gemm_tiles.restype = I
     return lib
 
 
@@ -191,3 +194,8 @@ def svdq_debug_timeout_probe(stream=None) -> None:
 
 def svdq_debug_override_capability(major: int, minor: int = 0) -> None:
     lib.svdq_debug_override_capability(int(major), int(minor))
+
+
+def svdq_debug_force_gemm_tiles(mode: int) -> None:
+    """0 = automatic, 1 = single-CTA 128x256 tiles, 2 = CTA-pair 256x256 tiles (nvfp4 GEMM)."""
+    _check(lib.svdq_debug_force_gemm_tiles(int(mode)), "svdq_debug_force_gemm_tiles")

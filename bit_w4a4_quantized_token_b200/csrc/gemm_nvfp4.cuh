@@ -38,8 +38,9 @@ constexpr int kThreads = 32 * (kEpiWarp0 + kEpiWarps);
 constexpr uint32_t kMmaWarp = 2;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COL = 0;               // 256 fp32 columns
-constexpr uint32_t SFA_COL = 256;             // 4 k-steps x 4 columns
-constexpr uint32_t SFB_COL = 272;             // 4 k-steps x 8 columns
+constexpr uint32_t SF_COL = 256;              // scale factors of ring stage s at SF_COL + 48 s:
+constexpr uint32_t SF_STAGE_COLS = 48;        //   4 k-steps x 4 columns (A), then 4 k-steps x 8 columns (B)
+static_assert(SF_COL + kStages * SF_STAGE_COLS <= TMEM_COLS, "scale-factor columns do not fit in TMEM");
 constexpr size_t SMEM_BYTES = 1024 + (size_t)kStages * STAGE_BYTES + 256;
 }  // namespace gm
 
@@ -193,14 +194,24 @@ __global__ void __launch_bounds__(gm::kThreads, 1)
                         const uint32_t sfa = sb + B_BYTES;
                         const uint32_t sfb = sfa + SFA_BYTES;
                         const int nks = min(4, a.kg4 - 4 * kk);
+                        // Scale blocks go to this stage's own TMEM columns, and the
+                        // copies for K-step j + 1 are issued before the MMA of step j:
+                        // the tensor pipe runs its instructions in order, so copies
+                        // queued behind an MMA overlap it, while a batch of copies in
+                        // front of the MMAs would not.
+                        const uint32_t t_sfa = tmem + SF_COL + SF_STAGE_COLS * (uint32_t)s;
+                        const uint32_t t_sfb = t_sfa + 16u;
+                        auto copy_scales = [&](int j) {
+                            tmem_cp_32x128b_x4(t_sfa + 4u * j, desc_sf_block(sfa + 512u * j));
+                            tmem_cp_32x128b_x4(t_sfb + 8u * j, desc_sf_block(sfb + 512u * j));
+                            tmem_cp_32x128b_x4(t_sfb + 8u * j + 4u, desc_sf_block(sfb + 2048u + 512u * j));
+                        };
+                        copy_scales(0);
                         for (int j = 0; j < nks; ++j) {
-                            tmem_cp_32x128b_x4(tmem + SFA_COL + 4u * j, desc_sf_block(sfa + 512u * j));
-                            tmem_cp_32x128b_x4(tmem + SFB_COL + 8u * j, desc_sf_block(sfb + 512u * j));
-                            tmem_cp_32x128b_x4(tmem + SFB_COL + 8u * j + 4u, desc_sf_block(sfb + 2048u + 512u * j));
-                        }
-                        for (int j = 0; j < nks; ++j)
+                            if (j + 1 < nks) copy_scales(j + 1);
                             mma_nvfp4(tmem + ACC_COL, desc_sw128(sa + 32u * j), desc_sw128(sb + 32u * j), idesc_fp4,
-                                      tmem + SFA_COL + 4u * j, tmem + SFB_COL + 8u * j, (kk > 0 || j > 0) ? 1u : 0u);
+                                      t_sfa + 4u * j, t_sfb + 8u * j, (kk > 0 || j > 0) ? 1u : 0u);
+                        }
                     } else {
                         const int c = (kk - n_kb) >> 1;
                         const int nks = min(4, (a.rank - 64 * c + 15) / 16);

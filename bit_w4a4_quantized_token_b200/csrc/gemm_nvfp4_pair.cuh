@@ -1,0 +1,362 @@
+// gemm_nvfp4_pair.cuh -- the block-scaled FP4 GEMM of the SVDQ W4A4 layer on
+// CTA pairs (tcgen05 cta_group::2), for M > 128.
+//
+// Computes exactly what gemm_nvfp4_kernel computes (see gemm_nvfp4.cuh: FP4 x FP4
+// main loop, the hi and lo bf16 parts of the rank-r branch into the same fp32
+// accumulator, y = bf16(S_x S_w acc + b)), on 256 x 256 output tiles.  Each
+// tile belongs to a cluster of two CTAs on neighbouring SMs:
+//   * CTA r (r = 0, 1) loads rows 128 r .. 128 r + 127 of the tile's activation
+//     codes and rows 128 r .. 128 r + 127 of its weight codes, the scale block
+//     of its own 128 activation rows and the scale blocks of all 256 weight
+//     rows (the tensor core reads the weight scales of every column in both
+//     halves of the pair);
+//   * CTA 0 alone copies the scale blocks into both CTAs' TMEM and issues one
+//     M = 256, N = 256 MMA per 64 values of K; the accumulator rows of CTA r
+//     sit in CTA r's TMEM;
+//   * every load of either CTA completes on CTA 0's stage barrier, CTA 0's
+//     commits arrive on both CTAs' "stage free" and "accumulator full"
+//     barriers, and both CTAs' epilogue warps hand the accumulator back on
+//     CTA 0's barrier.
+// Against 128 x 256 tiles on single CTAs this halves the weight-code bytes
+// each SM loads per FLOP and the number of scale-block copies per FLOP.
+//
+// All scale blocks arrive by TMA (maps over the 512-byte blocks) so that the
+// peer CTA's loads can complete on CTA 0's barrier; a box that runs past the
+// end of a scale buffer is zero-filled, which only ever feeds rows or K-steps
+// whose results are discarded.  Only CTA 0's producers arrive on a stage
+// barrier, announcing the bytes of both CTAs (every box is counted in full,
+// zero-filled parts included); the peer's loads cannot land early because the
+// peer refills a stage only after CTA 0's MMAs have released it.
+//
+// One thread issuing TMA copies manages roughly one stage every 600-700
+// cycles, whatever the box size, and a stage of four K-steps lasts 512 cycles
+// of MMA; so each producer role runs on two lanes that take alternate stages.
+#pragma once
+#include "gemm_nvfp4.cuh"
+
+namespace svdq {
+namespace gp {
+constexpr int BM = 256;                        // tile rows (128 per CTA)
+constexpr int BN = 256;                        // tile columns (128 weight rows loaded per CTA)
+constexpr int BK_BYTES = 128;
+constexpr int kStages = 5;
+constexpr int A_BYTES = 128 * BK_BYTES;        // 16 KB: this CTA's 128 activation rows
+constexpr int B_BYTES = 128 * BK_BYTES;        // 16 KB: this CTA's 128 weight rows
+constexpr int SFA_BYTES = 4 * 512;             // scale blocks of this CTA's 128 rows, 4 k-steps
+constexpr int SFB_BYTES = 8 * 512;             // scale blocks of all 256 weight rows, 4 k-steps
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+constexpr int kEpiWarps = 8;
+constexpr int kEpiWarp0 = 4;
+constexpr int kThreads = 32 * (kEpiWarp0 + kEpiWarps);
+constexpr uint32_t kMmaWarp = 2;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t ACC_COL = 0;
+// Scale factors in TMEM, one of two layouts:
+//  * streamed (any K): ring stage s uses columns SF_COL + 48 s: 4 k-steps x 4
+//    columns of activation scales, then 4 k-steps x 8 columns of weight scales;
+//  * resident activation scales (K <= 64 * kResidentKSteps): the activation
+//    scales of the whole K for the current 256-row tile stay at SFA_RES +
+//    4 k, copied once per run of tiles that share those rows, and the weight
+//    scales alternate between two sets of 32 columns at SFB_RES.  This takes
+//    the activation-scale copies (a third of all copies) off the tensor pipe.
+constexpr uint32_t SF_COL = 256;
+constexpr uint32_t SF_STAGE_COLS = 48;
+static_assert(SF_COL + kStages * SF_STAGE_COLS <= TMEM_COLS, "scale-factor columns do not fit in TMEM");
+constexpr int kResidentKSteps = 48;
+constexpr uint32_t SFA_RES = 256;
+constexpr uint32_t SFB_RES = SFA_RES + 4 * kResidentKSteps;   // 448: two sets of 32 columns
+static_assert(SFB_RES + 64 <= TMEM_COLS, "resident scale-factor columns do not fit in TMEM");
+constexpr uint32_t kFullArrivals = 3;          // CTA 0's three producer roles, for both CTAs' bytes
+constexpr int kLanesPerRole = 2;               // producer lanes per role, taking alternate stages
+constexpr uint32_t kAccEmptyArrivals = 2 * kEpiWarps;
+constexpr size_t SMEM_BYTES = 1024 + (size_t)kStages * STAGE_BYTES + 256;
+static_assert(SMEM_BYTES <= 227 * 1024, "stage ring does not fit in shared memory");
+}  // namespace gp
+
+enum : uint32_t {
+    kSiteGpEmpty = 24,
+    kSiteGpFull = 25,
+    kSiteGpAcc = 26,
+    kSiteGpDrain = 27,
+    kSiteGpAccEmpty = 28
+};
+
+__global__ void __launch_bounds__(gp::kThreads, 1)
+    gemm_nvfp4_pair_kernel(const __grid_constant__ CUtensorMap tm_xc, const __grid_constant__ CUtensorMap tm_wc,
+                           const __grid_constant__ CUtensorMap tm_sfa, const __grid_constant__ CUtensorMap tm_sfb,
+                           const __grid_constant__ CUtensorMap tm_L, const __grid_constant__ CUtensorMap tm_Lup,
+                           GemmArgs a) {
+    using namespace gp;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)kStages * STAGE_BYTES);
+    uint64_t* empty = full + kStages;
+    uint64_t* acc_full = empty + kStages;
+    uint64_t* acc_empty = acc_full + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
+    __shared__ int s_failed;
+    __shared__ int s_issued[gp::kStages];   // phases this CTA's A producers started in each stage
+
+    const uint32_t warp = warp_id(), lane = lane_id();
+    const uint32_t rank = cluster_ctarank();          // 0 = the CTA that issues the MMAs
+    const int cluster = (int)(blockIdx.x >> 1), n_clusters = (int)(gridDim.x >> 1);
+    const int n_kb = (a.K + 255) / 256;
+    const int n_lr = a.rank > 0 ? 2 * ((a.rank + 63) / 64) : 0;
+    const int per_tile = n_kb + n_lr;
+    const int total_tiles = a.m_tiles * a.n_tiles;    // m_tiles counts 256-row tiles here
+    // Each cluster takes a contiguous run of tiles, n fastest, so that it keeps
+    // the same 256 activation rows for several tiles in a row.
+    const int t_begin = (int)(((int64_t)total_tiles * cluster) / n_clusters);
+    const int t_end = (int)(((int64_t)total_tiles * (cluster + 1)) / n_clusters);
+    const bool sfa_res = a.kg4 <= kResidentKSteps;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&full[s], kFullArrivals);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(acc_full, 1);
+        mbar_init(acc_empty, kAccEmptyArrivals);
+        for (int s = 0; s < kStages; ++s) s_issued[s] = 0;
+        s_failed = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tensormap(&tm_xc);
+        prefetch_tensormap(&tm_wc);
+        prefetch_tensormap(&tm_sfa);
+        prefetch_tensormap(&tm_sfb);
+        if (a.rank > 0) {
+            prefetch_tensormap(&tm_L);
+            prefetch_tensormap(&tm_Lup);
+        }
+    }
+    if (warp == kMmaWarp) {   // the same warp in both CTAs, the same slot offset
+        tmem_alloc_pair(tmem_slot, TMEM_COLS);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    cluster_sync_all();       // barriers of both CTAs initialised, TMEM address written
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0 || warp == 1 || warp == 3) {
+        // ----------------------------------------------------------- producers
+        if (lane < (uint32_t)kLanesPerRole) {
+            const int role = warp == 0 ? 0 : (warp == 1 ? 1 : 2);   // A codes, B codes, scale blocks
+            const bool leader = rank == 0;
+            int it = 0;
+            bool ok = true;
+            for (int tile = t_begin; tile < t_end && ok; ++tile) {
+                const int m_tile = tile / a.n_tiles, n_tile = tile - m_tile * a.n_tiles;
+                const bool need_sfa = !sfa_res || tile == t_begin || n_tile == 0;
+                const int m0 = m_tile * BM + 128 * (int)rank;      // this CTA's activation rows
+                const int n0 = n_tile * BN + 128 * (int)rank;      // this CTA's weight rows
+                for (int kk = 0; kk < per_tile; ++kk, ++it) {
+                    if ((it % kLanesPerRole) != (int)lane) continue;
+                    const int s = it % kStages;
+                    const uint32_t ph = (uint32_t)(it / kStages) & 1u;
+                    if (!mbar_wait(&empty[s], ph ^ 1u, kSiteGpEmpty)) {
+                        s_failed = 1;
+                        ok = false;
+                        break;
+                    }
+                    uint8_t* sa = smem + (size_t)s * STAGE_BYTES;
+                    uint8_t* sb = sa + A_BYTES;
+                    uint8_t* sfa = sb + B_BYTES;
+                    uint8_t* sfb = sfa + SFA_BYTES;
+                    const uint32_t bar = cluster_addr(&full[s], 0);   // CTA 0 counts every load
+                    if (kk < n_kb) {
+                        const int kb = kk;
+                        if (role == 0) {
+                            if (leader) mbar_arrive_expect_tx(&full[s], 2u * A_BYTES);
+                            tma_load_2d_pair(sa, &tm_xc, bar, kb * BK_BYTES, m0);
+                            atomicAdd(&s_issued[s], 1);
+                        } else if (role == 1) {
+                            if (leader) mbar_arrive_expect_tx(&full[s], 2u * B_BYTES);
+                            tma_load_2d_pair(sb, &tm_wc, bar, kb * BK_BYTES, n0);
+                        } else {
+                            if (leader)
+                                mbar_arrive_expect_tx(&full[s], 2u * ((need_sfa ? SFA_BYTES : 0) + SFB_BYTES));
+                            if (need_sfa) tma_load_3d_pair(sfa, &tm_sfa, bar, 0, 4 * kb, 2 * m_tile + (int)rank);
+                            tma_load_3d_pair(sfb, &tm_sfb, bar, 0, 4 * kb, 2 * n_tile);   // both weight row blocks
+                        }
+                    } else {
+                        const int c = (kk - n_kb) >> 1, part = (kk - n_kb) & 1;
+                        if (role == 0) {
+                            if (leader) mbar_arrive_expect_tx(&full[s], 2u * A_BYTES);
+                            tma_load_3d_pair(sa, &tm_L, bar, c * 64, m0, part);
+                            atomicAdd(&s_issued[s], 1);
+                        } else if (role == 1) {
+                            if (leader) mbar_arrive_expect_tx(&full[s], 2u * B_BYTES);
+                            tma_load_2d_pair(sb, &tm_Lup, bar, c * 64, n0);
+                        } else {
+                            if (leader) mbar_arrive(&full[s]);
+                        }
+                    }
+                }
+            }
+        }
+    } else if (warp == kMmaWarp) {
+        // ------------------------------------------------- MMA issuer (CTA 0)
+        if (rank == 0 && lane == 0) {
+            // The tensor pipe queues very few instructions, so every cycle this
+            // thread spends between MMAs is a bubble: stage and phase are kept
+            // incrementally, descriptors are formed once per stage and advanced
+            // by adding to their address field, and full stages are unrolled.
+            const uint32_t idesc_fp4 = idesc_m(idesc_nvfp4(BN), BM);
+            const uint32_t idesc_lr = idesc_m(idesc_bf16_f32(BN), BM);
+            const uint32_t smem0 = smem_u32(smem);
+            bool ok = true;
+            int local = 0, s = 0, it = 0;
+            uint32_t ph = 0;
+            for (int tile = t_begin; tile < t_end && ok; ++tile, ++local) {
+                const int n_tile = tile % a.n_tiles;
+                const bool need_sfa = !sfa_res || tile == t_begin || n_tile == 0;
+                if (!mbar_wait(acc_empty, ((uint32_t)local & 1u) ^ 1u, kSiteGpAccEmpty)) {
+                    s_failed = 1;
+                    break;
+                }
+                tc_fence_after();
+                for (int kk = 0; kk < per_tile; ++kk, ++it) {
+                    if (!mbar_wait(&full[s], ph, kSiteGpFull)) {
+                        ok = false;
+                        s_failed = 1;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sa = smem0 + (uint32_t)s * STAGE_BYTES;
+                    const uint32_t sb = sa + A_BYTES;
+                    const uint64_t da = desc_sw128(sa), db = desc_sw128(sb);   // + 2 per K-step of 32 bytes
+                    if (kk < n_kb) {
+                        const uint64_t dfa = desc_sf_block(sb + B_BYTES);                // + 32 per 512-byte block
+                        const uint64_t dfb = desc_sf_block(sb + B_BYTES + SFA_BYTES);
+                        const int nks = min(4, a.kg4 - 4 * kk);
+                        // Activation-scale columns of K-step j and the weight-scale columns.
+                        const uint32_t ta = sfa_res ? tmem + SFA_RES + 16u * (uint32_t)kk
+                                                    : tmem + SF_COL + SF_STAGE_COLS * (uint32_t)s;
+                        const uint32_t tb = sfa_res ? tmem + SFB_RES + 32u * (uint32_t)(it & 1)
+                                                    : tmem + SF_COL + SF_STAGE_COLS * (uint32_t)s + 16u;
+                        // Copies for K-step j + 1 go in before the MMA of step j, so
+                        // that they queue behind an MMA instead of in front of one.
+                        auto copy_scales = [&](int j) {
+                            if (need_sfa) tmem_cp_32x128b_x4_pair(ta + 4u * j, dfa + 32u * j);
+                            tmem_cp_32x128b_x4_pair(tb + 8u * j, dfb + 32u * j);
+                            tmem_cp_32x128b_x4_pair(tb + 8u * j + 4u, dfb + 128u + 32u * j);
+                        };
+                        auto mma = [&](int j) {
+                            mma_nvfp4_pair(tmem + ACC_COL, da + 2u * j, db + 2u * j, idesc_fp4, ta + 4u * j,
+                                           tb + 8u * j, (kk > 0 || j > 0) ? 1u : 0u);
+                        };
+                        copy_scales(0);
+                        if (nks == 4) {
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                if (j < 3) copy_scales(j + 1);
+                                mma(j);
+                            }
+                        } else {
+                            for (int j = 0; j < nks; ++j) {
+                                if (j + 1 < nks) copy_scales(j + 1);
+                                mma(j);
+                            }
+                        }
+                    } else {
+                        const int c = (kk - n_kb) >> 1;
+                        const int nks = min(4, (a.rank - 64 * c + 15) / 16);
+                        for (int j = 0; j < nks; ++j)
+                            mma_bf16_pair(tmem + ACC_COL, da + 2u * j, db + 2u * j, idesc_lr, 1u);
+                    }
+                    tc_commit_pair(&empty[s], 0x3);
+                    if (++s == kStages) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                }
+                if (ok) tc_commit_pair(acc_full, 0x3);
+            }
+        }
+    } else if (warp >= (uint32_t)kEpiWarp0) {
+        // ------------------------------------------------------------ epilogue
+        const uint32_t q = warp & 3u;
+        const int half = (int)(warp - kEpiWarp0) >> 2;
+        const int row = (int)(32u * q + lane);
+        const float S = __fmul_rn(*a.x_scale, *a.w_scale);
+        const uint32_t acc_empty_leader = cluster_addr(acc_empty, 0);
+        int local = 0;
+        for (int tile = t_begin; tile < t_end; ++tile, ++local) {
+            const int m_tile = tile / a.n_tiles, n_tile = tile - m_tile * a.n_tiles;
+            const int64_t grow = (int64_t)m_tile * BM + 128 * (int64_t)rank + row;
+            const int nbase = n_tile * BN + 128 * half;
+            if (!mbar_wait(acc_full, (uint32_t)local & 1u, kSiteGpAcc)) {
+                s_failed = 1;
+                break;
+            }
+            tc_fence_after();
+            uint32_t acc[128];
+            tmem_ld_32x32b_x32(tmem + ((32u * q) << 16) + ACC_COL + 128u * half + 0u,
+                               *reinterpret_cast<uint32_t(*)[32]>(acc + 0));
+            tmem_ld_32x32b_x32(tmem + ((32u * q) << 16) + ACC_COL + 128u * half + 32u,
+                               *reinterpret_cast<uint32_t(*)[32]>(acc + 32));
+            tmem_ld_32x32b_x32(tmem + ((32u * q) << 16) + ACC_COL + 128u * half + 64u,
+                               *reinterpret_cast<uint32_t(*)[32]>(acc + 64));
+            tmem_ld_32x32b_x32(tmem + ((32u * q) << 16) + ACC_COL + 128u * half + 96u,
+                               *reinterpret_cast<uint32_t(*)[32]>(acc + 96));
+            tmem_ld_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(acc_empty_leader);   // this half of the pair is drained
+            if (grow >= a.M) continue;
+            __nv_bfloat16* yrow = a.y + grow * (int64_t)a.N;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const int n = nbase + 16 * c;
+                if (n >= a.N) break;
+                float bv[16];
+                if (a.bias) {
+                    const uint4 w0 = __ldg(reinterpret_cast<const uint4*>(a.bias + n));
+                    const uint4 w1 = __ldg(reinterpret_cast<const uint4*>(a.bias + n) + 1);
+                    const uint32_t ws[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+                    for (int p = 0; p < 8; ++p) {
+                        bv[2 * p] = bf16lo_to_f32(ws[p]);
+                        bv[2 * p + 1] = bf16hi_to_f32(ws[p]);
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) bv[i] = 0.0f;
+                }
+                uint32_t packed[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const float o0 = fmaf(__uint_as_float(acc[16 * c + 2 * i]), S, bv[2 * i]);
+                    const float o1 = fmaf(__uint_as_float(acc[16 * c + 2 * i + 1]), S, bv[2 * i + 1]);
+                    const __nv_bfloat162 h = __floats2bfloat162_rn(o0, o1);
+                    packed[i] = *reinterpret_cast<const uint32_t*>(&h);
+                }
+                uint4* dst = reinterpret_cast<uint4*>(yrow + n);
+                dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+                dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+            }
+        }
+    }
+
+    __syncthreads();
+    if (s_failed && rank == 0 && warp == 0 && lane == 0) {
+        // after a timeout, let the loads already issued land before either CTA
+        // exits (both CTAs' loads complete on CTA 0's barriers; best effort:
+        // each wait is bounded)
+        for (int s = 0; s < kStages; ++s) {
+            const int n = reinterpret_cast<volatile int*>(s_issued)[s];
+            if (n > 0) mbar_wait(&full[s], (uint32_t)(n - 1) & 1u, kSiteGpDrain);
+        }
+    }
+    tc_fence_before();
+    cluster_sync_all();   // no remote arrival or MMA may target a CTA that has exited
+    if (warp == kMmaWarp) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem, TMEM_COLS);
+    }
+}
+
+}  // namespace svdq

@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstdint>
 #include <cstdio>
 #include <cstring>
@@ -16,6 +17,7 @@
 #include "quantize.cuh"
 #include "quantize_act.cuh"
 #include "gemm_nvfp4.cuh"
+#include "gemm_nvfp4_pair.cuh"
 #include "int4.cuh"
 
 namespace svdq {
@@ -61,6 +63,7 @@ int64_t round_up(int64_t v, int64_t m) { return (v + m - 1) / m * m; }
 std::mutex g_mutex;
 int g_override_major = -1, g_override_minor = 0;
 constexpr int kMaxDevices = 64;
+std::atomic<int> g_gemm_tiles_mode{0};   // svdq_debug_force_gemm_tiles
 bool g_device_ready[kMaxDevices];
 
 // Budget of dynamic shared memory for the activation quantizer (the opt-in
@@ -116,7 +119,9 @@ svdq_status check_device() {
             cudaFuncSetAttribute(quantize_act_kernel<kPrecInt4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kQuantSmemBudget) != cudaSuccess ||
             cudaFuncSetAttribute(gemm_int4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)i4::SMEM_BYTES) != cudaSuccess)
+                                 (int)i4::SMEM_BYTES) != cudaSuccess ||
+            cudaFuncSetAttribute(gemm_nvfp4_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)gp::SMEM_BYTES) != cudaSuccess)
             return cuda_fail("setting kernel shared-memory limits");
         g_device_ready[dev] = true;
     }
@@ -175,6 +180,25 @@ bool make_map_3d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint6
                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS)
         snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled (3-D) failed (CUresult %d)", (int)r);
+    return r == CUDA_SUCCESS;
+}
+
+// Scale blocks viewed as a 3-D tensor of 32-bit words [row_blocks][kg4][128]:
+// one 512-byte block (128 rows x 4 groups) per (row block, 64 columns of K);
+// boxes of 4 consecutive K blocks of `box_row_blocks` row blocks, unswizzled.
+bool make_sf_map(CUtensorMap* m, const void* base, uint64_t row_blocks, uint64_t kg4, uint32_t box_row_blocks) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {128, kg4, row_blocks};
+    const cuuint64_t strides[2] = {512, 512 * kg4};
+    const cuuint32_t box[3] = {128, 4, box_row_blocks};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<void*>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS)
+        snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled (scale blocks) failed (CUresult %d)",
+                 (int)r);
     return r == CUDA_SUCCESS;
 }
 
@@ -348,6 +372,94 @@ svdq_status gemm_nvfp4(const void* x_codes, const void* x_scales, const float* x
     const int grid = (int)std::min<int64_t>(mt * nt, num_sms());
     gemm_nvfp4_kernel<<<grid, gm::kThreads, gm::SMEM_BYTES, st>>>(tm_xc, tm_wc, tm_L, tm_Lup, a);
     return launch_status("gemm_nvfp4_kernel launch");
+}
+
+// Clusters of two CTAs that fit on the device at once (one CTA per SM).
+int pair_clusters() {
+    static int per_dev[kMaxDevices];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= kMaxDevices) return num_sms() / 2;
+    if (per_dev[dev] == 0) {
+        cudaLaunchConfig_t cfg = {};
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.gridDim = dim3(2 * (unsigned)num_sms(), 1, 1);
+        cfg.blockDim = dim3(gp::kThreads, 1, 1);
+        cfg.dynamicSmemBytes = gp::SMEM_BYTES;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, gemm_nvfp4_pair_kernel, &cfg) != cudaSuccess || n <= 0) {
+            cudaGetLastError();
+            n = num_sms() / 2;
+        }
+        per_dev[dev] = n;
+    }
+    return per_dev[dev];
+}
+
+// M > 128: 256 x 256 tiles on CTA pairs.
+svdq_status gemm_nvfp4_pair(const void* x_codes, const void* x_scales, const float* x_scale, int64_t M,
+                            const void* w_codes, const void* w_scales, const float* w_scale, int64_t N, int64_t K,
+                            const void* lowrank, const void* L_up_t, int rank, const void* bias, void* y,
+                            cudaStream_t st) {
+    CUtensorMap tm_xc, tm_wc, tm_sfa, tm_sfb, tm_L, tm_Lup;
+    const int64_t kg4 = K / 64;
+    if (!make_map(&tm_xc, CU_TENSOR_MAP_DATA_TYPE_UINT8, x_codes, (uint64_t)K / 2, (uint64_t)M, (uint64_t)K / 2,
+                  gp::BK_BYTES, 128) ||
+        !make_map(&tm_wc, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_codes, (uint64_t)K / 2, (uint64_t)N, (uint64_t)K / 2,
+                  gp::BK_BYTES, 128) ||
+        !make_sf_map(&tm_sfa, x_scales, (uint64_t)((M + 127) / 128), (uint64_t)kg4, 1) ||
+        !make_sf_map(&tm_sfb, w_scales, (uint64_t)((N + 127) / 128), (uint64_t)kg4, 2))
+        return SVDQ_ERR_CUDA;
+    if (rank > 0) {
+        if (!make_map_3d(&tm_L, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, lowrank, (uint64_t)rank, (uint64_t)M, 2,
+                         (uint64_t)rank * 2, 64, 128, 1) ||
+            !make_map(&tm_Lup, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L_up_t, (uint64_t)rank, (uint64_t)N,
+                      (uint64_t)rank * 2, 64, 128))
+            return SVDQ_ERR_CUDA;
+    } else {
+        tm_L = tm_xc;
+        tm_Lup = tm_wc;
+    }
+    GemmArgs a;
+    a.x_scales = reinterpret_cast<const uint8_t*>(x_scales);
+    a.w_scales = reinterpret_cast<const uint8_t*>(w_scales);
+    a.x_scale = x_scale;
+    a.w_scale = w_scale;
+    a.bias = reinterpret_cast<const __nv_bfloat16*>(bias);
+    a.y = reinterpret_cast<__nv_bfloat16*>(y);
+    a.M = (int)M;
+    a.N = (int)N;
+    a.K = (int)K;
+    a.rank = rank;
+    a.kg4 = (int)kg4;
+    a.n_sf_blocks = (int)((N + 127) / 128);
+    const int64_t mt = (M + gp::BM - 1) / gp::BM, nt = (N + gp::BN - 1) / gp::BN;
+    if (mt * nt > (int64_t(1) << 30)) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+    a.m_tiles = (int)mt;
+    a.n_tiles = (int)nt;
+    const int clusters = (int)std::min<int64_t>(mt * nt, pair_clusters());
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(2 * (unsigned)clusters, 1, 1);
+    cfg.blockDim = dim3(gp::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = gp::SMEM_BYTES;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, gemm_nvfp4_pair_kernel, tm_xc, tm_wc, tm_sfa, tm_sfb, tm_L, tm_Lup, a) !=
+        cudaSuccess)
+        return cuda_fail("gemm_nvfp4_pair_kernel launch");
+    return launch_status("gemm_nvfp4_pair_kernel launch");
 }
 
 svdq_status int4_gemm(const void* x_codes, const void* x_scales, int64_t M, const void* w_codes, const void* w_scales,
@@ -603,9 +715,14 @@ svdq_status svdq_gemm_w4a4(svdq_precision p, int group_size, const void* x_codes
     }
     SVDQ_TRY(check_device());
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    if (p == SVDQ_NVFP4)
+    if (p == SVDQ_NVFP4) {
+        const int mode = g_gemm_tiles_mode.load();
+        if (mode == 2 || (mode == 0 && M > 128))
+            return gemm_nvfp4_pair(x_codes, x_scales, x_tensor_scale, M, w_codes, w_scales, w_tensor_scale, N, K,
+                                   lowrank_act, L_up_t, rank, bias, y, st);
         return gemm_nvfp4(x_codes, x_scales, x_tensor_scale, M, w_codes, w_scales, w_tensor_scale, N, K, lowrank_act,
                           L_up_t, rank, bias, y, st);
+    }
     return int4_gemm(x_codes, x_scales, M, w_codes, w_scales, N, K, lowrank_act, L_up_t, rank, bias, y, st);
 }
 
@@ -637,6 +754,15 @@ svdq_status svdq_debug_timeout_probe(svdq_stream_t stream) {
     SVDQ_TRY(check_device());
     timeout_probe_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>();
     return launch_status("timeout_probe_kernel launch");
+}
+
+svdq_status svdq_debug_force_gemm_tiles(int mode) {
+    if (mode < 0 || mode > 2) {
+        snprintf(g_last_error, sizeof(g_last_error), "svdq_debug_force_gemm_tiles: mode %d is not 0, 1 or 2", mode);
+        return SVDQ_ERR_INVALID_ARG;
+    }
+    g_gemm_tiles_mode.store(mode);
+    return SVDQ_OK;
 }
 
 void svdq_debug_override_capability(int major, int minor) {

@@ -118,6 +118,17 @@ def test_capability_check_rejects_other_devices(L):
         L.svdq_debug_override_capability(-1)
 
 
+def test_force_gemm_tiles_hook(L):
+    """Modes 0, 1, 2 are accepted (no device needed); anything else is rejected with a message."""
+    for mode in (1, 2, 0):
+        L.svdq_debug_force_gemm_tiles(mode)
+    for bad in (-1, 3):
+        with pytest.raises(L.SvdqError) as e:
+            L.svdq_debug_force_gemm_tiles(bad)
+        assert e.value.status == L.SVDQ_ERR_INVALID_ARG
+        assert "not 0, 1 or 2" in L.lib.svdq_last_error().decode()
+
+
 def test_quantize_act_workspace_bytes(L):
     # QKV shape: 36 row blocks x 4 K-splits x 128 rows x rank 32 fp32, plus a 256-byte counter block
     assert L.svdq_quantize_act_workspace_bytes("nvfp4", 4608, 3072, 32) == 256 + 36 * 4 * 128 * 32 * 4

@@ -45,6 +45,20 @@ def test_small_cases_full(case):
     check_case(case)
 
 
+@pytest.mark.parametrize("mode", [1, 2], ids=["single_cta_tiles", "cta_pair_tiles"])
+@pytest.mark.parametrize("case", SMALL, ids=lambda c: c.name)
+def test_small_cases_each_gemm_kernel(case, mode):
+    """Both nvfp4 GEMM kernels (128 x 256 tiles on one CTA, 256 x 256 tiles on
+    a CTA pair) on every small case, whatever M would pick."""
+    from bit_w4a4_quantized_token_b200 import _lib
+
+    _lib.svdq_debug_force_gemm_tiles(mode)
+    try:
+        check_case(case)
+    finally:
+        _lib.svdq_debug_force_gemm_tiles(0)
+
+
 def test_static_tensor_scale():
     case = W.scaled(W.QKV, M=160, K=512, N=256, rank=32, name="static_S")
     check_case(case, x_tensor_scale=0.0625)
