@@ -51,23 +51,25 @@ constexpr int kThreads = 32 * (kEpiWarp0 + kEpiWarps);
 constexpr uint32_t kMmaWarp = 2;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COL = 0;
-// Scale factors in TMEM, one of two layouts:
-//  * streamed (any K): ring stage s uses columns SF_COL + 48 s: 4 k-steps x 4
-//    columns of activation scales, then 4 k-steps x 8 columns of weight scales;
+// Scale factors in TMEM.  Stages alternate between two "scale sets"; one of
+// two layouts:
+//  * streamed (any K): set b at SF_COL + 48 b: 4 k-steps x 4 columns of
+//    activation scales, then 4 k-steps x 8 columns of weight scales;
 //  * resident activation scales (K <= 64 * kResidentKSteps): the activation
 //    scales of the whole K for the current 256-row tile stay at SFA_RES +
-//    4 k, copied once per run of tiles that share those rows, and the weight
-//    scales alternate between two sets of 32 columns at SFB_RES.  This takes
-//    the activation-scale copies (a third of all copies) off the tensor pipe.
+//    4 k, copied once per run of tiles that share those rows, and set b holds
+//    only weight scales, at SFB_RES + 32 b.  This takes the activation-scale
+//    copies (a third of all copies) off the tensor pipe.
 constexpr uint32_t SF_COL = 256;
-constexpr uint32_t SF_STAGE_COLS = 48;
-static_assert(SF_COL + kStages * SF_STAGE_COLS <= TMEM_COLS, "scale-factor columns do not fit in TMEM");
+constexpr uint32_t SF_SET_COLS = 48;
+static_assert(SF_COL + 2 * SF_SET_COLS <= TMEM_COLS, "scale-factor columns do not fit in TMEM");
 constexpr int kResidentKSteps = 48;
 constexpr uint32_t SFA_RES = 256;
 constexpr uint32_t SFB_RES = SFA_RES + 4 * kResidentKSteps;   // 448: two sets of 32 columns
 static_assert(SFB_RES + 64 <= TMEM_COLS, "resident scale-factor columns do not fit in TMEM");
 constexpr uint32_t kFullArrivals = 3;          // CTA 0's three producer roles, for both CTAs' bytes
 constexpr int kLanesPerRole = 2;               // producer lanes per role, taking alternate stages
+constexpr uint32_t kCopyWarp = 3;              // issues the scale-block copies into TMEM
 constexpr uint32_t kAccEmptyArrivals = 2 * kEpiWarps;
 constexpr size_t SMEM_BYTES = 1024 + (size_t)kStages * STAGE_BYTES + 256;
 static_assert(SMEM_BYTES <= 227 * 1024, "stage ring does not fit in shared memory");
@@ -78,7 +80,11 @@ enum : uint32_t {
     kSiteGpFull = 25,
     kSiteGpAcc = 26,
     kSiteGpDrain = 27,
-    kSiteGpAccEmpty = 28
+    kSiteGpAccEmpty = 28,
+    kSiteGpSfReady = 29,
+    kSiteGpSfFree = 30,
+    kSiteGpCopyFull = 31,
+    kSiteGpCopyAcc = 32
 };
 
 __global__ void __launch_bounds__(gp::kThreads, 1)
@@ -93,7 +99,9 @@ __global__ void __launch_bounds__(gp::kThreads, 1)
     uint64_t* empty = full + kStages;
     uint64_t* acc_full = empty + kStages;
     uint64_t* acc_empty = acc_full + 1;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
+    uint64_t* sf_ready = acc_empty + 1;       // [2] copies of a scale set done (copy warp -> MMA)
+    uint64_t* sf_free = sf_ready + 2;         // [2] MMAs reading a scale set done (MMA -> copy warp)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sf_free + 2);
     __shared__ int s_failed;
     __shared__ int s_issued[gp::kStages];   // phases this CTA's A producers started in each stage
 
@@ -117,6 +125,10 @@ __global__ void __launch_bounds__(gp::kThreads, 1)
         }
         mbar_init(acc_full, 1);
         mbar_init(acc_empty, kAccEmptyArrivals);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&sf_ready[b], 1);
+            mbar_init(&sf_free[b], 1);
+        }
         for (int s = 0; s < kStages; ++s) s_issued[s] = 0;
         s_failed = 0;
         fence_barrier_init();
@@ -140,10 +152,13 @@ __global__ void __launch_bounds__(gp::kThreads, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 0 || warp == 1 || warp == 3) {
+    if (warp == 0 || warp == 1) {
         // ----------------------------------------------------------- producers
-        if (lane < (uint32_t)kLanesPerRole) {
-            const int role = warp == 0 ? 0 : (warp == 1 ? 1 : 2);   // A codes, B codes, scale blocks
+        // warp 0 lanes 0-1: activation codes; warp 1 lanes 0-1: weight codes,
+        // lanes 2-3: scale blocks.  Each role's two lanes take alternate stages.
+        if (lane < (uint32_t)(warp == 0 ? kLanesPerRole : 2 * kLanesPerRole)) {
+            const int role = warp == 0 ? 0 : (lane < (uint32_t)kLanesPerRole ? 1 : 2);
+            const uint32_t rlane = lane % (uint32_t)kLanesPerRole;
             const bool leader = rank == 0;
             int it = 0;
             bool ok = true;
@@ -153,7 +168,7 @@ __global__ void __launch_bounds__(gp::kThreads, 1)
                 const int m0 = m_tile * BM + 128 * (int)rank;      // this CTA's activation rows
                 const int n0 = n_tile * BN + 128 * (int)rank;      // this CTA's weight rows
                 for (int kk = 0; kk < per_tile; ++kk, ++it) {
-                    if ((it % kLanesPerRole) != (int)lane) continue;
+                    if ((it % kLanesPerRole) != (int)rlane) continue;
                     const int s = it % kStages;
                     const uint32_t ph = (uint32_t)(it / kStages) & 1u;
                     if (!mbar_wait(&empty[s], ph ^ 1u, kSiteGpEmpty)) {
@@ -197,6 +212,59 @@ __global__ void __launch_bounds__(gp::kThreads, 1)
                 }
             }
         }
+    } else if (warp == kCopyWarp) {
+        // ----------------------------------------- scale-block copies (CTA 0)
+        // Copies are issued from their own thread: a shared-memory access by a
+        // thread with copies in flight waits for them, so the MMA thread,
+        // which must wait on a barrier every stage, issues MMAs only.
+        if (rank == 0 && lane == 0) {
+            const uint32_t smem0 = smem_u32(smem);
+            bool ok = true;
+            int local = 0, s = 0, it = 0;
+            uint32_t ph = 0;
+            for (int tile = t_begin; tile < t_end && ok; ++tile, ++local) {
+                const int n_tile = tile % a.n_tiles;
+                const bool need_sfa = !sfa_res || tile == t_begin || n_tile == 0;
+                // resident activation scales are overwritten only after every
+                // MMA of the previous tile (which read them) has completed
+                if (sfa_res && need_sfa && tile != t_begin &&
+                    !mbar_wait(acc_full, (uint32_t)(local - 1) & 1u, kSiteGpCopyAcc)) {
+                    s_failed = 1;
+                    break;
+                }
+                for (int kk = 0; kk < per_tile; ++kk, ++it) {
+                    const int b = it & 1;
+                    const int use = it >> 1;
+                    if ((use > 0 && !mbar_wait(&sf_free[b], (uint32_t)(use - 1) & 1u, kSiteGpSfFree)) ||
+                        !mbar_wait(&full[s], ph, kSiteGpCopyFull)) {
+                        ok = false;
+                        s_failed = 1;
+                        break;
+                    }
+                    tc_fence_after();
+                    if (kk < n_kb) {
+                        const uint32_t sfa = smem0 + (uint32_t)s * STAGE_BYTES + A_BYTES + B_BYTES;
+                        const uint64_t dfa = desc_sf_block(sfa);                 // + 32 per 512-byte block
+                        const uint64_t dfb = desc_sf_block(sfa + SFA_BYTES);
+                        const int nks = min(4, a.kg4 - 4 * kk);
+                        const uint32_t ta = sfa_res ? tmem + SFA_RES + 16u * (uint32_t)kk
+                                                    : tmem + SF_COL + SF_SET_COLS * (uint32_t)b;
+                        const uint32_t tb = sfa_res ? tmem + SFB_RES + 32u * (uint32_t)b
+                                                    : tmem + SF_COL + SF_SET_COLS * (uint32_t)b + 16u;
+                        for (int j = 0; j < nks; ++j) {
+                            if (need_sfa) tmem_cp_32x128b_x4_pair(ta + 4u * j, dfa + 32u * j);
+                            tmem_cp_32x128b_x4_pair(tb + 8u * j, dfb + 32u * j);
+                            tmem_cp_32x128b_x4_pair(tb + 8u * j + 4u, dfb + 128u + 32u * j);
+                        }
+                    }
+                    tc_commit_pair(&sf_ready[b], 0x1);
+                    if (++s == kStages) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                }
+            }
+        }
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------- MMA issuer (CTA 0)
         if (rank == 0 && lane == 0) {
@@ -211,55 +279,39 @@ __global__ void __launch_bounds__(gp::kThreads, 1)
             int local = 0, s = 0, it = 0;
             uint32_t ph = 0;
             for (int tile = t_begin; tile < t_end && ok; ++tile, ++local) {
-                const int n_tile = tile % a.n_tiles;
-                const bool need_sfa = !sfa_res || tile == t_begin || n_tile == 0;
                 if (!mbar_wait(acc_empty, ((uint32_t)local & 1u) ^ 1u, kSiteGpAccEmpty)) {
                     s_failed = 1;
                     break;
                 }
                 tc_fence_after();
                 for (int kk = 0; kk < per_tile; ++kk, ++it) {
-                    if (!mbar_wait(&full[s], ph, kSiteGpFull)) {
+                    const int b = it & 1;
+                    // the copy thread saw the stage full before its scale copies
+                    // completed; the second wait is then already satisfied
+                    if (!mbar_wait(&sf_ready[b], (uint32_t)(it >> 1) & 1u, kSiteGpSfReady) ||
+                        !mbar_wait(&full[s], ph, kSiteGpFull)) {
                         ok = false;
                         s_failed = 1;
                         break;
                     }
                     tc_fence_after();
                     const uint32_t sa = smem0 + (uint32_t)s * STAGE_BYTES;
-                    const uint32_t sb = sa + A_BYTES;
-                    const uint64_t da = desc_sw128(sa), db = desc_sw128(sb);   // + 2 per K-step of 32 bytes
+                    const uint64_t da = desc_sw128(sa), db = desc_sw128(sa + A_BYTES);   // + 2 per 32-byte K-step
                     if (kk < n_kb) {
-                        const uint64_t dfa = desc_sf_block(sb + B_BYTES);                // + 32 per 512-byte block
-                        const uint64_t dfb = desc_sf_block(sb + B_BYTES + SFA_BYTES);
                         const int nks = min(4, a.kg4 - 4 * kk);
-                        // Activation-scale columns of K-step j and the weight-scale columns.
                         const uint32_t ta = sfa_res ? tmem + SFA_RES + 16u * (uint32_t)kk
-                                                    : tmem + SF_COL + SF_STAGE_COLS * (uint32_t)s;
-                        const uint32_t tb = sfa_res ? tmem + SFB_RES + 32u * (uint32_t)(it & 1)
-                                                    : tmem + SF_COL + SF_STAGE_COLS * (uint32_t)s + 16u;
-                        // Copies for K-step j + 1 go in before the MMA of step j, so
-                        // that they queue behind an MMA instead of in front of one.
-                        auto copy_scales = [&](int j) {
-                            if (need_sfa) tmem_cp_32x128b_x4_pair(ta + 4u * j, dfa + 32u * j);
-                            tmem_cp_32x128b_x4_pair(tb + 8u * j, dfb + 32u * j);
-                            tmem_cp_32x128b_x4_pair(tb + 8u * j + 4u, dfb + 128u + 32u * j);
-                        };
+                                                    : tmem + SF_COL + SF_SET_COLS * (uint32_t)b;
+                        const uint32_t tb = sfa_res ? tmem + SFB_RES + 32u * (uint32_t)b
+                                                    : tmem + SF_COL + SF_SET_COLS * (uint32_t)b + 16u;
                         auto mma = [&](int j) {
                             mma_nvfp4_pair(tmem + ACC_COL, da + 2u * j, db + 2u * j, idesc_fp4, ta + 4u * j,
                                            tb + 8u * j, (kk > 0 || j > 0) ? 1u : 0u);
                         };
-                        copy_scales(0);
                         if (nks == 4) {
 #pragma unroll
-                            for (int j = 0; j < 4; ++j) {
-                                if (j < 3) copy_scales(j + 1);
-                                mma(j);
-                            }
+                            for (int j = 0; j < 4; ++j) mma(j);
                         } else {
-                            for (int j = 0; j < nks; ++j) {
-                                if (j + 1 < nks) copy_scales(j + 1);
-                                mma(j);
-                            }
+                            for (int j = 0; j < nks; ++j) mma(j);
                         }
                     } else {
                         const int c = (kk - n_kb) >> 1;
@@ -268,6 +320,7 @@ __global__ void __launch_bounds__(gp::kThreads, 1)
                             mma_bf16_pair(tmem + ACC_COL, da + 2u * j, db + 2u * j, idesc_lr, 1u);
                     }
                     tc_commit_pair(&empty[s], 0x3);
+                    tc_commit_pair(&sf_free[b], 0x1);
                     if (++s == kStages) {
                         s = 0;
                         ph ^= 1u;
