@@ -197,5 +197,6 @@ def svdq_debug_override_capability(major: int, minor: int = 0) -> None:
 
 
 def svdq_debug_force_gemm_tiles(mode: int) -> None:
-    """0 = automatic, 1 = single-CTA 128x256 tiles, 2 = CTA-pair 256x256 tiles (nvfp4 GEMM)."""
+    """nvfp4 GEMM kernel: 0 = automatic, 1 = single-CTA 128x256 tiles, 2 = CTA-pair 256x256
+    tiles, 3 = CTA-pair 256x128 tiles where K allows (else 256x256)."""
     _check(lib.svdq_debug_force_gemm_tiles(int(mode)), "svdq_debug_force_gemm_tiles")

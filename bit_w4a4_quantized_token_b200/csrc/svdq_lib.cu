@@ -18,6 +18,7 @@
 #include "quantize_act.cuh"
 #include "gemm_nvfp4.cuh"
 #include "gemm_nvfp4_pair.cuh"
+#include "gemm_nvfp4_pair128.cuh"
 #include "int4.cuh"
 
 namespace svdq {
@@ -121,7 +122,9 @@ svdq_status check_device() {
             cudaFuncSetAttribute(gemm_int4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)i4::SMEM_BYTES) != cudaSuccess ||
             cudaFuncSetAttribute(gemm_nvfp4_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)gp::SMEM_BYTES) != cudaSuccess)
+                                 (int)gp::SMEM_BYTES) != cudaSuccess ||
+            cudaFuncSetAttribute(gemm_nvfp4_pair128_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)gq::SMEM_BYTES) != cudaSuccess)
             return cuda_fail("setting kernel shared-memory limits");
         g_device_ready[dev] = true;
     }
@@ -186,12 +189,13 @@ bool make_map_3d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint6
 // Scale blocks viewed as a 3-D tensor of 32-bit words [row_blocks][kg4][128]:
 // one 512-byte block (128 rows x 4 groups) per (row block, 64 columns of K);
 // boxes of 4 consecutive K blocks of `box_row_blocks` row blocks, unswizzled.
-bool make_sf_map(CUtensorMap* m, const void* base, uint64_t row_blocks, uint64_t kg4, uint32_t box_row_blocks) {
+bool make_sf_map(CUtensorMap* m, const void* base, uint64_t row_blocks, uint64_t kg4, uint32_t box_row_blocks,
+                 uint32_t box_ksteps = 4) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t dims[3] = {128, kg4, row_blocks};
     const cuuint64_t strides[2] = {512, 512 * kg4};
-    const cuuint32_t box[3] = {128, 4, box_row_blocks};
+    const cuuint32_t box[3] = {128, box_ksteps, box_row_blocks};
     const cuuint32_t estr[3] = {1, 1, 1};
     const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<void*>(base), dims, strides, box, estr,
                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -374,12 +378,14 @@ svdq_status gemm_nvfp4(const void* x_codes, const void* x_scales, const float* x
     return launch_status("gemm_nvfp4_kernel launch");
 }
 
-// Clusters of two CTAs that fit on the device at once (one CTA per SM).
+// Clusters of two CTAs that fit on the device at once (one CTA per SM; both
+// pair kernels have the same block size and nearly all of shared memory).
 int pair_clusters() {
     static int per_dev[kMaxDevices];
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= kMaxDevices) return num_sms() / 2;
+    static_assert(gq::kThreads == gp::kThreads, "pair kernels differ in block size");
     if (per_dev[dev] == 0) {
         cudaLaunchConfig_t cfg = {};
         cudaLaunchAttribute attr[1];
@@ -400,6 +406,75 @@ int pair_clusters() {
         per_dev[dev] = n;
     }
     return per_dev[dev];
+}
+
+// 256 x 128 tiles on CTA pairs with the weight scales resident in TMEM (M >
+// 128, K <= 3072, K % 512 == 0).  Selected only on request: on B200 its MMA
+// thread issues an N = 128 MMA and its scale copy in about 205 cycles, against
+// about 170 cycles per N = 256 MMA (twice the work) in the 256 x 256 kernel,
+// so it is the slower of the two (136 against 111 us on the 4608 x 3072 x
+// 9216 projection).
+bool pair128_applies(int64_t M, int64_t K) {
+    return M > 128 && K % 512 == 0 && K / 64 <= gq::kMaxKSteps;
+}
+
+svdq_status gemm_nvfp4_pair128(const void* x_codes, const void* x_scales, const float* x_scale, int64_t M,
+                               const void* w_codes, const void* w_scales, const float* w_scale, int64_t N, int64_t K,
+                               const void* lowrank, const void* L_up_t, int rank, const void* bias, void* y,
+                               cudaStream_t st) {
+    CUtensorMap tm_xc, tm_wc, tm_sfa, tm_sfb, tm_L, tm_Lup;
+    const int64_t kg4 = K / 64;
+    if (!make_map(&tm_xc, CU_TENSOR_MAP_DATA_TYPE_UINT8, x_codes, (uint64_t)K / 2, (uint64_t)M, (uint64_t)K / 2,
+                  gq::CHUNK, 128) ||
+        !make_map(&tm_wc, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_codes, (uint64_t)K / 2, (uint64_t)N, (uint64_t)K / 2,
+                  gq::CHUNK, 64) ||
+        !make_sf_map(&tm_sfa, x_scales, (uint64_t)((M + 127) / 128), (uint64_t)kg4, 1, gq::KSTEPS) ||
+        !make_sf_map(&tm_sfb, w_scales, (uint64_t)((N + 127) / 128), (uint64_t)kg4, 1, gq::KSTEPS))
+        return SVDQ_ERR_CUDA;
+    if (rank > 0) {
+        if (!make_map_3d(&tm_L, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, lowrank, (uint64_t)rank, (uint64_t)M, 2,
+                         (uint64_t)rank * 2, 64, 128, 1) ||
+            !make_map(&tm_Lup, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L_up_t, (uint64_t)rank, (uint64_t)N,
+                      (uint64_t)rank * 2, 64, 64))
+            return SVDQ_ERR_CUDA;
+    } else {
+        tm_L = tm_xc;
+        tm_Lup = tm_wc;
+    }
+    GemmArgs a;
+    a.x_scales = reinterpret_cast<const uint8_t*>(x_scales);
+    a.w_scales = reinterpret_cast<const uint8_t*>(w_scales);
+    a.x_scale = x_scale;
+    a.w_scale = w_scale;
+    a.bias = reinterpret_cast<const __nv_bfloat16*>(bias);
+    a.y = reinterpret_cast<__nv_bfloat16*>(y);
+    a.M = (int)M;
+    a.N = (int)N;
+    a.K = (int)K;
+    a.rank = rank;
+    a.kg4 = (int)kg4;
+    a.n_sf_blocks = (int)((N + 127) / 128);
+    const int64_t mt = (M + gq::BM - 1) / gq::BM, nt = (N + gq::BN - 1) / gq::BN;
+    if (mt * nt > (int64_t(1) << 30)) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+    a.m_tiles = (int)mt;
+    a.n_tiles = (int)nt;
+    const int clusters = (int)std::min<int64_t>(mt * nt, pair_clusters());
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(2 * (unsigned)clusters, 1, 1);
+    cfg.blockDim = dim3(gq::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = gq::SMEM_BYTES;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, gemm_nvfp4_pair128_kernel, tm_xc, tm_wc, tm_sfa, tm_sfb, tm_L, tm_Lup, a) !=
+        cudaSuccess)
+        return cuda_fail("gemm_nvfp4_pair128_kernel launch");
+    return launch_status("gemm_nvfp4_pair128_kernel launch");
 }
 
 // M > 128: 256 x 256 tiles on CTA pairs.
@@ -717,7 +792,10 @@ svdq_status svdq_gemm_w4a4(svdq_precision p, int group_size, const void* x_codes
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (p == SVDQ_NVFP4) {
         const int mode = g_gemm_tiles_mode.load();
-        if (mode == 2 || (mode == 0 && M > 128))
+        if (mode == 3 && pair128_applies(M, K))
+            return gemm_nvfp4_pair128(x_codes, x_scales, x_tensor_scale, M, w_codes, w_scales, w_tensor_scale, N, K,
+                                      lowrank_act, L_up_t, rank, bias, y, st);
+        if (mode == 2 || mode == 3 || (mode == 0 && M > 128))
             return gemm_nvfp4_pair(x_codes, x_scales, x_tensor_scale, M, w_codes, w_scales, w_tensor_scale, N, K,
                                    lowrank_act, L_up_t, rank, bias, y, st);
         return gemm_nvfp4(x_codes, x_scales, x_tensor_scale, M, w_codes, w_scales, w_tensor_scale, N, K, lowrank_act,
@@ -757,8 +835,9 @@ svdq_status svdq_debug_timeout_probe(svdq_stream_t stream) {
 }
 
 svdq_status svdq_debug_force_gemm_tiles(int mode) {
-    if (mode < 0 || mode > 2) {
-        snprintf(g_last_error, sizeof(g_last_error), "svdq_debug_force_gemm_tiles: mode %d is not 0, 1 or 2", mode);
+    if (mode < 0 || mode > 3) {
+        snprintf(g_last_error, sizeof(g_last_error), "svdq_debug_force_gemm_tiles: mode %d is not 0, 1, 2 or 3",
+                 mode);
         return SVDQ_ERR_INVALID_ARG;
     }
     g_gemm_tiles_mode.store(mode);

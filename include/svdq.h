@@ -206,11 +206,14 @@ svdq_status svdq_device_status(int clear, int* site);
  *    status word then reads SVDQ_ERR_TIMEOUT.  Used to test failure detection.
  *  svdq_debug_override_capability: pretend the device has compute capability
  *    major.minor (major = -1 removes the override), to test the device check.
- *  svdq_debug_force_gemm_tiles: choose the nvfp4 GEMM kernel regardless of M:
- *    0 = automatic (128 x 256 tiles on single CTAs when M <= 128, 256 x 256
- *    tiles on CTA pairs otherwise), 1 = always single CTAs, 2 = always CTA
- *    pairs.  Both kernels compute the same y; this exists so that tests can
- *    run each on the same inputs.  Any other value is SVDQ_ERR_INVALID_ARG. */
+ *  svdq_debug_force_gemm_tiles: choose the nvfp4 GEMM kernel: 0 = automatic
+ *    (M <= 128: 128 x 256 tiles on single CTAs; M > 128: 256 x 256 tiles on
+ *    CTA pairs), 1 = always single CTAs, 2 = always 256 x 256 CTA-pair tiles,
+ *    3 = 256 x 128 CTA-pair tiles with the weight scales resident in tensor
+ *    memory where M > 128, K % 512 == 0 and K <= 3072 (a slower alternative,
+ *    never chosen automatically), else as 2.  All kernels compute the same y;
+ *    this exists so that tests can run each on the same inputs.  Any other
+ *    value is SVDQ_ERR_INVALID_ARG. */
 svdq_status svdq_debug_set_wait_limit_ns(uint64_t ns);
 svdq_status svdq_debug_timeout_probe(svdq_stream_t stream);
 void svdq_debug_override_capability(int major, int minor);
