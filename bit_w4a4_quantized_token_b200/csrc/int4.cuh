@@ -318,9 +318,17 @@ __global__ void __launch_bounds__(i4::kThreads, 1)
                     }
                 }
                 tmem_ld_wait();
+                // acc += float(P) * (sx * sw), two columns per instruction.  A
+                // group's partial sum P is at most 64 * 8 * 8 = 4096 in magnitude,
+                // so it converts exactly without the (low-throughput) I2F unit.
 #pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    acc[32 * h + i] = fmaf((float)(int)r[i], __fmul_rn(sx, sw[i]), acc[32 * h + i]);
+                for (int i = 0; i < 32; i += 2) {
+                    float p0, p1, s0, s1;
+                    fadd2_rn(i2f_biased(r[i]), i2f_biased(r[i + 1]), -kMagicI2F, -kMagicI2F, p0, p1);
+                    fmul2_rn(sx, sx, sw[i], sw[i + 1], s0, s1);
+                    ffma2_rn(p0, p1, s0, s1, acc[32 * h + i], acc[32 * h + i + 1], acc[32 * h + i],
+                             acc[32 * h + i + 1]);
+                }
             }
             give(use);
             ++use;

@@ -298,6 +298,37 @@ __device__ __forceinline__ void fmul2_rn(float a0, float a1, float b0, float b1,
         : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
 }
 
+// (c0, c1) = (a0 * b0 + d0, a1 * b1 + d1), each rounded once to nearest even.
+__device__ __forceinline__ void ffma2_rn(float a0, float a1, float b0, float b1, float d0, float d1, float& c0,
+                                         float& c1) {
+    asm("{\n\t.reg .b64 ra, rb, rd, rc;\n\t"
+        "mov.b64 ra, {%2, %3};\n\t"
+        "mov.b64 rb, {%4, %5};\n\t"
+        "mov.b64 rd, {%6, %7};\n\t"
+        "fma.rn.f32x2 rc, ra, rb, rd;\n\t"
+        "mov.b64 {%0, %1}, rc;\n\t}\n"
+        : "=f"(c0), "=f"(c1)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(d0), "f"(d1));
+}
+
+// (c0, c1) = (a0 + b0, a1 + b1), each rounded to nearest even.
+__device__ __forceinline__ void fadd2_rn(float a0, float a1, float b0, float b1, float& c0, float& c1) {
+    asm("{\n\t.reg .b64 ra, rb, rc;\n\t"
+        "mov.b64 ra, {%2, %3};\n\t"
+        "mov.b64 rb, {%4, %5};\n\t"
+        "add.rn.f32x2 rc, ra, rb;\n\t"
+        "mov.b64 {%0, %1}, rc;\n\t}\n"
+        : "=f"(c0), "=f"(c1)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
+// Exact int32 -> float for |v| < 2^22 on the integer and FP32 pipes: the bit
+// pattern of 1.5 * 2^23 plus v is the float 1.5 * 2^23 + v (the unit in the
+// last place there is 1), so subtracting 1.5 * 2^23 leaves v.  The caller does
+// the subtraction (packed, two values at a time).
+constexpr float kMagicI2F = 12582912.0f;   // 1.5 * 2^23
+__device__ __forceinline__ float i2f_biased(uint32_t v) { return __uint_as_float(v + 0x4B400000u); }
+
 // ----------------------------------------------------- CTA pairs (cta_group::2)
 __device__ __forceinline__ uint32_t cluster_ctarank() {
     uint32_t r;
