@@ -292,13 +292,28 @@ __global__ void __launch_bounds__(i4::kThreads, 1)
             give(use);
             ++use;
         }
+        // The group scales are read from global memory once per group and used
+        // at once, so the lines of group g + 2 are pulled into L1 while group g
+        // is processed (shared memory is taken by the stage rings).  On the
+        // 4608 x 3072 x 9216 shape this measured neutral: the epilogue is bound
+        // by instruction issue (a scale, a convert and an FMA per element and
+        // group), not by these loads.
+        auto prefetch_scales = [&](int g) {
+            if (lane == 0) {
+                asm volatile("prefetch.global.L1 [%0];" ::"l"(a.w_scales + (int64_t)g * a.rows_pad_n + nb));
+                asm volatile("prefetch.global.L1 [%0];" ::"l"(a.x_scales + (int64_t)g * a.rows_pad_m + m0 + 32 * q));
+            }
+        };
+        prefetch_scales(0);
+        if (groups > 1) prefetch_scales(1);
         for (int g = 0; g < groups && ok; ++g) {
+            if (g + 2 < groups) prefetch_scales(g + 2);
+            const float sx = (grow < a.M) ? __bfloat162float(__ushort_as_bfloat16(a.x_scales[(int64_t)g * a.rows_pad_m + grow]))
+                                          : 0.0f;
             if (!take(use)) {
                 ok = false;
                 break;
             }
-            const float sx = (grow < a.M) ? __bfloat162float(__ushort_as_bfloat16(a.x_scales[(int64_t)g * a.rows_pad_m + grow]))
-                                          : 0.0f;
             const uint16_t* swp = a.w_scales + (int64_t)g * a.rows_pad_n + nb;
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
