@@ -10,15 +10,17 @@
 //     of its own 128 activation rows and the scale blocks of all 256 weight
 //     rows (the tensor core reads the weight scales of every column in both
 //     halves of the pair);
-//   * CTA 0 alone copies the scale blocks into both CTAs' TMEM and issues one
-//     M = 256, N = 256 MMA per 64 values of K; the accumulator rows of CTA r
-//     sit in CTA r's TMEM;
+//   * CTA 0 alone copies the scale blocks into both CTAs' TMEM (a copy warp)
+//     and issues one M = 256, N = 256 MMA per 64 values of K (the MMA warp);
+//     the accumulator rows of CTA r sit in CTA r's TMEM;
 //   * every load of either CTA completes on CTA 0's stage barrier, CTA 0's
 //     commits arrive on both CTAs' "stage free" and "accumulator full"
 //     barriers, and both CTAs' epilogue warps hand the accumulator back on
 //     CTA 0's barrier.
 // Against 128 x 256 tiles on single CTAs this halves the weight-code bytes
-// each SM loads per FLOP and the number of scale-block copies per FLOP.
+// each SM loads per FLOP and the number of scale-block copies per FLOP; with
+// the activation scales resident in TMEM (K <= 3072, below) two copies per
+// MMA remain, and those copies, not the loads, set the pace.
 //
 // All scale blocks arrive by TMA (maps over the 512-byte blocks) so that the
 // peer CTA's loads can complete on CTA 0's barrier; a box that runs past the
