@@ -71,7 +71,6 @@ constexpr uint32_t SFB_RES = SFA_RES + 4 * kResidentKSteps;   // 448: two sets o
 static_assert(SFB_RES + 64 <= TMEM_COLS, "resident scale-factor columns do not fit in TMEM");
 constexpr uint32_t kFullArrivals = 3;          // CTA 0's three producer roles, for both CTAs' bytes
 constexpr int kLanesPerRole = 2;               // producer lanes per role, taking alternate stages
-constexpr uint32_t kCopyWarp = 3;              // issues the scale-block copies into TMEM
 constexpr uint32_t kAccEmptyArrivals = 2 * kEpiWarps;
 constexpr size_t SMEM_BYTES = 1024 + (size_t)kStages * STAGE_BYTES + 256;
 static_assert(SMEM_BYTES <= 227 * 1024, "stage ring does not fit in shared memory");
@@ -82,12 +81,31 @@ enum : uint32_t {
     kSiteGpFull = 25,
     kSiteGpAcc = 26,
     kSiteGpDrain = 27,
-    kSiteGpAccEmpty = 28,
-    kSiteGpSfReady = 29,
-    kSiteGpSfFree = 30,
-    kSiteGpCopyFull = 31,
-    kSiteGpCopyAcc = 32
+    kSiteGpAccEmpty = 28
 };
+
+// One stage of four K-steps, issued by the MMA thread: the scale-block copies
+// of K-step j + 1 go in right before the MMA of step j.  The tensor pipe keeps
+// only a few instructions queued, so this sequence is written to have nothing
+// between its tcgen05 instructions but address arithmetic on registers: every
+// cycle the issuing thread spends elsewhere (branches, loads, waits) is a cycle
+// the pipe may sit idle.  WITH_SFA: also copy the activation scales.
+template <bool WITH_SFA>
+__device__ __forceinline__ void gp_issue_stage(uint32_t acc, uint64_t da, uint64_t db, uint64_t dfa, uint64_t dfb,
+                                               uint32_t ta, uint32_t tb, uint32_t idesc, uint32_t acc0) {
+    if (WITH_SFA) tmem_cp_32x128b_x4_pair(ta, dfa);
+    tmem_cp_32x128b_x4_pair(tb, dfb);
+    tmem_cp_32x128b_x4_pair(tb + 4u, dfb + 128u);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        if (j < 3) {
+            if (WITH_SFA) tmem_cp_32x128b_x4_pair(ta + 4u * (j + 1), dfa + 32u * (j + 1));
+            tmem_cp_32x128b_x4_pair(tb + 8u * (j + 1), dfb + 32u * (j + 1));
+            tmem_cp_32x128b_x4_pair(tb + 8u * (j + 1) + 4u, dfb + 128u + 32u * (j + 1));
+        }
+        mma_nvfp4_pair(acc, da + 2u * j, db + 2u * j, idesc, ta + 4u * j, tb + 8u * j, j == 0 ? acc0 : 1u);
+    }
+}
 
 __global__ void __launch_bounds__(gp::kThreads, 1)
     gemm_nvfp4_pair_kernel(const __grid_constant__ CUtensorMap tm_xc, const __grid_constant__ CUtensorMap tm_wc,
@@ -101,9 +119,7 @@ __global__ void __launch_bounds__(gp::kThreads, 1)
     uint64_t* empty = full + kStages;
     uint64_t* acc_full = empty + kStages;
     uint64_t* acc_empty = acc_full + 1;
-    uint64_t* sf_ready = acc_empty + 1;       // [2] copies of a scale set done (copy warp -> MMA)
-    uint64_t* sf_free = sf_ready + 2;         // [2] MMAs reading a scale set done (MMA -> copy warp)
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sf_free + 2);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
     __shared__ int s_failed;
     __shared__ int s_issued[gp::kStages];   // phases this CTA's A producers started in each stage
 
@@ -127,10 +143,6 @@ __global__ void __launch_bounds__(gp::kThreads, 1)
         }
         mbar_init(acc_full, 1);
         mbar_init(acc_empty, kAccEmptyArrivals);
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(&sf_ready[b], 1);
-            mbar_init(&sf_free[b], 1);
-        }
         for (int s = 0; s < kStages; ++s) s_issued[s] = 0;
         s_failed = 0;
         fence_barrier_init();
@@ -214,84 +226,27 @@ __global__ void __launch_bounds__(gp::kThreads, 1)
                 }
             }
         }
-    } else if (warp == kCopyWarp) {
-        // ----------------------------------------- scale-block copies (CTA 0)
-        // Copies are issued from their own thread: a shared-memory access by a
-        // thread with copies in flight waits for them, so the MMA thread,
-        // which must wait on a barrier every stage, issues MMAs only.
+    } else if (warp == kMmaWarp) {
+        // ------------------------------------------ copies + MMAs (CTA 0 only)
         if (rank == 0 && lane == 0) {
+            const uint32_t idesc_fp4 = idesc_m(idesc_nvfp4(BN), BM);
+            const uint32_t idesc_lr = idesc_m(idesc_bf16_f32(BN), BM);
             const uint32_t smem0 = smem_u32(smem);
+            const int nks_last = a.kg4 - 4 * (n_kb - 1);   // K-steps in the last stage (1..4)
             bool ok = true;
             int local = 0, s = 0, it = 0;
             uint32_t ph = 0;
             for (int tile = t_begin; tile < t_end && ok; ++tile, ++local) {
                 const int n_tile = tile % a.n_tiles;
                 const bool need_sfa = !sfa_res || tile == t_begin || n_tile == 0;
-                // resident activation scales are overwritten only after every
-                // MMA of the previous tile (which read them) has completed
-                if (sfa_res && need_sfa && tile != t_begin &&
-                    !mbar_wait(acc_full, (uint32_t)(local - 1) & 1u, kSiteGpCopyAcc)) {
-                    s_failed = 1;
-                    break;
-                }
-                for (int kk = 0; kk < per_tile; ++kk, ++it) {
-                    const int b = it & 1;
-                    const int use = it >> 1;
-                    if ((use > 0 && !mbar_wait(&sf_free[b], (uint32_t)(use - 1) & 1u, kSiteGpSfFree)) ||
-                        !mbar_wait(&full[s], ph, kSiteGpCopyFull)) {
-                        ok = false;
-                        s_failed = 1;
-                        break;
-                    }
-                    tc_fence_after();
-                    if (kk < n_kb) {
-                        const uint32_t sfa = smem0 + (uint32_t)s * STAGE_BYTES + A_BYTES + B_BYTES;
-                        const uint64_t dfa = desc_sf_block(sfa);                 // + 32 per 512-byte block
-                        const uint64_t dfb = desc_sf_block(sfa + SFA_BYTES);
-                        const int nks = min(4, a.kg4 - 4 * kk);
-                        const uint32_t ta = sfa_res ? tmem + SFA_RES + 16u * (uint32_t)kk
-                                                    : tmem + SF_COL + SF_SET_COLS * (uint32_t)b;
-                        const uint32_t tb = sfa_res ? tmem + SFB_RES + 32u * (uint32_t)b
-                                                    : tmem + SF_COL + SF_SET_COLS * (uint32_t)b + 16u;
-                        for (int j = 0; j < nks; ++j) {
-                            if (need_sfa) tmem_cp_32x128b_x4_pair(ta + 4u * j, dfa + 32u * j);
-                            tmem_cp_32x128b_x4_pair(tb + 8u * j, dfb + 32u * j);
-                            tmem_cp_32x128b_x4_pair(tb + 8u * j + 4u, dfb + 128u + 32u * j);
-                        }
-                    }
-                    tc_commit_pair(&sf_ready[b], 0x1);
-                    if (++s == kStages) {
-                        s = 0;
-                        ph ^= 1u;
-                    }
-                }
-            }
-        }
-    } else if (warp == kMmaWarp) {
-        // ------------------------------------------------- MMA issuer (CTA 0)
-        if (rank == 0 && lane == 0) {
-            // The tensor pipe queues very few instructions, so every cycle this
-            // thread spends between MMAs is a bubble: stage and phase are kept
-            // incrementally, descriptors are formed once per stage and advanced
-            // by adding to their address field, and full stages are unrolled.
-            const uint32_t idesc_fp4 = idesc_m(idesc_nvfp4(BN), BM);
-            const uint32_t idesc_lr = idesc_m(idesc_bf16_f32(BN), BM);
-            const uint32_t smem0 = smem_u32(smem);
-            bool ok = true;
-            int local = 0, s = 0, it = 0;
-            uint32_t ph = 0;
-            for (int tile = t_begin; tile < t_end && ok; ++tile, ++local) {
                 if (!mbar_wait(acc_empty, ((uint32_t)local & 1u) ^ 1u, kSiteGpAccEmpty)) {
                     s_failed = 1;
                     break;
                 }
                 tc_fence_after();
-                for (int kk = 0; kk < per_tile; ++kk, ++it) {
-                    const int b = it & 1;
-                    // the copy thread saw the stage full before its scale copies
-                    // completed; the second wait is then already satisfied
-                    if (!mbar_wait(&sf_ready[b], (uint32_t)(it >> 1) & 1u, kSiteGpSfReady) ||
-                        !mbar_wait(&full[s], ph, kSiteGpFull)) {
+                // FP4 stages
+                for (int kk = 0; kk < n_kb; ++kk, ++it) {
+                    if (!mbar_wait(&full[s], ph, kSiteGpFull)) {
                         ok = false;
                         s_failed = 1;
                         break;
@@ -299,30 +254,49 @@ __global__ void __launch_bounds__(gp::kThreads, 1)
                     tc_fence_after();
                     const uint32_t sa = smem0 + (uint32_t)s * STAGE_BYTES;
                     const uint64_t da = desc_sw128(sa), db = desc_sw128(sa + A_BYTES);   // + 2 per 32-byte K-step
-                    if (kk < n_kb) {
-                        const int nks = min(4, a.kg4 - 4 * kk);
-                        const uint32_t ta = sfa_res ? tmem + SFA_RES + 16u * (uint32_t)kk
-                                                    : tmem + SF_COL + SF_SET_COLS * (uint32_t)b;
-                        const uint32_t tb = sfa_res ? tmem + SFB_RES + 32u * (uint32_t)b
-                                                    : tmem + SF_COL + SF_SET_COLS * (uint32_t)b + 16u;
-                        auto mma = [&](int j) {
+                    const uint64_t dfa = desc_sf_block(sa + A_BYTES + B_BYTES);         // + 32 per 512 bytes
+                    const uint64_t dfb = dfa + (uint64_t)(SFA_BYTES >> 4);
+                    // activation-scale columns of this stage's K-steps, weight-scale set
+                    const uint32_t ta = sfa_res ? tmem + SFA_RES + 16u * (uint32_t)kk
+                                                : tmem + SF_COL + SF_SET_COLS * (uint32_t)(it & 1);
+                    const uint32_t tb = sfa_res ? tmem + SFB_RES + 32u * (uint32_t)(it & 1) : ta + 16u;
+                    const uint32_t acc0 = kk > 0 ? 1u : 0u;
+                    if (kk + 1 < n_kb || nks_last == 4) {
+                        if (need_sfa)
+                            gp_issue_stage<true>(tmem + ACC_COL, da, db, dfa, dfb, ta, tb, idesc_fp4, acc0);
+                        else
+                            gp_issue_stage<false>(tmem + ACC_COL, da, db, dfa, dfb, ta, tb, idesc_fp4, acc0);
+                    } else {
+                        // a last stage of fewer than four K-steps
+                        for (int j = 0; j < nks_last; ++j) {
+                            if (need_sfa) tmem_cp_32x128b_x4_pair(ta + 4u * j, dfa + 32u * j);
+                            tmem_cp_32x128b_x4_pair(tb + 8u * j, dfb + 32u * j);
+                            tmem_cp_32x128b_x4_pair(tb + 8u * j + 4u, dfb + 128u + 32u * j);
                             mma_nvfp4_pair(tmem + ACC_COL, da + 2u * j, db + 2u * j, idesc_fp4, ta + 4u * j,
                                            tb + 8u * j, (kk > 0 || j > 0) ? 1u : 0u);
-                        };
-                        if (nks == 4) {
-#pragma unroll
-                            for (int j = 0; j < 4; ++j) mma(j);
-                        } else {
-                            for (int j = 0; j < nks; ++j) mma(j);
                         }
-                    } else {
-                        const int c = (kk - n_kb) >> 1;
-                        const int nks = min(4, (a.rank - 64 * c + 15) / 16);
-                        for (int j = 0; j < nks; ++j)
-                            mma_bf16_pair(tmem + ACC_COL, da + 2u * j, db + 2u * j, idesc_lr, 1u);
                     }
                     tc_commit_pair(&empty[s], 0x3);
-                    tc_commit_pair(&sf_free[b], 0x1);
+                    if (++s == kStages) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                }
+                // rank-r stages: bf16 MMAs of the hi and lo parts into the same accumulator
+                for (int kk = n_kb; kk < per_tile && ok; ++kk, ++it) {
+                    if (!mbar_wait(&full[s], ph, kSiteGpFull)) {
+                        ok = false;
+                        s_failed = 1;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sa = smem0 + (uint32_t)s * STAGE_BYTES;
+                    const uint64_t da = desc_sw128(sa), db = desc_sw128(sa + A_BYTES);
+                    const int c = (kk - n_kb) >> 1;
+                    const int nks = min(4, (a.rank - 64 * c + 15) / 16);
+                    for (int j = 0; j < nks; ++j)
+                        mma_bf16_pair(tmem + ACC_COL, da + 2u * j, db + 2u * j, idesc_lr, 1u);
+                    tc_commit_pair(&empty[s], 0x3);
                     if (++s == kStages) {
                         s = 0;
                         ph ^= 1u;
