@@ -35,7 +35,7 @@ METRIC = "SVDQ W4A4 linear TFLOPS (2MNK) and % of B200 dense FP4 tensor peak"
 # they are now (profiles/gemm_nvfp4_pair_qkv.md, profiles/quantize_act_nvfp4_qkv.md).
 # Set an entry to None whenever its kernel changes until it is profiled again.
 PROFILED_DRAM_BYTES = {
-    "gemm_nvfp4_pair_kernel": None,
+    "gemm_nvfp4_pair_kernel": 25369344 + 32259072,
     "quantize_act_kernel": 28766208 + 0,
 }
 UNIT = "TFLOPS"
