@@ -81,19 +81,65 @@ def aggregate(per_rank_flops: float, world: int, t_max_s: float) -> float:
 
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
-    """Samples SM clocks and throttle reasons with nvidia-smi while running."""
+    """SM clock, power and clock-event (throttle) reasons of one GPU while the
+    timed region runs.
+
+    NVML is polled every millisecond from a thread (read-only queries; ctypes
+    releases the GIL), so that even a timed region of a few milliseconds gets
+    samples; only samples taken between begin() and end() count.  Without NVML
+    it falls back to nvidia-smi at 100 ms."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits
+    REASON_BITS = (("sw_power_cap", 0x4), ("hw_slowdown", 0x8), ("sw_thermal_slowdown", 0x20),
+                   ("hw_thermal_slowdown", 0x40), ("hw_power_brake_slowdown", 0x80))
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: int, torch_device=None):
         self.gpu = gpu_index
+        self.torch_device = torch_device
         self.proc = None
         self.lines = []
+        self.samples = []          # (t, sm_mhz, power_w, reason bits)
         self._t = None
+        self._stop = threading.Event()
+        self._nvml = None
+        self._handle = None
+        self._max_mhz = None
+        self.t_begin = self.t_end = None
+
+    def _nvml_handle(self):
+        import pynvml
+
+        pynvml.nvmlInit()
+        handle = None
+        if self.torch_device is not None:
+            try:
+                import torch
+
+                u = str(torch.cuda.get_device_properties(self.torch_device).uuid)
+                handle = pynvml.nvmlDeviceGetHandleByUUID(u if u.startswith("GPU-") else "GPU-" + u)
+            except Exception:
+                handle = None
+        if handle is None:
+            idx = self.gpu
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+            ids = [v.strip() for v in vis.split(",") if v.strip()]
+            if ids and all(v.isdigit() for v in ids) and self.gpu < len(ids):
+                idx = int(ids[self.gpu])
+            handle = pynvml.nvmlDeviceGetHandleByIndex(idx)
+        return pynvml, handle
 
     def start(self):
+        try:
+            self._nvml, self._handle = self._nvml_handle()
+            self._max_mhz = float(self._nvml.nvmlDeviceGetMaxClockInfo(self._handle, self._nvml.NVML_CLOCK_SM))
+            self._t = threading.Thread(target=self._poll_nvml, daemon=True)
+            self._t.start()
+            return
+        except Exception:
+            self._nvml = None
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
@@ -103,11 +149,46 @@ class ClockSampler:
         except OSError:
             self.proc = None
 
+    def _poll_nvml(self):
+        nv, h = self._nvml, self._handle
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self._stop.is_set():
+            try:
+                t = time.perf_counter()
+                sm = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+                rs = int(get_reasons(h))
+                self.samples.append((t, sm, pw, rs))
+            except Exception:
+                break
+            time.sleep(0.001)
+
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.perf_counter(), line.strip()))
+
+    def begin(self):
+        self.t_begin = time.perf_counter()
+
+    def end(self):
+        self.t_end = time.perf_counter()
+
+    def _in_region(self, t):
+        return (self.t_begin is None or t >= self.t_begin) and (self.t_end is None or t <= self.t_end)
 
     def stop(self) -> dict:
+        if self._nvml is not None:
+            self._stop.set()
+            if self._t:
+                self._t.join(timeout=2)
+            rows = [r for r in self.samples if self._in_region(r[0])]
+            if not rows:
+                return {"sm_mhz": None, "sm_max_mhz": self._max_mhz, "reasons": ["no samples in the timed region"]}
+            reasons = sorted({name for _, _, _, bits in rows for name, bit in self.REASON_BITS if bits & bit})
+            return {"sm_mhz": statistics.median(r[1] for r in rows), "sm_max_mhz": self._max_mhz,
+                    "reasons": reasons, "samples": len(rows), "power_w_max": max(r[2] for r in rows),
+                    "source": "NVML every 1 ms during the timed region"}
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         self.proc.terminate()
@@ -119,7 +200,7 @@ class ClockSampler:
             self._t.join(timeout=2)
         sm, smax, power, reasons = [], [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        for t, ln in self.lines:
             parts = [p.strip() for p in ln.split(",")]
             if len(parts) < 9:
                 continue
@@ -136,7 +217,7 @@ class ClockSampler:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
         loaded = [s for s, p in zip(sm, power) if p > 0.3 * max(power)] or sm
         return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
-                "samples": len(sm), "power_w_max": max(power)}
+                "samples": len(sm), "power_w_max": max(power), "source": "nvidia-smi every 100 ms"}
 
 
 # ------------------------------------------------------------------ CUDA arm
@@ -193,14 +274,15 @@ def run_cuda(args) -> dict | None:
         raise RuntimeError(f"device status {st} at site {site} during warm-up")
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
-    sampler = ClockSampler(local)
+    sampler = ClockSampler(local, dev)
     sampler.start()
-    time.sleep(0.3)
+    time.sleep(0.05)
     if world > 1:
         import torch.distributed as dist
 
         dist.barrier()
     torch.cuda.synchronize(dev)
+    sampler.begin()
     for i in range(args.steps):
         flush.fill_(i & 0xFF)
         evs[i][0].record(stream)
@@ -209,6 +291,7 @@ def run_cuda(args) -> dict | None:
         gemm()
         evs[i][2].record(stream)
     torch.cuda.synchronize(dev)
+    sampler.end()
     if world > 1:
         dist.barrier()
     clocks = sampler.stop()
