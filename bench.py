@@ -80,13 +80,44 @@ def aggregate(per_rank_flops: float, world: int, t_max_s: float) -> float:
 
 
 # ------------------------------------------------------------------ clocks
+# Polls one GPU's SM clock, power and clock-event reasons through NVML every
+# millisecond and prints "t,sm_mhz,power_w,reason_bits" lines (t: the
+# system-wide monotonic clock).  Read-only queries; run as its own process so
+# that the bench's Python launch loop cannot starve it of the GIL.
+SAMPLER_SRC = r"""
+import sys, time
+import pynvml
+pynvml.nvmlInit()
+h = None
+if sys.argv[1]:
+    try:
+        h = pynvml.nvmlDeviceGetHandleByUUID(sys.argv[1])
+    except Exception:
+        h = None
+if h is None:
+    h = pynvml.nvmlDeviceGetHandleByIndex(int(sys.argv[2]))
+print("max,%d" % pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM), flush=True)
+get_r = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+while True:
+    t = time.monotonic()
+    sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+    try:
+        pw = pynvml.nvmlDeviceGetPowerUsage(h) / 1000.0
+    except Exception:
+        pw = 0.0
+    try:
+        rs = int(get_r(h))
+    except Exception:
+        rs = 0
+    print("%.6f,%d,%.1f,%d" % (t, sm, pw, rs), flush=True)
+    time.sleep(0.001)
+"""
+
+
 class ClockSampler:
     """SM clock, power and clock-event (throttle) reasons of one GPU while the
-    timed region runs.
-
-    NVML is polled every millisecond from a thread (read-only queries; ctypes
-    releases the GIL), so that even a timed region of a few milliseconds gets
-    samples; only samples taken between begin() and end() count.  Without NVML
+    timed region runs: a child process polls NVML every millisecond (see
+    SAMPLER_SRC); only samples between begin() and end() count.  Without NVML
     it falls back to nvidia-smi at 100 ms."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -100,97 +131,70 @@ class ClockSampler:
         self.gpu = gpu_index
         self.torch_device = torch_device
         self.proc = None
+        self.mode = None
         self.lines = []
-        self.samples = []          # (t, sm_mhz, power_w, reason bits)
         self._t = None
-        self._stop = threading.Event()
-        self._nvml = None
-        self._handle = None
-        self._max_mhz = None
+        self._ready = threading.Event()
+        self.max_mhz = None
         self.t_begin = self.t_end = None
 
-    def _nvml_handle(self):
-        import pynvml
-
-        pynvml.nvmlInit()
-        handle = None
+    def _nvml_index_and_uuid(self):
+        idx = self.gpu
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+        ids = [v.strip() for v in vis.split(",") if v.strip()]
+        if ids and all(v.isdigit() for v in ids) and self.gpu < len(ids):
+            idx = int(ids[self.gpu])
+        uuid = ""
         if self.torch_device is not None:
             try:
                 import torch
 
                 u = str(torch.cuda.get_device_properties(self.torch_device).uuid)
-                handle = pynvml.nvmlDeviceGetHandleByUUID(u if u.startswith("GPU-") else "GPU-" + u)
+                uuid = u if u.startswith("GPU-") else "GPU-" + u
             except Exception:
-                handle = None
-        if handle is None:
-            idx = self.gpu
-            vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
-            ids = [v.strip() for v in vis.split(",") if v.strip()]
-            if ids and all(v.isdigit() for v in ids) and self.gpu < len(ids):
-                idx = int(ids[self.gpu])
-            handle = pynvml.nvmlDeviceGetHandleByIndex(idx)
-        return pynvml, handle
+                uuid = ""
+        return idx, uuid
 
     def start(self):
+        idx, uuid = self._nvml_index_and_uuid()
         try:
-            self._nvml, self._handle = self._nvml_handle()
-            self._max_mhz = float(self._nvml.nvmlDeviceGetMaxClockInfo(self._handle, self._nvml.NVML_CLOCK_SM))
-            self._t = threading.Thread(target=self._poll_nvml, daemon=True)
+            self.proc = subprocess.Popen([sys.executable, "-c", SAMPLER_SRC, uuid, str(idx)],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.mode = "nvml"
+            self._t = threading.Thread(target=self._read, daemon=True)
             self._t.start()
-            return
-        except Exception:
-            self._nvml = None
+            self._ready.wait(timeout=20.0)
+            if self.max_mhz is not None:
+                return
+            self._kill()
+        except OSError:
+            self.proc = None
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
                  "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.mode = "smi"
+            self.lines = []
             self._t = threading.Thread(target=self._read, daemon=True)
             self._t.start()
         except OSError:
             self.proc = None
-
-    def _poll_nvml(self):
-        nv, h = self._nvml, self._handle
-        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
-            nv.nvmlDeviceGetCurrentClocksThrottleReasons
-        while not self._stop.is_set():
-            try:
-                t = time.perf_counter()
-                sm = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
-                pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
-                rs = int(get_reasons(h))
-                self.samples.append((t, sm, pw, rs))
-            except Exception:
-                break
-            time.sleep(0.001)
+            self.mode = None
 
     def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append((time.perf_counter(), line.strip()))
+        proc = self.proc
+        for line in proc.stdout:
+            line = line.strip()
+            if self.mode == "nvml" and line.startswith("max,"):
+                self.max_mhz = float(line.split(",")[1])
+                self._ready.set()
+                continue
+            self.lines.append((time.monotonic(), line))
+        self._ready.set()      # the poller ended (or never started): stop waiting for it
 
-    def begin(self):
-        self.t_begin = time.perf_counter()
-
-    def end(self):
-        self.t_end = time.perf_counter()
-
-    def _in_region(self, t):
-        return (self.t_begin is None or t >= self.t_begin) and (self.t_end is None or t <= self.t_end)
-
-    def stop(self) -> dict:
-        if self._nvml is not None:
-            self._stop.set()
-            if self._t:
-                self._t.join(timeout=2)
-            rows = [r for r in self.samples if self._in_region(r[0])]
-            if not rows:
-                return {"sm_mhz": None, "sm_max_mhz": self._max_mhz, "reasons": ["no samples in the timed region"]}
-            reasons = sorted({name for _, _, _, bits in rows for name, bit in self.REASON_BITS if bits & bit})
-            return {"sm_mhz": statistics.median(r[1] for r in rows), "sm_max_mhz": self._max_mhz,
-                    "reasons": reasons, "samples": len(rows), "power_w_max": max(r[2] for r in rows),
-                    "source": "NVML every 1 ms during the timed region"}
+    def _kill(self):
         if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+            return
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
@@ -198,9 +202,41 @@ class ClockSampler:
             self.proc.kill()
         if self._t:
             self._t.join(timeout=2)
+
+    def begin(self):
+        self.t_begin = time.monotonic()
+
+    def end(self):
+        self.t_end = time.monotonic()
+
+    def _in_region(self, t):
+        return (self.t_begin is None or t >= self.t_begin) and (self.t_end is None or t <= self.t_end)
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no clock sampler available"]}
+        self._kill()
+        if self.mode == "nvml":
+            rows = []
+            for _, ln in self.lines:
+                parts = ln.split(",")
+                if len(parts) != 4:
+                    continue
+                try:
+                    t, sm, pw, rs = float(parts[0]), float(parts[1]), float(parts[2]), int(parts[3])
+                except ValueError:
+                    continue
+                if self._in_region(t):
+                    rows.append((sm, pw, rs))
+            if not rows:
+                return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["no samples in the timed region"]}
+            reasons = sorted({name for _, _, bits in rows for name, bit in self.REASON_BITS if bits & bit})
+            return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": self.max_mhz,
+                    "reasons": reasons, "samples": len(rows), "power_w_max": max(r[1] for r in rows),
+                    "source": "NVML every 1 ms during the timed region"}
         sm, smax, power, reasons = [], [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for t, ln in self.lines:
+        for _, ln in self.lines:
             parts = [p.strip() for p in ln.split(",")]
             if len(parts) < 9:
                 continue
