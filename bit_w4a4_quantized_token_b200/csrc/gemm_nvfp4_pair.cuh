@@ -10,9 +10,10 @@
 //     of its own 128 activation rows and the scale blocks of all 256 weight
 //     rows (the tensor core reads the weight scales of every column in both
 //     halves of the pair);
-//   * CTA 0 alone copies the scale blocks into both CTAs' TMEM (a copy warp)
-//     and issues one M = 256, N = 256 MMA per 64 values of K (the MMA warp);
-//     the accumulator rows of CTA r sit in CTA r's TMEM;
+//   * one thread of CTA 0 copies the scale blocks into both CTAs' TMEM and
+//     issues one M = 256, N = 256 MMA per 64 values of K, each copy right
+//     before the MMA ahead of the one that reads it; the accumulator rows of
+//     CTA r sit in CTA r's TMEM;
 //   * every load of either CTA completes on CTA 0's stage barrier, CTA 0's
 //     commits arrive on both CTAs' "stage free" and "accumulator full"
 //     barriers, and both CTAs' epilogue warps hand the accumulator back on
