@@ -1,18 +1,24 @@
 """Benchmark of the SVDQ W4A4 linear layer (nvfp4, group 16, rank 32).
 
-One step = one forward of the layer on the fused-QKV projection of a DiT at
-1024x1024 (4096 image + 512 text tokens): M=4608, K=3072, N=9216, rank 32,
-i.e. svdq_quantize_act followed by svdq_gemm_w4a4, inputs resident in HBM,
-L2 flushed (256 MiB write) before every step.  The weight side is packed
-once before timing (offline in the layer's life cycle).
+One step = one forward of the layer: svdq_quantize_act followed by
+svdq_gemm_w4a4, inputs resident in HBM, L2 flushed (256 MiB write) before
+every step outside the timed events.  The headline workload is the fused-QKV
+projection of a DiT at 1024x1024 (4096 image + 512 text tokens): M=4608,
+K=3072, N=9216, rank 32.  The weight side is packed once before timing
+(offline in the layer's life cycle).  Each step is replayed from a CUDA graph
+of the two launches, so host launch overhead stays out of the device time.
+The other DiT shapes (MLP fc1 / fc2, the batch-4 attention out-projection over
+ranks 0..128, the int4 variant) are reported under "extra" with the same
+measurements.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {cuda,reference}]
+                    [--config NAME] [--no-extra] [--dynamic-scale] [--no-cpu-baseline]
 
 Multi-GPU (torchrun, one rank per GPU): every rank runs its own batch of
 tokens through its own replica of the packed weight (weak scaling, no
 collective on the data path); the step time is the max over ranks.
---impl reference times the CPU oracle on the host cores on a bounded sample
-of rows of the same workload.
+--impl reference times the CPU oracle on the host cores: each step is the
+oracle on a bounded sample of rows of the same workload.
 """
 from __future__ import annotations
 
@@ -30,16 +36,14 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "SVDQ W4A4 linear TFLOPS (2MNK) and % of B200 dense FP4 tensor peak"
-
-# DRAM bytes (read + write) per launch from one ncu capture of the kernels as
-# they are now (profiles/gemm_nvfp4_pair_qkv.md, profiles/quantize_act_nvfp4_qkv.md).
-# Set an entry to None whenever its kernel changes until it is profiled again.
-PROFILED_DRAM_BYTES = {
-    "gemm_nvfp4_pair_kernel": 25369344 + 32259072,
-    "quantize_act_kernel": 28766208 + 0,
-}
 UNIT = "TFLOPS"
 FP4_OVER_BF16 = 4.0        # nominal dense FP4 : BF16 tensor throughput on B200 (9 : 2.25 PFLOP/s)
+# dense block-scaled FP4 work one SM retires per clock: an M128 N256 K64
+# kind::mxf4nvf4 MMA (4.19 MFLOP) every 128 cycles, measured on this B200
+FP4_FLOP_PER_CLK_SM = 32768
+# DRAM bytes per launch taken from ncu captures, with the hash of the kernel
+# sources they were taken on; a value whose sources changed since is not used
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic.json")
 
 
 def load_peaks() -> dict:
@@ -256,11 +260,257 @@ class ClockSampler:
                 "samples": len(sm), "power_w_max": max(power), "source": "nvidia-smi every 100 ms"}
 
 
+# ------------------------------------------------------------------ helpers
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+
+    return platform.processor() or "unknown"
+
+
+def workload_config(case, dynamic_scale: bool, world: int) -> dict:
+    """The `config` object of both arms (identical for the same workload)."""
+    names = {"qkv": "DiT fused-QKV projection, 1024^2 (4096 image + 512 text tokens)",
+             "fc1": "DiT MLP fc1, 1024^2 (4096 image + 512 text tokens)",
+             "fc2": "DiT MLP fc2, 1024^2 (4096 image + 512 text tokens), GELU input",
+             "int4_qkv": "DiT fused-QKV projection, int4 W4A4 variant"}
+    name = names.get(case.name, f"batch-4 DiT attention out-projection, rank {case.rank}"
+                     if case.name.startswith("outproj") else case.name)
+    return {"workload": name, "M": case.M, "K": case.K, "N": case.N, "rank": case.rank,
+            "group_size": case.group_size, "precision": case.precision,
+            "x_tensor_scale": "dynamic (amax pre-pass)" if dynamic_scale else "static (calibrated)",
+            "l2": "flushed before every step (256 MiB write, outside the timed events)",
+            "step": "svdq_quantize_act + svdq_gemm_w4a4", "parallelism": f"replicas x{world} (tokens)"}
+
+
+def quant_bytes(case) -> int:
+    """Algorithmic HBM bytes of the activation quantizer: x read once; codes,
+    group scales and the rank-r activations (hi and lo bf16 planes) written once."""
+    M, K, r = case.M, case.K, case.rank
+    if case.precision == "nvfp4":
+        return M * K * 2 + M * K // 2 + M * K // 16 + 4 * M * r
+    return M * K * 2 + M * K // 2 + 2 * M * K // 64 + 4 * M * r
+
+
+def gemm_bytes(case) -> int:
+    """Algorithmic HBM bytes of the GEMM: both operands' codes and scales read
+    once, the rank-r operands and bias read once, y written once."""
+    M, K, N, r = case.M, case.K, case.N, case.rank
+    sc = (M + N) * K // 16 if case.precision == "nvfp4" else 2 * (M + N) * K // 64
+    return (M + N) * K // 2 + sc + 4 * M * r + 2 * N * r + 2 * N + 2 * M * N
+
+
+def profiled_traffic(kernel: str):
+    """(bytes per launch, note) from the committed ncu summary when the kernel's
+    sources are unchanged since it was taken, else (None, why)."""
+    import hashlib
+
+    try:
+        with open(TRAFFIC_FILE) as f:
+            entry = json.load(f)["kernels"][kernel]
+    except (OSError, KeyError, ValueError):
+        return None, "no ncu capture recorded for this kernel"
+    h = hashlib.sha256()
+    for rel in entry["source_files"]:
+        try:
+            with open(os.path.join(ROOT, rel), "rb") as f:
+                h.update(f.read())
+        except OSError:
+            return None, f"source {rel} missing"
+    if h.hexdigest() != entry["source_sha256"]:
+        return None, "kernel sources changed since the ncu capture"
+    return int(entry["dram_bytes_per_launch"]), f"ncu capture on the {entry['workload']} workload"
+
+
+def fp4_peaks(peaks: dict, sm_mhz) -> dict:
+    """The FP4 roofline: measured bf16 burst x the nominal FP4:BF16 ratio, and
+    the MMA rate at the SM clock sampled during the run."""
+    out = {"peak": peaks["bf16_tflops"] * FP4_OVER_BF16,
+           "peak_source": f"{peaks['source']} bf16 burst {peaks['bf16_tflops']} x {FP4_OVER_BF16} (nominal FP4:BF16)"}
+    if sm_mhz:
+        out["peak_at_clock"] = 148 * FP4_FLOP_PER_CLK_SM * sm_mhz * 1e6 / 1e12
+    return out
+
+
 # ------------------------------------------------------------------ CUDA arm
+class Shape:
+    """One workload on the device: packed weight, buffers, graphs of the step."""
+
+    def __init__(self, case, dev, stream, dynamic_scale=False):
+        import torch
+
+        from bit_w4a4_quantized_token_b200 import _lib, layer
+        from bit_w4a4_quantized_token_b200 import workloads as W
+
+        self.case, self.dev, self.stream = case, dev, stream
+        inp = W.make_inputs(case)
+        self.x_host = inp["x"]
+        d = {k: v.to(dev) for k, v in inp.items()}
+        r = case.rank
+        self.packed = layer.pack_weight(d["R"], d["lam"], d["L_down"] if r else None, d["L_up"] if r else None,
+                                        d["b"], precision=case.precision)
+        self.x = d["x"]
+        self.q = layer.alloc_act(self.packed, case.M, dev)
+        self.y = torch.empty(case.M, case.N, dtype=torch.bfloat16, device=dev)
+        # static activation tensor scale, calibrated once (the amax pre-pass)
+        layer.quantize_act(self.x, self.packed, out=self.q)
+        self.compute_scale = 1 if dynamic_scale else 0
+        self._lib = _lib
+        torch.cuda.synchronize(dev)
+
+    def quant(self):
+        c, p, q = self.case, self.packed, self.q
+        self._lib.svdq_quantize_act(c.precision, c.group_size, self.x, c.M, c.K, p.inv_lambda, q.x_tensor_scale,
+                                    self.compute_scale, p.w_tensor_scale, p.L_down_t, c.rank, q.x_codes, q.x_scales,
+                                    q.lowrank_act, q.workspace, stream=self.stream)
+
+    def gemm(self):
+        c, p, q = self.case, self.packed, self.q
+        self._lib.svdq_gemm_w4a4(c.precision, c.group_size, q.x_codes, q.x_scales, q.x_tensor_scale, c.M, p.w_codes,
+                                 p.w_scales, p.w_tensor_scale, c.N, c.K, q.lowrank_act, p.L_up_t, c.rank, p.bias, self.y,
+                                 stream=self.stream)
+
+    def graphs(self):
+        """CUDA graphs of the step and of each kernel (captured after warm-up)."""
+        import torch
+
+        gs = {}
+        for name, fns in (("step", (self.quant, self.gemm)), ("quant", (self.quant,)), ("gemm", (self.gemm,))):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=self.stream):
+                for fn in fns:
+                    fn()
+            gs[name] = g
+        return gs
+
+
+def time_qkv_fusion(dev, stream, flush, steps: int) -> dict:
+    """The QKV projection with the attention-input RMSNorm + RoPE (24 heads of
+    128): fused into the GEMM epilogue against the unfused path (the plain
+    GEMM, then the separate norm + rotary pass over its bf16 output)."""
+    import torch
+
+    from bit_w4a4_quantized_token_b200 import _lib
+    from bit_w4a4_quantized_token_b200 import workloads as W
+
+    case = W.QKV
+    heads = case.N // (3 * W.QKV_HEAD_DIM)
+    with torch.cuda.stream(stream):
+        sh = Shape(case, dev, stream)
+        ex = W.qkv_inputs(case.M, heads)
+        d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in ex.items()}
+    p, q = sh.packed, sh.q
+
+    def fused():
+        _lib.svdq_gemm_w4a4_qkv_norm_rope("nvfp4", 16, q.x_codes, q.x_scales, q.x_tensor_scale, case.M, p.w_codes,
+                                          p.w_scales, p.w_tensor_scale, case.N, case.K, q.lowrank_act, p.L_up_t,
+                                          case.rank, p.bias, heads, W.QKV_HEAD_DIM, d["norm_q"], d["norm_k"],
+                                          W.QKV_EPS, d["cos"], d["sin"], sh.y, stream=stream)
+
+    def norm_rope():
+        _lib.svdq_qkv_norm_rope(sh.y, sh.y, case.M, heads, W.QKV_HEAD_DIM, d["norm_q"], d["norm_k"], W.QKV_EPS,
+                                d["cos"], d["sin"], stream=stream)
+
+    gs = {}
+    for name, fns in (("fused", (sh.quant, fused)), ("unfused", (sh.quant, sh.gemm, norm_rope))):
+        with torch.cuda.stream(stream):
+            for i in range(3):
+                flush.fill_(i)
+                for fn in fns:
+                    fn()
+        torch.cuda.synchronize(dev)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for fn in fns:
+                fn()
+        gs[name] = g
+    res = {}
+    for name, g in gs.items():
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        torch.cuda.synchronize(dev)
+        with torch.cuda.stream(stream):
+            for i in range(steps):
+                flush.fill_(i & 0xFF)
+                evs[i][0].record(stream)
+                g.replay()
+                evs[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+        res[name] = sum(a.elapsed_time(b) for a, b in evs) / steps / 1e3
+    st, site = _lib.svdq_device_status(clear=True)
+    if st != 0:
+        raise RuntimeError(f"device status {st} at site {site} in the QKV fusion leg")
+    del gs, sh
+    return {"workload": "DiT fused-QKV projection + per-head RMSNorm + RoPE (24 heads x 128), M=4608 K=3072 N=9216 "
+                        "rank 32",
+            "step_us": {"fused": round(res["fused"] * 1e6, 2), "unfused": round(res["unfused"] * 1e6, 2)},
+            "speedup": round(res["unfused"] / res["fused"], 3),
+            "value": round(case.flops / res["fused"] / 1e12, 2), "unit": UNIT,
+            "unfused_step": "svdq_quantize_act + svdq_gemm_w4a4 + svdq_qkv_norm_rope (in place)",
+            "fused_step": "svdq_quantize_act + svdq_gemm_w4a4_qkv_norm_rope"}
+
+
+def time_graphs(shape, gs, steps, flush, sampler=None):
+    """Device time per step of each graph (CUDA events on the launching stream,
+    L2 flushed before every replay, outside the events)."""
+    import torch
+
+    st = shape.stream
+    res = {}
+    for name in ("step", "quant", "gemm"):
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        torch.cuda.synchronize(shape.dev)
+        if sampler is not None and name == "step":
+            sampler.begin()
+        with torch.cuda.stream(st):
+            for i in range(steps):
+                flush.fill_(i & 0xFF)
+                evs[i][0].record(st)
+                gs[name].replay()
+                evs[i][1].record(st)
+        torch.cuda.synchronize(shape.dev)
+        if sampler is not None and name == "step":
+            sampler.end()
+        res[name] = sum(a.elapsed_time(b) for a, b in evs) / steps / 1e3
+    return res
+
+
+def shape_report(case, t: dict, peaks: dict, sm_mhz, world: int) -> dict:
+    flops = case.flops
+    fp = fp4_peaks(peaks, sm_mhz)
+    gemm_tf = flops / t["gemm"] / 1e12
+    qb = quant_bytes(case)
+    out = {"workload": workload_config(case, False, world)["workload"],
+           "M": case.M, "K": case.K, "N": case.N, "rank": case.rank, "precision": case.precision,
+           "value": round(aggregate(flops, world, t["step"]), 2), "unit": UNIT if case.precision == "nvfp4" else "TOPS",
+           "breakdown_us": {"step": round(t["step"] * 1e6, 2), "quantize_act": round(t["quant"] * 1e6, 2),
+                            "gemm_w4a4": round(t["gemm"] * 1e6, 2)},
+           "quantizer_roofline": {"bound": "hbm", "achieved": round(qb / t["quant"] / 1e9, 1),
+                                  "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                  "frac": round(qb / t["quant"] / 1e9 / peaks["hbm_gbs"], 4), "bytes": qb}}
+    if case.precision == "nvfp4":
+        g = {"bound": "tensor", "achieved": round(gemm_tf, 2), "peak": round(fp["peak"], 1), "unit": "TFLOP/s",
+             "frac": round(gemm_tf / fp["peak"], 4)}
+        if "peak_at_clock" in fp:
+            g["frac_at_clock"] = round(gemm_tf / fp["peak_at_clock"], 4)
+        out["roofline"] = g
+    else:
+        out["roofline"] = {"bound": "issue (per-group rescale on the CUDA cores)", "achieved": round(gemm_tf, 2),
+                           "unit": "TOP/s"}
+    if case.rank:
+        out["lowrank_flops_not_counted"] = 2 * case.M * case.rank * (case.K + 2 * case.N)
+    return out
+
+
 def run_cuda(args) -> dict | None:
     import torch
 
-    from bit_w4a4_quantized_token_b200 import _lib, layer
+    from bit_w4a4_quantized_token_b200 import _lib
     from bit_w4a4_quantized_token_b200 import workloads as W
 
     world, rank, local = dist_env()
@@ -273,194 +523,138 @@ def run_cuda(args) -> dict | None:
 
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
-    case = W.QKV
-    M, K, N, r = case.M, case.K, case.N, case.rank
-    inp = W.make_inputs(case)
-    d = {k: v.to(dev) for k, v in inp.items()}
-    stream = torch.cuda.current_stream(dev)
-    packed = layer.pack_weight(d["R"], d["lam"], d["L_down"], d["L_up"], d["b"], precision="nvfp4")
-    q = layer.alloc_act(packed, M, dev)
-    y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
-    # static activation tensor scale, calibrated once (the amax pre-pass)
-    layer.quantize_act(d["x"], packed, out=q)
-    if args.dynamic_scale:
-        compute_scale = 1
-    else:
-        compute_scale = 0
+    case = W.BY_NAME[args.config]
+    stream = torch.cuda.Stream(dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-    x = d["x"]
-
-    def step():
-        _lib.svdq_quantize_act("nvfp4", 16, x, M, K, packed.inv_lambda, q.x_tensor_scale, compute_scale,
-                               packed.w_tensor_scale, packed.L_down_t, r, q.x_codes, q.x_scales, q.lowrank_act,
-                               q.workspace, stream=stream)
-
-    def gemm():
-        _lib.svdq_gemm_w4a4("nvfp4", 16, q.x_codes, q.x_scales, q.x_tensor_scale, M, packed.w_codes,
-                            packed.w_scales, packed.w_tensor_scale, N, K, q.lowrank_act, packed.L_up_t, r,
-                            packed.bias, y, stream=stream)
-
-    for _ in range(args.warmup):
-        flush.fill_(1)
-        step()
-        gemm()
+    with torch.cuda.stream(stream):
+        sh = Shape(case, dev, stream, args.dynamic_scale)
+        for i in range(args.warmup):
+            flush.fill_(i & 0xFF)
+            sh.quant()
+            sh.gemm()
     torch.cuda.synchronize(dev)
     st, site = _lib.svdq_device_status(clear=True)
     if st != 0:
         raise RuntimeError(f"device status {st} at site {site} during warm-up")
+    gs = sh.graphs()
+    for g in gs.values():   # warm the graphs too
+        for i in range(2):
+            flush.fill_(i)
+            g.replay()
+    torch.cuda.synchronize(dev)
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     sampler = ClockSampler(local, dev)
     sampler.start()
     time.sleep(0.05)
     if world > 1:
-        import torch.distributed as dist
-
         dist.barrier()
-    torch.cuda.synchronize(dev)
-    sampler.begin()
-    for i in range(args.steps):
-        flush.fill_(i & 0xFF)
-        evs[i][0].record(stream)
-        step()
-        evs[i][1].record(stream)
-        gemm()
-        evs[i][2].record(stream)
-    torch.cuda.synchronize(dev)
-    sampler.end()
+    t = time_graphs(sh, gs, args.steps, flush, sampler)
     if world > 1:
         dist.barrier()
     clocks = sampler.stop()
     st, site = _lib.svdq_device_status(clear=True)
     if st != 0:
         raise RuntimeError(f"device status {st} at site {site} in the timed region")
-    t_quant = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps / 1e3
-    t_gemm = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps / 1e3
-    t_step = max_over_ranks(t_quant + t_gemm, world, dev)
-    t_gemm_max = max_over_ranks(t_gemm, world, dev)
-    t_quant_max = max_over_ranks(t_quant, world, dev)
+    t = {k: max_over_ranks(v, world, dev) for k, v in t.items()}
 
     # end to end through the public API: pinned host x -> device, forward, y -> pinned host
-    x_host = inp["x"].pin_memory()
-    y_host = torch.empty(M, N, dtype=torch.bfloat16).pin_memory()
-    x_dev = torch.empty_like(x)
+    x_host = sh.x_host.pin_memory()
+    y_host = torch.empty(case.M, case.N, dtype=torch.bfloat16).pin_memory()
     e2e_steps = max(1, min(args.steps, 20))
-    for _ in range(2):
-        x_dev.copy_(x_host, non_blocking=True)
-        layer.gemm(layer.quantize_act(x_dev, packed, out=q, x_tensor_scale=q.x_tensor_scale), packed, y=y)
-        y_host.copy_(y, non_blocking=True)
-    torch.cuda.synchronize(dev)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if world > 1:
-        dist.barrier()
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        x_dev.copy_(x_host, non_blocking=True)
-        _lib.svdq_quantize_act("nvfp4", 16, x_dev, M, K, packed.inv_lambda, q.x_tensor_scale, compute_scale,
-                               packed.w_tensor_scale, packed.L_down_t, r, q.x_codes, q.x_scales, q.lowrank_act,
-                               q.workspace, stream=stream)
-        gemm()
-        y_host.copy_(y, non_blocking=True)
-    e1.record(stream)
+    with torch.cuda.stream(stream):
+        for i in range(2 + e2e_steps):
+            if i == 2:
+                torch.cuda.synchronize(dev)
+                if world > 1:
+                    dist.barrier()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+            sh.x.copy_(x_host, non_blocking=True)
+            sh.quant()
+            sh.gemm()
+            y_host.copy_(sh.y, non_blocking=True)
+        e1.record(stream)
     torch.cuda.synchronize(dev)
     t_e2e = max_over_ranks(e0.elapsed_time(e1) / e2e_steps / 1e3, world, dev)
-    # the int4 W4A4 variant on the same QKV shape (group 64, bf16 scales): reported beside the headline
-    int4 = time_int4(args, dev, stream, flush)
+    del gs
+
+    peaks = load_peaks()
+    report = shape_report(case, t, peaks, clocks.get("sm_mhz"), world)
+    extra = {}
+    if world == 1 and not args.no_extra:
+        names = ["qkv", "fc1", "fc2"] + [f"outproj_r{r}" for r in (0, 16, 32, 64, 128)] + ["int4_qkv"]
+        for name in names:
+            if name == case.name:
+                continue
+            c = W.BY_NAME[name]
+            with torch.cuda.stream(stream):
+                s2 = Shape(c, dev, stream)
+                for i in range(3):
+                    flush.fill_(i)
+                    s2.quant()
+                    s2.gemm()
+            g2 = s2.graphs()
+            t2 = time_graphs(s2, g2, max(3, min(args.steps, 10)), flush)
+            st, site = _lib.svdq_device_status(clear=True)
+            if st != 0:
+                raise RuntimeError(f"device status {st} at site {site} on {name}")
+            extra[name] = shape_report(c, t2, peaks, clocks.get("sm_mhz"), world)
+            del g2, s2
+            torch.cuda.empty_cache()
+        extra["qkv_norm_rope"] = time_qkv_fusion(dev, stream, flush, max(3, min(args.steps, 10)))
+        torch.cuda.empty_cache()
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
     if rank != 0:
         return None
 
-    flops = case.flops
-    peaks = load_peaks()
-    fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16
-    gemm_tflops = flops / t_gemm_max / 1e12
-    quant_bytes = M * K * 2 + M * K // 2 + M * K // 16 + 4 * M * r + K * 4
-    launches = (2 if not args.dynamic_scale else 4) * args.steps   # quantize_act + gemm per step
-    extra = {"int4_qkv": int4}
+    traffic, traffic_note = profiled_traffic("gemm_nvfp4_pair_kernel")
+    qtraffic, qtraffic_note = profiled_traffic("quantize_act_kernel")
+    roofline = dict(report["roofline"], kernel="gemm_nvfp4_pair_kernel",
+                    peak_source=fp4_peaks(peaks, None)["peak_source"], traffic=traffic, traffic_note=traffic_note,
+                    algorithmic_bytes=gemm_bytes(case))
+    if "frac_at_clock" in roofline:
+        roofline["peak_at_clock_note"] = (f"148 SMs x {FP4_FLOP_PER_CLK_SM} FLOP/clk x the sampled "
+                                          f"{clocks.get('sm_mhz')} MHz; the 60 % target is judged against `peak`")
+    qroof = dict(report["quantizer_roofline"], kernel="quantize_act_kernel", traffic=qtraffic,
+                 traffic_note=qtraffic_note)
+    # our kernels launched in the timed passes: the step graph (quantizer, GEMM)
+    # and then the quantizer and GEMM graphs alone, `steps` replays each
+    n_quant = 1 + (2 if args.dynamic_scale else 0)   # + the amax pre-pass and its finalisation
+    launches = 2 * (n_quant + 1) * args.steps
     return {
         "metric": METRIC,
-        "value": round(aggregate(flops, world, t_step), 3),
+        "value": report["value"],
         "unit": UNIT,
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
-        "ms_per_step": round(t_step * 1e3, 5),
+        "ms_per_step": round(t["step"] * 1e3, 5),
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "nvfp4 (e2m1 x e2m1, ue4m3 group scales) -> fp32 accumulate -> bf16",
+        "dtype": "nvfp4 (e2m1 x e2m1, ue4m3 group scales) -> fp32 accumulate -> bf16"
+                 if case.precision == "nvfp4" else "int4 x int4 (bf16 group scales) -> int32 / fp32 -> bf16",
         "data": "synthetic (seeded DiT-shaped activations with 1% outlier channels; random-init weights)",
-        "config": {"workload": "DiT fused-QKV projection, 1024^2 (4096 image + 512 text tokens)",
-                   "M": M, "K": K, "N": N, "rank": r, "group_size": 16, "precision": "nvfp4",
-                   "x_tensor_scale": "dynamic (amax pre-pass)" if args.dynamic_scale else "static (calibrated)",
-                   "l2": "flushed before every step (256 MiB write, outside the timed events)",
-                   "step": "svdq_quantize_act + svdq_gemm_w4a4", "parallelism": f"replicas x{world} (tokens)"},
-        "breakdown_us": {"quantize_act": round(t_quant_max * 1e6, 2), "gemm_w4a4": round(t_gemm_max * 1e6, 2)},
-        "roofline": {"bound": "tensor", "kernel": "gemm_nvfp4_pair_kernel", "achieved": round(gemm_tflops, 2),
-                     "peak": round(fp4_peak, 1), "unit": "TFLOP/s", "frac": round(gemm_tflops / fp4_peak, 4),
-                     "peak_source": f"{peaks['source']} bf16 burst {peaks['bf16_tflops']} x {FP4_OVER_BF16} (nominal FP4:BF16)",
-                     "traffic": PROFILED_DRAM_BYTES.get("gemm_nvfp4_pair_kernel")},
-        "quantizer_roofline": {"bound": "hbm", "kernel": "quantize_act_kernel",
-                               "achieved": round(quant_bytes / t_quant_max / 1e9, 1), "peak": peaks["hbm_gbs"],
-                               "unit": "GB/s", "frac": round(quant_bytes / t_quant_max / 1e9 / peaks["hbm_gbs"], 4),
-                               "traffic": PROFILED_DRAM_BYTES.get("quantize_act_kernel")},
-        "e2e": {"value": round(aggregate(flops, world, t_e2e), 3), "unit": UNIT,
-                "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2},
+        "config": workload_config(case, args.dynamic_scale, world),
+        "breakdown_us": report["breakdown_us"],
+        "roofline": roofline,
+        "quantizer_roofline": qroof,
+        "e2e": {"value": round(aggregate(case.flops, world, t_e2e), 3), "unit": UNIT,
+                "h2d_bytes_per_step": case.M * case.K * 2, "d2h_bytes_per_step": case.M * case.N * 2},
         "gpu_launches": launches,
         "clocks": clocks,
         "extra": extra,
     }
 
 
-def time_int4(args, dev, stream, flush) -> dict:
-    """Device time of the int4 W4A4 layer (quantize + GEMM) on the QKV shape."""
-    import torch
-
-    from bit_w4a4_quantized_token_b200 import _lib, layer
-    from bit_w4a4_quantized_token_b200 import workloads as W
-
-    case = W.INT4_QKV
-    M, K, N, r = case.M, case.K, case.N, case.rank
-    inp = W.make_inputs(case)
-    d = {k: v.to(dev) for k, v in inp.items()}
-    packed = layer.pack_weight(d["R"], d["lam"], d["L_down"], d["L_up"], d["b"], precision="int4")
-    q = layer.alloc_act(packed, M, dev)
-    y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
-    steps = max(3, min(args.steps, 10))
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
-    for i in range(args.warmup + steps):
-        flush.fill_(i & 0xFF)
-        j = i - args.warmup
-        if j >= 0:
-            evs[j][0].record(stream)
-        layer.quantize_act(d["x"], packed, out=q, stream=stream)
-        if j >= 0:
-            evs[j][1].record(stream)
-        layer.gemm(q, packed, y=y, stream=stream)
-        if j >= 0:
-            evs[j][2].record(stream)
-    torch.cuda.synchronize(dev)
-    st, site = _lib.svdq_device_status(clear=True)
-    if st != 0:
-        raise RuntimeError(f"device status {st} at site {site} in the int4 leg")
-    tq = sum(e[0].elapsed_time(e[1]) for e in evs) / steps / 1e3
-    tg = sum(e[1].elapsed_time(e[2]) for e in evs) / steps / 1e3
-    return {"workload": "int4 W4A4 QKV projection M=4608 K=3072 N=9216 rank 32 group 64",
-            "value": round(case.flops / (tq + tg) / 1e12, 2), "unit": "TOPS",
-            "breakdown_us": {"quantize_act": round(tq * 1e6, 2), "gemm_w4a4": round(tg * 1e6, 2)}}
-
-
 # ------------------------------------------------------------------ CPU oracle
-def oracle_sample(target_s: float = 10.0):
-    """Times the CPU oracle on a bounded sample of rows of the same workload."""
-    import numpy as np
-
+def oracle_setup(case):
+    """Inputs of the workload and the offline (untimed) weight side, for the oracle."""
     from bit_w4a4_quantized_token_b200 import workloads as W
     from oracle import oracle as O
 
-    case = W.QKV
     inp = W.make_inputs(case)
     x, lam = W.bits(inp["x"]), inp["lam"].numpy()
     Ld, Lu, b = W.bits(inp["L_down"]), W.bits(inp["L_up"]), W.bits(inp["b"])
@@ -469,48 +663,74 @@ def oracle_sample(target_s: float = 10.0):
     wc, ws = O.nvfp4_quantize(R, None, S_w)
     wd = O.nvfp4_dequant(wc, ws, S_w)          # weight packing is offline: not timed
     S_x = O.nvfp4_tensor_scale(x, lam)         # static scale, as in the CUDA arm
-
-    def run(rows: int) -> float:
-        xs = np.ascontiguousarray(x[:rows])
-        t0 = time.perf_counter()
-        xc, xsc = O.nvfp4_quantize(xs, lam, S_x)
-        L = O.lowrank_down(xs, lam, Ld)
-        xd = O.nvfp4_dequant(xc, xsc, S_x)
-        O.nvfp4_linear(xd, wd, L, Lu, b)
-        return time.perf_counter() - t0
-
-    t64 = run(64)
-    rows = int(min(case.M, max(64, 64 * round(target_s / max(t64, 1e-3)))))
-    t = run(rows)
-    tflops = 2 * rows * case.N * case.K / t / 1e12
-    return case, rows, t, tflops, O.num_threads()
+    return {"x": x, "lam": lam, "Ld": Ld, "Lu": Lu, "b": b, "wd": wd, "S_x": S_x}
 
 
-def cpu_baseline_obj(target_s: float = 10.0) -> dict:
-    case, rows, t, tflops, cores = oracle_sample(target_s)
-    return {"value": round(tflops, 6), "unit": UNIT, "cores": cores, "kind": "oracle",
-            "sample": f"{rows} of {case.M} token rows of the QKV workload (quantize + rank-r + fp64 GEMM + bias), "
-                      f"{t:.1f} s on {cores} threads"}
+def oracle_pass(o, rows: int, start: int = 0) -> float:
+    """One oracle forward on `rows` token rows (quantize + rank-r + fp64 GEMM + bias); seconds."""
+    import numpy as np
+
+    from oracle import oracle as O
+
+    xs = np.ascontiguousarray(o["x"][start:start + rows])
+    t0 = time.perf_counter()
+    xc, xsc = O.nvfp4_quantize(xs, o["lam"], o["S_x"])
+    L = O.lowrank_down(xs, o["lam"], o["Ld"])
+    xd = O.nvfp4_dequant(xc, xsc, o["S_x"])
+    O.nvfp4_linear(xd, o["wd"], L, o["Lu"], o["b"])
+    return time.perf_counter() - t0
+
+
+def rows_for(o, case, seconds: float) -> int:
+    t64 = oracle_pass(o, 64)
+    return int(min(case.M, max(64, 64 * round(seconds / max(t64, 1e-3)))))
+
+
+def cpu_baseline_obj(case, target_s: float = 10.0) -> dict:
+    from oracle import oracle as O
+
+    o = oracle_setup(case)
+    rows = rows_for(o, case, target_s)
+    t = oracle_pass(o, rows)
+    cores = O.num_threads()
+    return {"value": round(2 * rows * case.N * case.K / t / 1e12, 6), "unit": UNIT, "cores": cores,
+            "cpu": cpu_model(), "kind": "oracle",
+            "sample": f"{rows} of {case.M} token rows of the {case.name} workload (quantize + rank-r + fp64 GEMM "
+                      f"+ bias), {t:.1f} s on {cores} threads"}
 
 
 def run_reference(args) -> dict | None:
+    """The oracle as it stands, timed on the host cores: `warmup` untimed and
+    `steps` timed passes, each over the same bounded sample of rows."""
+    from bit_w4a4_quantized_token_b200 import workloads as W
+    from oracle import oracle as O
+
     world, rank, _ = dist_env()
     if rank != 0:
         return None
-    cb = cpu_baseline_obj(target_s=max(3.0, min(20.0, 4.0 * args.steps)))
-    from bit_w4a4_quantized_token_b200 import workloads as W
-
-    case = W.QKV
-    v = cb["value"]
+    case = W.BY_NAME[args.config]
+    o = oracle_setup(case)
+    # size one pass so that warm-up + timed passes take about two minutes
+    per_pass = max(1.0, min(10.0, 120.0 / (args.steps + args.warmup)))
+    rows = rows_for(o, case, per_pass)
+    for i in range(args.warmup):
+        oracle_pass(o, rows, start=(i * rows) % max(1, case.M - rows + 1))
+    ts = [oracle_pass(o, rows, start=(i * rows) % max(1, case.M - rows + 1)) for i in range(args.steps)]
+    t = sum(ts) / len(ts)
+    v = 2 * rows * case.N * case.K / t / 1e12
+    cores = O.num_threads()
+    cb = {"value": round(v, 6), "unit": UNIT, "cores": cores, "cpu": cpu_model(), "kind": "oracle",
+          "sample": f"{rows} of {case.M} token rows of the {case.name} workload per step "
+                    f"(quantize + rank-r + fp64 GEMM + bias), {args.steps} timed + {args.warmup} warm-up passes, "
+                    f"{t:.2f} s per pass on {cores} threads"}
     return {
-        "impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": round(case.flops / (v * 1e12) * 1e3, 3) if v else None,
+        "impl": "reference", "metric": METRIC, "value": round(v, 6), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(t * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": {"workload": "DiT fused-QKV projection, 1024^2 (4096 image + 512 text tokens)",
-                                        "M": case.M, "K": case.K, "N": case.N, "rank": case.rank,
-                                        "group_size": 16, "precision": "nvfp4"},
+        "data": "synthetic (seeded DiT-shaped activations with 1% outlier channels; random-init weights)",
+        "config": workload_config(case, args.dynamic_scale, world),
         "cpu_baseline": cb,
-        "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "e2e": {"value": round(v, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
 
@@ -520,6 +740,10 @@ def main():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
+    ap.add_argument("--config", default="qkv",
+                    choices=["qkv", "fc1", "fc2", "outproj_r0", "outproj_r16", "outproj_r32", "outproj_r64",
+                             "outproj_r128", "int4_qkv"], help="the headline workload (default: the QKV projection)")
+    ap.add_argument("--no-extra", action="store_true", help="skip the other DiT shapes")
     ap.add_argument("--dynamic-scale", action="store_true", help="derive S_x by the amax pre-pass every step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -532,7 +756,9 @@ def main():
         world, rank, _ = dist_env()
         cb = None
         if world == 1 and not args.no_cpu_baseline:
-            cb = cpu_baseline_obj(target_s=10.0)
+            from bit_w4a4_quantized_token_b200 import workloads as W
+
+            cb = cpu_baseline_obj(W.BY_NAME[args.config] if args.config != "int4_qkv" else W.QKV, target_s=10.0)
         out = run_cuda(args)
         if out is not None:
             out["cpu_baseline"] = cb

@@ -30,9 +30,11 @@ GROUP_SIZES = {"nvfp4": 16, "int4": 64}
 EXPORTS = (
     "svdq_status_string", "svdq_abi_version", "svdq_last_error", "svdq_buffer_sizes", "svdq_pack_weight",
     "svdq_quantize_act_workspace_bytes", "svdq_quantize_act", "svdq_quantize_act_noalloc", "svdq_gemm_w4a4",
+    "svdq_gemm_w4a4_qkv_norm_rope", "svdq_qkv_norm_rope", "svdq_gemm_w4a16", "svdq_svd_split_workspace_bytes",
+    "svdq_svd_split",
     "svdq_device_status",
     "svdq_debug_set_wait_limit_ns", "svdq_debug_timeout_probe", "svdq_debug_override_capability",
-    "svdq_debug_force_gemm_tiles",
+    "svdq_debug_force_gemm_tiles", "svdq_debug_force_quant_plan",
 )
 
 
@@ -74,6 +76,18 @@ def _load():
     lib.svdq_quantize_act_noalloc.restype = I
     lib.svdq_gemm_w4a4.argtypes = [I, I, P, P, P, I64, P, P, P, I64, I64, P, P, I, P, P, P]
     lib.svdq_gemm_w4a4.restype = I
+    F = ctypes.c_float
+    lib.svdq_gemm_w4a4_qkv_norm_rope.argtypes = [I, I, P, P, P, I64, P, P, P, I64, I64, P, P, I, P, I, I, P, P, F,
+                                                 P, P, P, P]
+    lib.svdq_gemm_w4a4_qkv_norm_rope.restype = I
+    lib.svdq_qkv_norm_rope.argtypes = [P, P, I64, I, I, P, P, F, P, P, P]
+    lib.svdq_qkv_norm_rope.restype = I
+    lib.svdq_gemm_w4a16.argtypes = [P, I64, P, P, I64, I64, P, P, P]
+    lib.svdq_gemm_w4a16.restype = I
+    lib.svdq_svd_split_workspace_bytes.argtypes = [I64, I64, I, I, ctypes.POINTER(ctypes.c_size_t)]
+    lib.svdq_svd_split_workspace_bytes.restype = I
+    lib.svdq_svd_split.argtypes = [P, P, I64, I64, I, P, I, I, P, P, P, P, P, ctypes.c_size_t, P]
+    lib.svdq_svd_split.restype = I
     lib.svdq_device_status.argtypes = [I, ctypes.POINTER(ctypes.c_int)]
     lib.svdq_device_status.restype = I
     lib.svdq_debug_set_wait_limit_ns.argtypes = [U64]
@@ -84,6 +98,8 @@ def _load():
     lib.svdq_debug_override_capability.restype = None
     lib.svdq_debug_force_gemm_tiles.argtypes = [I]
     lib.svdq_debug_force_gemm_tiles.restype = I
+    lib.svdq_debug_force_quant_plan.argtypes = [I]
+    lib.svdq_debug_force_quant_plan.restype = I
     return lib
 
 
@@ -177,6 +193,45 @@ def svdq_gemm_w4a4(precision, group_size, x_codes, x_scales, x_tensor_scale, M, 
                               _stream(stream)), "svdq_gemm_w4a4")
 
 
+def svdq_gemm_w4a4_qkv_norm_rope(precision, group_size, x_codes, x_scales, x_tensor_scale, M, w_codes, w_scales,
+                                 w_tensor_scale, N, K, lowrank_act, L_up_t, rank, bias, heads, head_dim, norm_q,
+                                 norm_k, eps, rope_cos, rope_sin, y, stream=None) -> None:
+    _check(lib.svdq_gemm_w4a4_qkv_norm_rope(_prec(precision), int(group_size), _ptr(x_codes), _ptr(x_scales),
+                                            _ptr(x_tensor_scale), int(M), _ptr(w_codes), _ptr(w_scales),
+                                            _ptr(w_tensor_scale), int(N), int(K), _ptr(lowrank_act), _ptr(L_up_t),
+                                            int(rank), _ptr(bias), int(heads), int(head_dim), _ptr(norm_q),
+                                            _ptr(norm_k), float(eps), _ptr(rope_cos), _ptr(rope_sin), _ptr(y),
+                                            _stream(stream)), "svdq_gemm_w4a4_qkv_norm_rope")
+
+
+def svdq_qkv_norm_rope(y_in, y_out, M, heads, head_dim, norm_q, norm_k, eps, rope_cos, rope_sin,
+                       stream=None) -> None:
+    _check(lib.svdq_qkv_norm_rope(_ptr(y_in), _ptr(y_out), int(M), int(heads), int(head_dim), _ptr(norm_q),
+                                  _ptr(norm_k), float(eps), _ptr(rope_cos), _ptr(rope_sin), _stream(stream)),
+           "svdq_qkv_norm_rope")
+
+
+def svdq_gemm_w4a16(x, M, w_codes, w_scales, N, K, bias, y, stream=None) -> None:
+    _check(lib.svdq_gemm_w4a16(_ptr(x), int(M), _ptr(w_codes), _ptr(w_scales), int(N), int(K), _ptr(bias), _ptr(y),
+                               _stream(stream)), "svdq_gemm_w4a16")
+
+
+def svdq_svd_split_workspace_bytes(N: int, K: int, rank: int, oversample: int) -> int:
+    out = ctypes.c_size_t(0)
+    _check(lib.svdq_svd_split_workspace_bytes(int(N), int(K), int(rank), int(oversample), ctypes.byref(out)),
+           "svdq_svd_split_workspace_bytes")
+    return int(out.value)
+
+
+def svdq_svd_split(W, lam, N, K, rank, omega, oversample, power_iters, R, L_down, L_up, singular_values,
+                   workspace, workspace_bytes=0, stream=None) -> None:
+    if workspace is not None and not isinstance(workspace, int) and not workspace_bytes:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    _check(lib.svdq_svd_split(_ptr(W), _ptr(lam), int(N), int(K), int(rank), _ptr(omega), int(oversample),
+                              int(power_iters), _ptr(R), _ptr(L_down), _ptr(L_up), _ptr(singular_values),
+                              _ptr(workspace), int(workspace_bytes), _stream(stream)), "svdq_svd_split")
+
+
 def svdq_device_status(clear: bool = True) -> tuple[int, int]:
     """(status, site) after synchronising the device; does not raise."""
     site = ctypes.c_int(0)
@@ -197,6 +252,11 @@ def svdq_debug_override_capability(major: int, minor: int = 0) -> None:
 
 
 def svdq_debug_force_gemm_tiles(mode: int) -> None:
-    """nvfp4 GEMM kernel: 0 = automatic, 1 = single-CTA 128x256 tiles, 2 = CTA-pair 256x256
-    tiles, 3 = CTA-pair 256x128 tiles where K allows (else 256x256)."""
+    """nvfp4 GEMM kernel: 0 = automatic, 1 = single-CTA 128x256 tiles, 2 = CTA-pair tiles."""
     _check(lib.svdq_debug_force_gemm_tiles(int(mode)), "svdq_debug_force_gemm_tiles")
+
+
+def svdq_debug_force_quant_plan(mode: int) -> None:
+    """K-split reduction of the quantizer: 0 = automatic, 1 = workspace (global
+    memory), 2 = one thread-block cluster (distributed shared memory)."""
+    _check(lib.svdq_debug_force_quant_plan(int(mode)), "svdq_debug_force_quant_plan")

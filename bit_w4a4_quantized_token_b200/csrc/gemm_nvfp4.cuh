@@ -55,6 +55,15 @@ struct GemmArgs {
     int kg4;                     // K / 64: scale blocks per 128 rows
     int n_sf_blocks;             // ceil(N / 128): 128-row blocks present in w_scales
     int m_tiles, n_tiles;
+    // Fused QKV + RMSNorm + RoPE epilogue (pair kernel only; qk_cols == 0
+    // disables it): columns [0, q_cols) are the Q heads and [q_cols, qk_cols)
+    // the K heads (128 columns each) of a to_qkv projection.
+    const __nv_bfloat16* norm_q;   // [128] RMSNorm weights of the Q heads
+    const __nv_bfloat16* norm_k;   // [128] RMSNorm weights of the K heads
+    const float* rope_cos;         // [M, 64] per-token rotary tables
+    const float* rope_sin;
+    float eps;
+    int q_cols, qk_cols;
 };
 
 enum : uint32_t { kSiteGmEmpty = 16, kSiteGmFull = 17, kSiteGmAcc = 18, kSiteGmDrain = 19, kSiteGmAccEmpty = 20 };

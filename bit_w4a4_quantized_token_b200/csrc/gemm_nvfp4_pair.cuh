@@ -34,8 +34,19 @@
 // One thread issuing TMA copies manages roughly one stage every 600-700
 // cycles, whatever the box size, and a stage of four K-steps lasts 512 cycles
 // of MMA; so each producer role runs on two lanes that take alternate stages.
+//
+// With the fused QKV epilogue (kQkv, GemmArgs.qk_cols > 0) the warps whose 128
+// columns are a Q or K head apply that head's RMSNorm and rotary embedding
+// (qkv_norm_rope.cuh) to the fp32 results before the bf16 store.
+//
+// Measured alternative, not kept: four extra warps writing the scale factors
+// into TMEM with tcgen05.st (so that the MMA thread issues MMAs only) ran the
+// 4608 x 3072 x 9216 projection in 160-190 us against 107 us for this kernel;
+// their shared-memory reads of the staged scale blocks slowed the TMA fill of
+// the ring, whose stages then landed 3-5 us after issue.
 #pragma once
 #include "gemm_nvfp4.cuh"
+#include "qkv_norm_rope.cuh"
 
 namespace svdq {
 namespace gp {
@@ -108,6 +119,9 @@ __device__ __forceinline__ void gp_issue_stage(uint32_t acc, uint64_t da, uint64
     }
 }
 
+// kQkv: the fused QKV + RMSNorm + RoPE epilogue is compiled in (a separate
+// instantiation, so that the plain kernel keeps its registers).
+template <bool kQkv>
 __global__ void __launch_bounds__(gp::kThreads, 1)
     gemm_nvfp4_pair_kernel(const __grid_constant__ CUtensorMap tm_xc, const __grid_constant__ CUtensorMap tm_wc,
                            const __grid_constant__ CUtensorMap tm_sfa, const __grid_constant__ CUtensorMap tm_sfb,
@@ -166,6 +180,10 @@ __global__ void __launch_bounds__(gp::kThreads, 1)
     cluster_sync_all();       // barriers of both CTAs initialised, TMEM address written
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // Everything above overlaps the previous kernel under programmatic
+    // dependent launch (the activation quantizer releases its dependents
+    // early); from here on this kernel reads that kernel's outputs.
+    griddep_wait();
 
     if (warp == 0 || warp == 1) {
         // ----------------------------------------------------------- producers
@@ -338,6 +356,57 @@ __global__ void __launch_bounds__(gp::kThreads, 1)
             if (lane == 0) mbar_arrive_cluster(acc_empty_leader);   // this half of the pair is drained
             if (grow >= a.M) continue;
             __nv_bfloat16* yrow = a.y + grow * (int64_t)a.N;
+            if (kQkv && nbase < a.qk_cols) {
+                // this warp's 128 columns are one Q or K head of a to_qkv
+                // projection (qkv_norm_rope.cuh): RMSNorm over them, then the
+                // rotary pairs, on the fp32 values before the single bf16 rounding
+                float ss = 0.0f;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const int n = nbase + 16 * c;
+                    uint4 w0 = make_uint4(0u, 0u, 0u, 0u), w1 = w0;
+                    if (a.bias) {
+                        w0 = __ldg(reinterpret_cast<const uint4*>(a.bias + n));
+                        w1 = __ldg(reinterpret_cast<const uint4*>(a.bias + n) + 1);
+                    }
+                    const uint32_t ws[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+                    for (int p = 0; p < 8; ++p) {
+                        const float o0 = fmaf(__uint_as_float(acc[16 * c + 2 * p]), S, bf16lo_to_f32(ws[p]));
+                        const float o1 = fmaf(__uint_as_float(acc[16 * c + 2 * p + 1]), S, bf16hi_to_f32(ws[p]));
+                        acc[16 * c + 2 * p] = __float_as_uint(o0);
+                        acc[16 * c + 2 * p + 1] = __float_as_uint(o1);
+                        ss = fmaf(o0, o0, ss);
+                        ss = fmaf(o1, o1, ss);
+                    }
+                }
+                const float r = rsqrtf(ss * (1.0f / 128.0f) + a.eps);
+                const __nv_bfloat16* w = nbase < a.q_cols ? a.norm_q : a.norm_k;
+                const float4* cs4 = reinterpret_cast<const float4*>(a.rope_cos + grow * 64);
+                const float4* sn4 = reinterpret_cast<const float4*>(a.rope_sin + grow * 64);
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {   // 16 columns = 8 rotary pairs
+                    const uint4 g0 = __ldg(reinterpret_cast<const uint4*>(w + 16 * c));
+                    const uint4 g1 = __ldg(reinterpret_cast<const uint4*>(w + 16 * c) + 1);
+                    const uint32_t gs[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+                    const float4 c0 = __ldg(cs4 + 2 * c), c1 = __ldg(cs4 + 2 * c + 1);
+                    const float4 s0 = __ldg(sn4 + 2 * c), s1 = __ldg(sn4 + 2 * c + 1);
+                    const float cc[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+                    const float sc[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+                    uint32_t packed[8];
+#pragma unroll
+                    for (int p = 0; p < 8; ++p) {
+                        const float v0 = __uint_as_float(acc[16 * c + 2 * p]) * r * bf16lo_to_f32(gs[p]);
+                        const float v1 = __uint_as_float(acc[16 * c + 2 * p + 1]) * r * bf16hi_to_f32(gs[p]);
+                        const __nv_bfloat162 h = __floats2bfloat162_rn(v0 * cc[p] - v1 * sc[p], v1 * cc[p] + v0 * sc[p]);
+                        packed[p] = *reinterpret_cast<const uint32_t*>(&h);
+                    }
+                    uint4* dst = reinterpret_cast<uint4*>(yrow + nbase + 16 * c);
+                    dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+                    dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+                }
+                continue;
+            }
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
                 const int n = nbase + 16 * c;

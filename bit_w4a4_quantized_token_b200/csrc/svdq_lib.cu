@@ -18,7 +18,9 @@
 #include "quantize_act.cuh"
 #include "gemm_nvfp4.cuh"
 #include "gemm_nvfp4_pair.cuh"
-#include "gemm_nvfp4_pair128.cuh"
+#include "qkv_norm_rope.cuh"
+#include "svd_split.cuh"
+#include "gemm_w4a16.cuh"
 #include "int4.cuh"
 
 namespace svdq {
@@ -65,6 +67,7 @@ std::mutex g_mutex;
 int g_override_major = -1, g_override_minor = 0;
 constexpr int kMaxDevices = 64;
 std::atomic<int> g_gemm_tiles_mode{0};   // svdq_debug_force_gemm_tiles
+std::atomic<int> g_quant_plan_mode{0};   // svdq_debug_force_quant_plan
 bool g_device_ready[kMaxDevices];
 
 // Budget of dynamic shared memory for the activation quantizer (the opt-in
@@ -121,10 +124,12 @@ svdq_status check_device() {
                                  kQuantSmemBudget) != cudaSuccess ||
             cudaFuncSetAttribute(gemm_int4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)i4::SMEM_BYTES) != cudaSuccess ||
-            cudaFuncSetAttribute(gemm_nvfp4_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            cudaFuncSetAttribute(gemm_w4a16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)aw::SMEM_BYTES) != cudaSuccess ||
+            cudaFuncSetAttribute(gemm_nvfp4_pair_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)gp::SMEM_BYTES) != cudaSuccess ||
-            cudaFuncSetAttribute(gemm_nvfp4_pair128_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)gq::SMEM_BYTES) != cudaSuccess)
+            cudaFuncSetAttribute(gemm_nvfp4_pair_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)gp::SMEM_BYTES) != cudaSuccess)
             return cuda_fail("setting kernel shared-memory limits");
         g_device_ready[dev] = true;
     }
@@ -151,9 +156,11 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// 2-D row-major tensor [outer, inner] with 128-byte swizzled boxes.
+// 2-D row-major tensor [outer, inner] with 128-byte swizzled boxes (or
+// unswizzled ones).
 bool make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
-              uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
+              uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+              CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t dims[2] = {inner, outer};
@@ -161,8 +168,7 @@ bool make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t
     const cuuint32_t box[2] = {box_inner, box_outer};
     const cuuint32_t estr[2] = {1, 1};
     const CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                          swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS)
         snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled failed (CUresult %d)", (int)r);
     return r == CUDA_SUCCESS;
@@ -206,15 +212,23 @@ bool make_sf_map(CUtensorMap* m, const void* base, uint64_t row_blocks, uint64_t
     return r == CUDA_SUCCESS;
 }
 
-int g_num_sms = 0;
+// SM count of the current device (looked up once per device).
 int num_sms() {
-    if (g_num_sms == 0) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev);
-        if (g_num_sms <= 0) g_num_sms = 148;
+    static std::atomic<int> per_dev[kMaxDevices];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        return 148;
     }
-    return g_num_sms;
+    int n = per_dev[dev].load();
+    if (n == 0) {
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+            cudaGetLastError();
+            n = 148;
+        }
+        per_dev[dev].store(n);
+    }
+    return n;
 }
 
 // ---------------------------------------------------------- nvfp4 paths
@@ -260,11 +274,91 @@ int quant_splits(int64_t M, int64_t K) {
     return (int)std::max<int64_t>(sp, 1);
 }
 
+// Workspace of the K-split when its CTAs add their rank-r partials through
+// global memory (the upper bound: a launch that runs in cluster mode leaves
+// the workspace untouched).
 size_t quant_workspace_bytes(int64_t M, int64_t K, int rank) {
     const int sp = quant_splits(M, K);
     if (rank == 0 || sp == 1) return 0;
     const int64_t row_blocks = (M + qa::kRows - 1) / qa::kRows;
     return (size_t)round_up(row_blocks * 4, 256) + (size_t)row_blocks * sp * qa::kRows * rank * 4;
+}
+
+// Clusters of `c` quantizer CTAs that can be resident at once on the current
+// device (one CTA per SM), looked up once per device and size.
+int quant_max_clusters(int c) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        return 0;
+    }
+    static int cache[kMaxDevices][qa::kMaxCluster + 1];
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (cache[dev][c] == 0) {
+        cudaLaunchConfig_t cfg = {};
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = (unsigned)c;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.gridDim = dim3((unsigned)c * 256u, 1, 1);
+        cfg.blockDim = dim3(qa::kThreads, 1, 1);
+        cfg.dynamicSmemBytes = kQuantSmemBudget;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, quantize_act_kernel<kPrecNvfp4>, &cfg) != cudaSuccess || n < 0) {
+            cudaGetLastError();
+            n = 0;
+        }
+        cache[dev][c] = n + 1;   // stored + 1 so that 0 means "not looked up"
+    }
+    return cache[dev][c] - 1;
+}
+
+// How the K range is split: `splits` CTAs per 128-row block; cluster mode
+// (cluster == splits) when those CTAs can form one cluster and every row
+// block's cluster is resident at once, else the workspace (cluster == 1).
+struct QuantPlan {
+    int splits, cluster;
+};
+QuantPlan quant_plan(int64_t M, int64_t K, int rank) {
+    const int sp = quant_splits(M, K);
+    if (rank == 0 || sp == 1) return {sp, 1};
+    const int mode = g_quant_plan_mode.load();
+    if (mode == 1) return {sp, 1};
+    if (mode == 2) return {std::min(sp, qa::kMaxCluster), std::min(sp, qa::kMaxCluster)};
+    const int64_t row_blocks = (M + qa::kRows - 1) / qa::kRows;
+    for (int c = std::min(sp, qa::kMaxCluster); c >= 2; --c)
+        if (quant_max_clusters(c) >= row_blocks) return {c, c};
+    return {sp, 1};
+}
+
+// Launch with programmatic stream serialisation (the kernel waits for the
+// previous grid with griddepcontrol.wait) and an optional cluster shape.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_ex(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                      unsigned cluster_x, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[2];
+    int n = 0;
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+    if (cluster_x > 1) {
+        attr[n].id = cudaLaunchAttributeClusterDimension;
+        attr[n].val.clusterDim.x = cluster_x;
+        attr[n].val.clusterDim.y = 1;
+        attr[n].val.clusterDim.z = 1;
+        ++n;
+    }
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = (unsigned)n;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
 // Activation quantizer launch (both precisions).  x_scale / w_scale are only
@@ -284,6 +378,8 @@ svdq_status quantize_act_launch(int prec, const void* x, int64_t M, int64_t K, c
     }
     const int64_t row_blocks = (M + qa::kRows - 1) / qa::kRows;
     if (row_blocks > 65535) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+    const QuantPlan plan = quant_plan(M, K, rank);
+    if (plan.cluster == 1 && plan.splits > 1 && rank > 0 && workspace == nullptr) return SVDQ_ERR_INVALID_ARG;
     QuantActArgs a;
     a.inv_lambda = inv_lambda;
     a.x_scale = x_scale;
@@ -296,26 +392,32 @@ svdq_status quantize_act_launch(int prec, const void* x, int64_t M, int64_t K, c
     a.rank = rank;
     a.rows_pad = (int)round_up(M, 128);
     a.chunks = (int)(K / 64);
-    a.splits = quant_splits(M, K);
+    a.splits = plan.splits;
+    a.cluster = plan.cluster;
     a.counters = reinterpret_cast<unsigned int*>(workspace);
     a.partials = workspace ? reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(workspace) +
                                                        round_up(row_blocks * 4, 256))
                            : nullptr;
-    a.stage_bytes = (uint32_t)qa::kXBytes + (uint32_t)rank * 256u;   // x tile + hi and lo L_down_t tiles
-    a.max_chunks = (a.chunks + a.splits - 1) / a.splits;
-    const size_t fixed = 1024 + (size_t)a.max_chunks * qa::kCols * 4 + 128 * 4 + (2 * qa::kMaxStages + 1) * 8 + 16;
+    // stage: x tile, hi and lo L_down_t tiles, the chunk's 1/lambda; 1 KB aligned (128-byte swizzle)
+    a.invl_off = (uint32_t)qa::kXBytes + (uint32_t)rank * 256u;
+    a.stage_bytes = (uint32_t)round_up((int64_t)a.invl_off + qa::kInvlBytes, 1024);
+    const size_t fixed = 1024 + 128 * 4 + (2 * qa::kMaxStages + 1) * 8 + 16;
     const int stages = (int)std::min<size_t>(qa::kMaxStages, (kQuantSmemBudget - fixed) / a.stage_bytes);
-    if (stages < 2 || fixed >= (size_t)kQuantSmemBudget) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+    if (stages < 2) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+    // the rank-r partial is staged in the ring once streaming is over
+    if ((size_t)stages * a.stage_bytes < (size_t)qa::kRows * (rank + 4) * 4) return SVDQ_ERR_UNSUPPORTED_SHAPE;
     a.stages = stages;
     uint32_t tcols = 32;
     while ((int)tcols < 2 * rank) tcols *= 2;   // x . hi and x . lo accumulators
     a.tmem_cols = tcols;
     const size_t smem = fixed + (size_t)stages * a.stage_bytes;
     const dim3 grid((unsigned)a.splits, (unsigned)row_blocks, 1);
-    if (prec == kPrecNvfp4)
-        quantize_act_kernel<kPrecNvfp4><<<grid, qa::kThreads, smem, st>>>(tm_x, tm_ld, a);
-    else
-        quantize_act_kernel<kPrecInt4><<<grid, qa::kThreads, smem, st>>>(tm_x, tm_ld, a);
+    const unsigned cl = (unsigned)a.cluster;
+    const cudaError_t e =
+        prec == kPrecNvfp4
+            ? launch_ex(quantize_act_kernel<kPrecNvfp4>, grid, dim3(qa::kThreads), smem, st, cl, tm_x, tm_ld, a)
+            : launch_ex(quantize_act_kernel<kPrecInt4>, grid, dim3(qa::kThreads), smem, st, cl, tm_x, tm_ld, a);
+    if (e != cudaSuccess) return cuda_fail("quantize_act_kernel launch");
     return launch_status("quantize_act_kernel launch");
 }
 
@@ -325,6 +427,24 @@ svdq_status quantize_act_nvfp4(const void* x, int64_t M, int64_t K, const float*
     if (compute_scale) SVDQ_TRY(tensor_scale_prepass(x, inv_lambda, M, K, x_scale, st));
     return quantize_act_launch(kPrecNvfp4, x, M, K, inv_lambda, x_scale, w_scale, L_down_t, rank, x_codes, x_scales,
                                lowrank, workspace, st);
+}
+
+// --------------------------------------------------- offline SVD split
+size_t svd_split_workspace(int64_t N, int64_t K, int l) {
+    const size_t f = sizeof(float), d = sizeof(double);
+    const size_t mm = (size_t)sv::kMaxL * sv::kMaxL;
+    return (size_t)round_up((int64_t)(N * l * f), 256) + (size_t)round_up((int64_t)(K * l * f), 256) +
+           (size_t)sv::kGramBlocks * mm * d + 2 * mm * d + sv::kMaxL * d;
+}
+
+// Orthonormal columns of A [rows, l] in place: CholeskyQR2.
+svdq_status svd_orth(float* A, int64_t rows, int l, double* part, double* Rinv, cudaStream_t st) {
+    for (int pass = 0; pass < 2; ++pass) {
+        svd_gram_partial_kernel<<<sv::kGramBlocks, 256, 0, st>>>(A, rows, l, part);
+        svd_chol_inv_kernel<<<1, 64, 0, st>>>(part, sv::kGramBlocks, l, Rinv);
+        svd_apply_rinv_kernel<<<(unsigned)((rows + 255) / 256), 256, 0, st>>>(A, rows, l, Rinv);
+    }
+    return launch_status("SVD split: orthonormalisation");
 }
 
 // ----------------------------------------------------------- int4 paths
@@ -356,7 +476,7 @@ svdq_status gemm_nvfp4(const void* x_codes, const void* x_scales, const float* x
         tm_L = tm_xc;
         tm_Lup = tm_wc;
     }
-    GemmArgs a;
+    GemmArgs a = {};
     a.x_scales = reinterpret_cast<const uint8_t*>(x_scales);
     a.w_scales = reinterpret_cast<const uint8_t*>(w_scales);
     a.x_scale = x_scale;
@@ -381,12 +501,13 @@ svdq_status gemm_nvfp4(const void* x_codes, const void* x_scales, const float* x
 // Clusters of two CTAs that fit on the device at once (one CTA per SM; both
 // pair kernels have the same block size and nearly all of shared memory).
 int pair_clusters() {
-    static int per_dev[kMaxDevices];
+    static std::atomic<int> per_dev[kMaxDevices];
     int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 0 || dev >= kMaxDevices) return num_sms() / 2;
-    static_assert(gq::kThreads == gp::kThreads, "pair kernels differ in block size");
-    if (per_dev[dev] == 0) {
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        return num_sms() / 2;
+    }
+    if (per_dev[dev].load() == 0) {
         cudaLaunchConfig_t cfg = {};
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -399,89 +520,30 @@ int pair_clusters() {
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         int n = 0;
-        if (cudaOccupancyMaxActiveClusters(&n, gemm_nvfp4_pair_kernel, &cfg) != cudaSuccess || n <= 0) {
+        if (cudaOccupancyMaxActiveClusters(&n, gemm_nvfp4_pair_kernel<false>, &cfg) != cudaSuccess || n <= 0) {
             cudaGetLastError();
             n = num_sms() / 2;
         }
-        per_dev[dev] = n;
+        per_dev[dev].store(n);
     }
-    return per_dev[dev];
-}
-
-// 256 x 128 tiles on CTA pairs with the weight scales resident in TMEM (M >
-// 128, K <= 3072, K % 512 == 0).  Selected only on request: on B200 its MMA
-// thread issues an N = 128 MMA and its scale copy in about 205 cycles, against
-// about 170 cycles per N = 256 MMA (twice the work) in the 256 x 256 kernel,
-// so it is the slower of the two (136 against 111 us on the 4608 x 3072 x
-// 9216 projection).
-bool pair128_applies(int64_t M, int64_t K) {
-    return M > 128 && K % 512 == 0 && K / 64 <= gq::kMaxKSteps;
-}
-
-svdq_status gemm_nvfp4_pair128(const void* x_codes, const void* x_scales, const float* x_scale, int64_t M,
-                               const void* w_codes, const void* w_scales, const float* w_scale, int64_t N, int64_t K,
-                               const void* lowrank, const void* L_up_t, int rank, const void* bias, void* y,
-                               cudaStream_t st) {
-    CUtensorMap tm_xc, tm_wc, tm_sfa, tm_sfb, tm_L, tm_Lup;
-    const int64_t kg4 = K / 64;
-    if (!make_map(&tm_xc, CU_TENSOR_MAP_DATA_TYPE_UINT8, x_codes, (uint64_t)K / 2, (uint64_t)M, (uint64_t)K / 2,
-                  gq::CHUNK, 128) ||
-        !make_map(&tm_wc, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_codes, (uint64_t)K / 2, (uint64_t)N, (uint64_t)K / 2,
-                  gq::CHUNK, 64) ||
-        !make_sf_map(&tm_sfa, x_scales, (uint64_t)((M + 127) / 128), (uint64_t)kg4, 1, gq::KSTEPS) ||
-        !make_sf_map(&tm_sfb, w_scales, (uint64_t)((N + 127) / 128), (uint64_t)kg4, 1, gq::KSTEPS))
-        return SVDQ_ERR_CUDA;
-    if (rank > 0) {
-        if (!make_map_3d(&tm_L, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, lowrank, (uint64_t)rank, (uint64_t)M, 2,
-                         (uint64_t)rank * 2, 64, 128, 1) ||
-            !make_map(&tm_Lup, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L_up_t, (uint64_t)rank, (uint64_t)N,
-                      (uint64_t)rank * 2, 64, 64))
-            return SVDQ_ERR_CUDA;
-    } else {
-        tm_L = tm_xc;
-        tm_Lup = tm_wc;
-    }
-    GemmArgs a;
-    a.x_scales = reinterpret_cast<const uint8_t*>(x_scales);
-    a.w_scales = reinterpret_cast<const uint8_t*>(w_scales);
-    a.x_scale = x_scale;
-    a.w_scale = w_scale;
-    a.bias = reinterpret_cast<const __nv_bfloat16*>(bias);
-    a.y = reinterpret_cast<__nv_bfloat16*>(y);
-    a.M = (int)M;
-    a.N = (int)N;
-    a.K = (int)K;
-    a.rank = rank;
-    a.kg4 = (int)kg4;
-    a.n_sf_blocks = (int)((N + 127) / 128);
-    const int64_t mt = (M + gq::BM - 1) / gq::BM, nt = (N + gq::BN - 1) / gq::BN;
-    if (mt * nt > (int64_t(1) << 30)) return SVDQ_ERR_UNSUPPORTED_SHAPE;
-    a.m_tiles = (int)mt;
-    a.n_tiles = (int)nt;
-    const int clusters = (int)std::min<int64_t>(mt * nt, pair_clusters());
-    cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.gridDim = dim3(2 * (unsigned)clusters, 1, 1);
-    cfg.blockDim = dim3(gq::kThreads, 1, 1);
-    cfg.dynamicSmemBytes = gq::SMEM_BYTES;
-    cfg.stream = st;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, gemm_nvfp4_pair128_kernel, tm_xc, tm_wc, tm_sfa, tm_sfb, tm_L, tm_Lup, a) !=
-        cudaSuccess)
-        return cuda_fail("gemm_nvfp4_pair128_kernel launch");
-    return launch_status("gemm_nvfp4_pair128_kernel launch");
+    return per_dev[dev].load();
 }
 
 // M > 128: 256 x 256 tiles on CTA pairs.
+// The fused QKV + RMSNorm + RoPE epilogue's arguments (heads == 0: plain epilogue).
+struct QkvEpilogue {
+    int heads = 0;
+    const void* norm_q = nullptr;
+    const void* norm_k = nullptr;
+    float eps = 0.0f;
+    const float* rope_cos = nullptr;
+    const float* rope_sin = nullptr;
+};
+
 svdq_status gemm_nvfp4_pair(const void* x_codes, const void* x_scales, const float* x_scale, int64_t M,
                             const void* w_codes, const void* w_scales, const float* w_scale, int64_t N, int64_t K,
                             const void* lowrank, const void* L_up_t, int rank, const void* bias, void* y,
-                            cudaStream_t st) {
+                            cudaStream_t st, const QkvEpilogue& qkv = QkvEpilogue()) {
     CUtensorMap tm_xc, tm_wc, tm_sfa, tm_sfb, tm_L, tm_Lup;
     const int64_t kg4 = K / 64;
     if (!make_map(&tm_xc, CU_TENSOR_MAP_DATA_TYPE_UINT8, x_codes, (uint64_t)K / 2, (uint64_t)M, (uint64_t)K / 2,
@@ -501,7 +563,7 @@ svdq_status gemm_nvfp4_pair(const void* x_codes, const void* x_scales, const flo
         tm_L = tm_xc;
         tm_Lup = tm_wc;
     }
-    GemmArgs a;
+    GemmArgs a = {};
     a.x_scales = reinterpret_cast<const uint8_t*>(x_scales);
     a.w_scales = reinterpret_cast<const uint8_t*>(w_scales);
     a.x_scale = x_scale;
@@ -514,26 +576,28 @@ svdq_status gemm_nvfp4_pair(const void* x_codes, const void* x_scales, const flo
     a.rank = rank;
     a.kg4 = (int)kg4;
     a.n_sf_blocks = (int)((N + 127) / 128);
+    if (qkv.heads > 0) {
+        a.norm_q = reinterpret_cast<const __nv_bfloat16*>(qkv.norm_q);
+        a.norm_k = reinterpret_cast<const __nv_bfloat16*>(qkv.norm_k);
+        a.rope_cos = qkv.rope_cos;
+        a.rope_sin = qkv.rope_sin;
+        a.eps = qkv.eps;
+        a.q_cols = qkv.heads * 128;
+        a.qk_cols = 2 * qkv.heads * 128;
+    }
     const int64_t mt = (M + gp::BM - 1) / gp::BM, nt = (N + gp::BN - 1) / gp::BN;
     if (mt * nt > (int64_t(1) << 30)) return SVDQ_ERR_UNSUPPORTED_SHAPE;
     a.m_tiles = (int)mt;
     a.n_tiles = (int)nt;
     const int clusters = (int)std::min<int64_t>(mt * nt, pair_clusters());
-    cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.gridDim = dim3(2 * (unsigned)clusters, 1, 1);
-    cfg.blockDim = dim3(gp::kThreads, 1, 1);
-    cfg.dynamicSmemBytes = gp::SMEM_BYTES;
-    cfg.stream = st;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, gemm_nvfp4_pair_kernel, tm_xc, tm_wc, tm_sfa, tm_sfb, tm_L, tm_Lup, a) !=
-        cudaSuccess)
-        return cuda_fail("gemm_nvfp4_pair_kernel launch");
+    // programmatic dependent launch: the kernel's prologue overlaps the tail of
+    // the activation quantizer, which releases its dependents early
+    const cudaError_t e =
+        qkv.heads > 0 ? launch_ex(gemm_nvfp4_pair_kernel<true>, dim3(2 * (unsigned)clusters), dim3(gp::kThreads),
+                                  gp::SMEM_BYTES, st, 2u, tm_xc, tm_wc, tm_sfa, tm_sfb, tm_L, tm_Lup, a)
+                      : launch_ex(gemm_nvfp4_pair_kernel<false>, dim3(2 * (unsigned)clusters), dim3(gp::kThreads),
+                                  gp::SMEM_BYTES, st, 2u, tm_xc, tm_wc, tm_sfa, tm_sfb, tm_L, tm_Lup, a);
+    if (e != cudaSuccess) return cuda_fail("gemm_nvfp4_pair_kernel launch");
     return launch_status("gemm_nvfp4_pair_kernel launch");
 }
 
@@ -593,6 +657,7 @@ __global__ void timeout_probe_kernel() {
 constexpr size_t kNoAllocWorkspaceBytes = size_t(8) << 20;   // 8 MiB
 std::mutex g_noalloc_mutex;
 void* g_noalloc_addr[kMaxDevices];
+void* g_noalloc_ctx[kMaxDevices];   // context the cached address belongs to
 
 }  // namespace
 
@@ -608,8 +673,23 @@ svdq_status noalloc_workspace_address(void** out) {
         cudaGetLastError();
         return SVDQ_ERR_UNSUPPORTED_DEVICE;
     }
+    // the current context: a device reset replaces it, and with it the array's address
+    using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+    static CtxGetCurrentFn ctx_fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            ctx_fn = reinterpret_cast<CtxGetCurrentFn>(p);
+        else
+            cudaGetLastError();
+    });
+    CUcontext ctx = nullptr;
+    if (ctx_fn) ctx_fn(&ctx);
     std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-    if (!g_noalloc_addr[dev]) {
+    if (!g_noalloc_addr[dev] || g_noalloc_ctx[dev] != (void*)ctx) {
         void* p = nullptr;
         const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_workspace);
         if (e != cudaSuccess || p == nullptr) {
@@ -618,6 +698,7 @@ svdq_status noalloc_workspace_address(void** out) {
             return SVDQ_ERR_CUDA;
         }
         g_noalloc_addr[dev] = p;
+        g_noalloc_ctx[dev] = (void*)ctx;
     }
     *out = g_noalloc_addr[dev];
     return SVDQ_OK;
@@ -792,16 +873,194 @@ svdq_status svdq_gemm_w4a4(svdq_precision p, int group_size, const void* x_codes
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (p == SVDQ_NVFP4) {
         const int mode = g_gemm_tiles_mode.load();
-        if (mode == 3 && pair128_applies(M, K))
-            return gemm_nvfp4_pair128(x_codes, x_scales, x_tensor_scale, M, w_codes, w_scales, w_tensor_scale, N, K,
-                                      lowrank_act, L_up_t, rank, bias, y, st);
-        if (mode == 2 || mode == 3 || (mode == 0 && M > 128))
+        if (mode == 2 || (mode == 0 && M > 128))
             return gemm_nvfp4_pair(x_codes, x_scales, x_tensor_scale, M, w_codes, w_scales, w_tensor_scale, N, K,
                                    lowrank_act, L_up_t, rank, bias, y, st);
         return gemm_nvfp4(x_codes, x_scales, x_tensor_scale, M, w_codes, w_scales, w_tensor_scale, N, K, lowrank_act,
                           L_up_t, rank, bias, y, st);
     }
     return int4_gemm(x_codes, x_scales, M, w_codes, w_scales, N, K, lowrank_act, L_up_t, rank, bias, y, st);
+}
+
+// Checks of the fused QKV + RMSNorm + RoPE arguments shared by both entry points.
+static svdq_status check_qkv_args(int64_t M, int64_t N, int heads, int head_dim, const void* norm_q,
+                                  const void* norm_k, float eps, const float* rope_cos, const float* rope_sin) {
+    if (head_dim != 128 || heads < 1) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+    if (N != 3 * (int64_t)heads * head_dim) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+    if (!(eps > 0.0f) || !(eps < 1.0f)) return SVDQ_ERR_INVALID_ARG;
+    SVDQ_TRY(check_ptr(norm_q));
+    SVDQ_TRY(check_ptr(norm_k));
+    SVDQ_TRY(check_ptr(rope_cos));
+    SVDQ_TRY(check_ptr(rope_sin));
+    if (M < 1) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+    return SVDQ_OK;
+}
+
+svdq_status svdq_gemm_w4a4_qkv_norm_rope(svdq_precision p, int group_size, const void* x_codes, const void* x_scales,
+                                         const float* x_tensor_scale, int64_t M, const void* w_codes,
+                                         const void* w_scales, const float* w_tensor_scale, int64_t N, int64_t K,
+                                         const void* lowrank_act, const void* L_up_t, int rank, const void* bias,
+                                         int heads, int head_dim, const void* norm_q, const void* norm_k, float eps,
+                                         const float* rope_cos, const float* rope_sin, void* y,
+                                         svdq_stream_t stream) {
+    SVDQ_TRY(check_precision(p, group_size));
+    if (p != SVDQ_NVFP4) return SVDQ_ERR_INVALID_ARG;   // the fused epilogue belongs to the nvfp4 GEMM
+    SVDQ_TRY(check_rank(rank));
+    SVDQ_TRY(check_dims(M, K));
+    SVDQ_TRY(check_dims(N, K));
+    SVDQ_TRY(check_qkv_args(M, N, heads, head_dim, norm_q, norm_k, eps, rope_cos, rope_sin));
+    SVDQ_TRY(check_ptr(x_codes));
+    SVDQ_TRY(check_ptr(x_scales));
+    SVDQ_TRY(check_ptr(w_codes));
+    SVDQ_TRY(check_ptr(w_scales));
+    SVDQ_TRY(check_ptr(y));
+    SVDQ_TRY(check_opt_ptr(bias));
+    SVDQ_TRY(check_ptr(x_tensor_scale));
+    SVDQ_TRY(check_ptr(w_tensor_scale));
+    if (rank > 0) {
+        SVDQ_TRY(check_ptr(lowrank_act));
+        SVDQ_TRY(check_ptr(L_up_t));
+    }
+    SVDQ_TRY(check_device());
+    QkvEpilogue e;
+    e.heads = heads;
+    e.norm_q = norm_q;
+    e.norm_k = norm_k;
+    e.eps = eps;
+    e.rope_cos = rope_cos;
+    e.rope_sin = rope_sin;
+    return gemm_nvfp4_pair(x_codes, x_scales, x_tensor_scale, M, w_codes, w_scales, w_tensor_scale, N, K, lowrank_act,
+                           L_up_t, rank, bias, y, reinterpret_cast<cudaStream_t>(stream), e);
+}
+
+svdq_status svdq_qkv_norm_rope(const void* y_in, void* y_out, int64_t M, int heads, int head_dim, const void* norm_q,
+                               const void* norm_k, float eps, const float* rope_cos, const float* rope_sin,
+                               svdq_stream_t stream) {
+    SVDQ_TRY(check_ptr(y_in));
+    SVDQ_TRY(check_ptr(y_out));
+    if (M >= (int64_t(1) << 31)) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+    SVDQ_TRY(check_qkv_args(M, 3 * (int64_t)heads * head_dim, heads, head_dim, norm_q, norm_k, eps, rope_cos,
+                            rope_sin));
+    SVDQ_TRY(check_device());
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int64_t warps = M * 2 * heads;
+    const int64_t blocks = (warps + 7) / 8;
+    if (blocks > 0x7FFFFFFF) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+    qkv_norm_rope_kernel<<<(unsigned)blocks, 256, 0, st>>>(
+        reinterpret_cast<const __nv_bfloat16*>(y_in), reinterpret_cast<__nv_bfloat16*>(y_out), M, heads,
+        reinterpret_cast<const __nv_bfloat16*>(norm_q), reinterpret_cast<const __nv_bfloat16*>(norm_k), eps, rope_cos,
+        rope_sin);
+    SVDQ_TRY(launch_status("qkv_norm_rope_kernel launch"));
+    if (y_out != y_in) {
+        const int64_t n8 = M * heads * 128 / 8;
+        const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((n8 + 255) / 256, 8LL * num_sms()));
+        copy_v_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(y_in),
+                                             reinterpret_cast<__nv_bfloat16*>(y_out), M, heads);
+        SVDQ_TRY(launch_status("copy_v_kernel launch"));
+    }
+    return SVDQ_OK;
+}
+
+svdq_status svdq_gemm_w4a16(const void* x, int64_t M, const void* w_codes, const void* w_scales, int64_t N,
+                            int64_t K, const void* bias, void* y, svdq_stream_t stream) {
+    SVDQ_TRY(check_dims(M, K));
+    SVDQ_TRY(check_dims(N, K));
+    if (N % 16 != 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+    SVDQ_TRY(check_ptr(x));
+    SVDQ_TRY(check_ptr(w_codes));
+    SVDQ_TRY(check_ptr(w_scales));
+    SVDQ_TRY(check_ptr(y));
+    SVDQ_TRY(check_opt_ptr(bias));
+    const int64_t mt = (M + aw::BM - 1) / aw::BM, nt = (N + aw::BN - 1) / aw::BN;
+    if (mt > 0x7FFFFFFF || nt > 65535) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+    SVDQ_TRY(check_device());
+    CUtensorMap tm_x, tm_wc, tm_ws;
+    const int64_t n_pad = round_up(N, 128);
+    if (!make_map(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, 64, 128) ||
+        !make_map(&tm_wc, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_codes, (uint64_t)K / 2, (uint64_t)N, (uint64_t)K / 2, 32,
+                  256, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !make_map(&tm_ws, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w_scales, (uint64_t)n_pad, (uint64_t)(K / 64),
+                  (uint64_t)n_pad * 2, 256, 1, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return SVDQ_ERR_CUDA;
+    W4A16Args a;
+    a.bias = reinterpret_cast<const __nv_bfloat16*>(bias);
+    a.y = reinterpret_cast<__nv_bfloat16*>(y);
+    a.M = (int)M;
+    a.N = (int)N;
+    a.K = (int)K;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    gemm_w4a16_kernel<<<dim3((unsigned)mt, (unsigned)nt, 1), aw::kThreads, aw::SMEM_BYTES, st>>>(tm_x, tm_wc, tm_ws, a);
+    return launch_status("gemm_w4a16_kernel launch");
+}
+
+svdq_status svdq_svd_split_workspace_bytes(int64_t N, int64_t K, int rank, int oversample, size_t* bytes) {
+    if (!bytes) return SVDQ_ERR_INVALID_ARG;
+    if (rank < 1 || oversample < 0 || rank + oversample > sv::kMaxL) return SVDQ_ERR_INVALID_ARG;
+    SVDQ_TRY(check_dims(N, K));
+    if (rank > std::min(N, K)) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+    *bytes = svd_split_workspace(N, K, rank + oversample);
+    return SVDQ_OK;
+}
+
+svdq_status svdq_svd_split(const void* W, const float* lambda, int64_t N, int64_t K, int rank, const float* omega,
+                           int oversample, int power_iters, void* R, void* L_down, void* L_up,
+                           float* singular_values, void* workspace, size_t workspace_bytes, svdq_stream_t stream) {
+    if (rank < 1 || oversample < 0 || rank + oversample > sv::kMaxL || power_iters < 0 || power_iters > 16)
+        return SVDQ_ERR_INVALID_ARG;
+    SVDQ_TRY(check_dims(N, K));
+    if (rank > std::min(N, K) || N >= (int64_t(1) << 31) / sv::kMaxL) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+    SVDQ_TRY(check_ptr(W));
+    SVDQ_TRY(check_ptr(lambda));
+    SVDQ_TRY(check_ptr(omega));
+    SVDQ_TRY(check_ptr(R));
+    SVDQ_TRY(check_ptr(L_down));
+    SVDQ_TRY(check_ptr(L_up));
+    SVDQ_TRY(check_opt_ptr(singular_values));
+    SVDQ_TRY(check_ptr(workspace));
+    const int l = rank + oversample;
+    if (workspace_bytes < svd_split_workspace(N, K, l)) return SVDQ_ERR_INVALID_ARG;
+    SVDQ_TRY(check_device());
+    static std::once_flag jac_once;
+    static cudaError_t jac_err = cudaSuccess;
+    std::call_once(jac_once, [] {
+        jac_err = cudaFuncSetAttribute(svd_jacobi_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)kJacobiSmem);
+    });
+    if (jac_err != cudaSuccess) return cuda_fail("setting the Jacobi kernel's shared memory");
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+    float* Y = reinterpret_cast<float*>(ws);
+    ws += round_up(N * l * (int64_t)sizeof(float), 256);
+    float* Z = reinterpret_cast<float*>(ws);
+    ws += round_up(K * l * (int64_t)sizeof(float), 256);
+    double* part = reinterpret_cast<double*>(ws);
+    double* Rinv = part + (size_t)sv::kGramBlocks * sv::kMaxL * sv::kMaxL;
+    double* U = Rinv + (size_t)sv::kMaxL * sv::kMaxL;
+    double* evals = U + (size_t)sv::kMaxL * sv::kMaxL;
+    const __nv_bfloat16* Wb = reinterpret_cast<const __nv_bfloat16*>(W);
+    const unsigned gN = (unsigned)((N + sv::kTileR - 1) / sv::kTileR), gK = (unsigned)((K + sv::kTileR - 1) / sv::kTileR);
+    // range finder with subspace iteration
+    svd_w_times_kernel<<<gN, 256, 0, st>>>(Wb, lambda, N, K, omega, l, Y);
+    SVDQ_TRY(svd_orth(Y, N, l, part, Rinv, st));
+    for (int q = 0; q < power_iters; ++q) {
+        svd_wt_times_kernel<<<gK, 256, 0, st>>>(Wb, lambda, N, K, Y, l, Z);
+        SVDQ_TRY(svd_orth(Z, K, l, part, Rinv, st));
+        svd_w_times_kernel<<<gN, 256, 0, st>>>(Wb, lambda, N, K, Z, l, Y);
+        SVDQ_TRY(svd_orth(Y, N, l, part, Rinv, st));
+    }
+    // B^T = W_hat^T Q and the SVD of B from the eigen-decomposition of B B^T
+    svd_wt_times_kernel<<<gK, 256, 0, st>>>(Wb, lambda, N, K, Y, l, Z);
+    svd_gram_partial_kernel<<<sv::kGramBlocks, 256, 0, st>>>(Z, K, l, part);
+    svd_jacobi_kernel<<<1, 32, kJacobiSmem, st>>>(part, sv::kGramBlocks, l, evals, U);
+    SVDQ_TRY(launch_status("SVD split: small eigen-problem"));
+    const int64_t rows = std::max(N, K);
+    svd_factors_kernel<<<(unsigned)((rows + 255) / 256), 256, 0, st>>>(
+        Y, N, Z, K, l, rank, evals, U, reinterpret_cast<__nv_bfloat16*>(L_up),
+        reinterpret_cast<__nv_bfloat16*>(L_down), singular_values);
+    svd_residual_kernel<<<dim3((unsigned)((K + 63) / 64), (unsigned)((N + 31) / 32)), 256, 0, st>>>(
+        Wb, lambda, N, K, reinterpret_cast<const __nv_bfloat16*>(L_up), reinterpret_cast<const __nv_bfloat16*>(L_down),
+        rank, reinterpret_cast<__nv_bfloat16*>(R));
+    return launch_status("SVD split: factors and residual");
 }
 
 svdq_status svdq_device_status(int clear, int* site) {
@@ -835,12 +1094,21 @@ svdq_status svdq_debug_timeout_probe(svdq_stream_t stream) {
 }
 
 svdq_status svdq_debug_force_gemm_tiles(int mode) {
-    if (mode < 0 || mode > 3) {
-        snprintf(g_last_error, sizeof(g_last_error), "svdq_debug_force_gemm_tiles: mode %d is not 0, 1, 2 or 3",
+    if (mode < 0 || mode > 2) {
+        snprintf(g_last_error, sizeof(g_last_error), "svdq_debug_force_gemm_tiles: mode %d is not 0, 1 or 2",
                  mode);
         return SVDQ_ERR_INVALID_ARG;
     }
     g_gemm_tiles_mode.store(mode);
+    return SVDQ_OK;
+}
+
+svdq_status svdq_debug_force_quant_plan(int mode) {
+    if (mode < 0 || mode > 2) {
+        snprintf(g_last_error, sizeof(g_last_error), "svdq_debug_force_quant_plan: mode %d is not 0, 1 or 2", mode);
+        return SVDQ_ERR_INVALID_ARG;
+    }
+    g_quant_plan_mode.store(mode);
     return SVDQ_OK;
 }
 

@@ -107,3 +107,43 @@ def bits(t: torch.Tensor):
 
     assert t.dtype == torch.bfloat16
     return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+QKV_HEAD_DIM = 128          # FLUX-class DiT attention heads: 24 x 128 = 3072 = hidden size
+QKV_EPS = 1e-6
+
+
+def qkv_inputs(M: int, heads: int, seed: int = 7) -> dict:
+    """Extra inputs of the fused QKV + RMSNorm + RoPE path, drawn after the
+    layer's own: the Q and K RMSNorm weights ~ U[0.5, 2] (bf16) and one rotary
+    angle per (token, pair) ~ U[-pi, pi), given as fp32 cos and sin tables
+    [M, 64] (the per-token rotary embedding the attention block receives)."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    D = QKV_HEAD_DIM
+    wq = (torch.rand(D, generator=g, dtype=torch.float32) * 1.5 + 0.5).to(torch.bfloat16)
+    wk = (torch.rand(D, generator=g, dtype=torch.float32) * 1.5 + 0.5).to(torch.bfloat16)
+    theta = (torch.rand(M, D // 2, generator=g, dtype=torch.float64) * 2.0 - 1.0) * math.pi
+    return {"heads": heads, "head_dim": D, "eps": QKV_EPS, "norm_q": wq, "norm_k": wk,
+            "cos": torch.cos(theta).to(torch.float32), "sin": torch.sin(theta).to(torch.float32)}
+
+
+def svd_split_inputs(N: int, K: int, rank: int, oversample: int = 8, seed: int = 5) -> dict:
+    """Inputs of the offline SVD split: a weight W [N, K] (bf16) with a planted
+    rank-`rank` component -- orthonormal factors U [N, r] and V [K, r] from the
+    QR decomposition of Gaussian draws, singular values 30 * 0.93^i -- plus
+    Gaussian noise of standard deviation 0.1 / sqrt(K) (a few dominant
+    directions over a noise floor, like trained projection weights); the
+    smoothing divisors lambda ~ U[0.5, 4]; the Gaussian test matrix Omega
+    [K, rank + oversample] ~ N(0, 1) (fp32) that the randomized range finder
+    consumes."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    U, _ = torch.linalg.qr(torch.randn(N, rank, generator=g, dtype=torch.float64))
+    V, _ = torch.linalg.qr(torch.randn(K, rank, generator=g, dtype=torch.float64))
+    s = 30.0 * 0.93 ** torch.arange(rank, dtype=torch.float64)
+    noise = torch.randn(N, K, generator=g, dtype=torch.float64) * (0.1 / math.sqrt(K))
+    W = (U * s) @ V.T + noise
+    lam = torch.rand(K, generator=g, dtype=torch.float32) * 3.5 + 0.5
+    omega = torch.randn(K, rank + oversample, generator=g, dtype=torch.float32)
+    return {"W": W.to(torch.bfloat16), "lam": lam, "omega": omega, "rank": rank, "oversample": oversample}

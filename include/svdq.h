@@ -124,8 +124,13 @@ svdq_status svdq_pack_weight(svdq_precision precision, int group_size,
                              svdq_stream_t stream);
 
 /* Bytes of the workspace svdq_quantize_act needs for this shape (0 when it
- * needs none).  The workspace holds fp32 partial sums of the rank-r product
- * when K is split across several CTAs, plus one counter per 128-row block.
+ * needs none).  When K is split across several CTAs, each computes a partial
+ * rank-r product.  The CTAs of a 128-row block normally form one thread-block
+ * cluster and add their partials through distributed shared memory; when such
+ * clusters cannot all be resident at once (fewer SMs available than the split
+ * needs), they add them through this workspace instead: fp32 partial sums
+ * plus one counter per 128-row block.  The size returned covers that case;
+ * a call that runs in cluster mode leaves the workspace untouched.
  * Pure host function; errors as svdq_buffer_sizes. */
 svdq_status svdq_quantize_act_workspace_bytes(svdq_precision precision, int64_t M, int64_t K, int rank,
                                               size_t* bytes);
@@ -164,11 +169,14 @@ svdq_status svdq_quantize_act(svdq_precision precision, int group_size,
  * Arguments, outputs and errors are those of svdq_quantize_act, without the
  * workspace: the K-split workspace is a library-owned 8 MiB device array
  * (file-scope, so every GPU that loads the library holds it until the process
- * exits).  Shapes whose workspace, as reported by
- * svdq_quantize_act_workspace_bytes, exceeds 8 MiB are rejected with
- * SVDQ_ERR_UNSUPPORTED_SHAPE, and svdq_last_error() says so.
- * The first call on each device looks up the array's device address with
- * that device current; make that first call before any stream capture.
+ * exits).  It is used whenever the split's partials go through global memory
+ * (see svdq_quantize_act_workspace_bytes); in cluster mode it is not touched.
+ * Shapes whose workspace, as reported by svdq_quantize_act_workspace_bytes,
+ * exceeds 8 MiB are rejected with SVDQ_ERR_UNSUPPORTED_SHAPE, and
+ * svdq_last_error() says so.
+ * The first call on each device (and the first after that device's context
+ * was replaced, e.g. by cudaDeviceReset) looks up the array's device address
+ * with that device current; make that first call before any stream capture.
  * Each call zero-fills the array's counters on `stream` before its launch.
  * All calls share the one array and it keeps the last call's contents, so
  * calls that overlap on the GPU (other streams or threads) race on it.
@@ -193,6 +201,88 @@ svdq_status svdq_gemm_w4a4(svdq_precision precision, int group_size,
                            const void* lowrank_act, const void* L_up_t, int rank,
                            const void* bias, void* y, svdq_stream_t stream);
 
+/* The W4A4 GEMM of a fused to_qkv projection with the attention-input
+ * RMSNorm and rotary embedding applied in its epilogue (the fused operator of
+ * the original Nunchaku engine: the tutorial page's "structural rewrite"
+ * passage, one to_qkv projection then norm_q / norm_k per head and
+ * apply_rotary_emb; the Diffusers docs page "Nunchaku Lite", section "Fused
+ * kernels", "QKV+norm+RoPE" fusion).  nvfp4 only.
+ * Arguments up to bias are those of svdq_gemm_w4a4, with N = 3 * heads *
+ * head_dim: output columns [0, H D) are Q, [H D, 2 H D) K, [2 H D, 3 H D) V,
+ * each head-major.  For every row and every head of Q and K, on the fp32
+ * result v of the linear layer (before any bf16 rounding):
+ *     v' = v / sqrt(mean(v^2) + eps) * w      (w = norm_q for Q, norm_k for K)
+ *     out[2i] = v'[2i] cos[m,i] - v'[2i+1] sin[m,i]
+ *     out[2i+1] = v'[2i+1] cos[m,i] + v'[2i] sin[m,i]
+ * V is the plain linear output.  y receives bf16(out).
+ *   heads      H >= 1;  head_dim must be 128
+ *   norm_q, norm_k   device bf16 [head_dim]
+ *   eps        0 < eps < 1
+ *   rope_cos, rope_sin   device fp32 [M, head_dim / 2]: each token's rotary table
+ * Errors: as svdq_gemm_w4a4; INVALID_ARG for int4 or a bad eps;
+ * UNSUPPORTED_SHAPE when head_dim != 128 or N != 3 * heads * head_dim. */
+svdq_status svdq_gemm_w4a4_qkv_norm_rope(svdq_precision precision, int group_size,
+                                         const void* x_codes, const void* x_scales, const float* x_tensor_scale,
+                                         int64_t M, const void* w_codes, const void* w_scales,
+                                         const float* w_tensor_scale, int64_t N, int64_t K,
+                                         const void* lowrank_act, const void* L_up_t, int rank, const void* bias,
+                                         int heads, int head_dim, const void* norm_q, const void* norm_k, float eps,
+                                         const float* rope_cos, const float* rope_sin, void* y,
+                                         svdq_stream_t stream);
+
+/* The same RMSNorm + rotary embedding as a separate pass over a bf16 to_qkv
+ * output already in memory (the unfused path: the projection, then this):
+ *   y_in, y_out   device bf16 [M, 3 * heads * head_dim]; y_out may equal y_in
+ *                 (in place); otherwise the V columns are copied across.
+ * Other arguments and errors as svdq_gemm_w4a4_qkv_norm_rope. */
+svdq_status svdq_qkv_norm_rope(const void* y_in, void* y_out, int64_t M, int heads, int head_dim,
+                               const void* norm_q, const void* norm_k, float eps,
+                               const float* rope_cos, const float* rope_sin, svdq_stream_t stream);
+
+/* The weight-only int4 GEMM of the `awq_w4a16` scheme (the "INT4 weight-only
+ * AWQ-style kernel", int4 with group 64, of the Diffusers docs page "Nunchaku
+ * Lite", section "Supported quantization types"; its targets are listed in
+ * section "NunchakuLiteQuantizationConfig"):
+ *     y[m, n] = bf16( sum_k x[m, k] q[n, k] s[n, k / 64] + b[n] )
+ * The activation-aware scaling of AWQ is folded into W (and, inversely, into
+ * the layer feeding x) offline; x is used as it comes.
+ *   x          device bf16 [M, K] (values of magnitude below 65504)
+ *   w_codes, w_scales   the int4 weight as svdq_pack_weight(SVDQ_INT4, 64,
+ *              W, N, K, lambda = all ones, rank 0, ...) packs it: two's
+ *              complement codes [N, K/2] and bf16 scales [K/64, N_pad]
+ *   bias       device bf16 [N] or NULL;  y  device bf16 [M, N]
+ * Products q s are exact in fp16; the tensor cores multiply fp16 x fp16 with
+ * fp32 accumulation.  Sizes and errors as svdq_gemm_w4a4. */
+svdq_status svdq_gemm_w4a16(const void* x, int64_t M, const void* w_codes, const void* w_scales,
+                            int64_t N, int64_t K, const void* bias, void* y, svdq_stream_t stream);
+
+/* Offline split of a layer's weight into the low-rank branch and the residual
+ * that svdq_pack_weight quantizes (the SVDQuant decomposition the Diffusers
+ * docs page "Nunchaku Lite" builds on; the tutorial's offline quantization
+ * step, quantize_hf.py --rank 32):
+ *     W_hat = W diag(lambda) = L_up^T L_down^T + R
+ * with L_up^T L_down^T the best rank-r approximation of W_hat, computed by a
+ * randomized range finder with `power_iters` steps of subspace iteration
+ * (Halko, Martinsson and Tropp 2011) and R the residual with the bf16
+ * factors.  Then x W^T = (x / lambda) R^T + ((x / lambda) L_down) L_up: pass
+ * R, lambda, L_down and L_up to svdq_pack_weight.
+ *   W        device bf16 [N, K] (out x in)
+ *   lambda   device fp32 [K] smoothing divisors (> 0)
+ *   omega    device fp32 [K, rank + oversample]: a Gaussian test matrix, drawn
+ *            by the caller (for example N(0, 1) entries)
+ *   rank     1 <= rank <= min(N, K), rank + oversample <= 64
+ *   power_iters  0..16 (2 is ample when the spectrum decays past rank)
+ * Outputs (device, caller-allocated): R bf16 [N, K]; L_down bf16 [K, rank];
+ *   L_up bf16 [rank, N]; singular_values fp32 [rank + oversample] (the
+ *   approximations of the largest singular values of W_hat, decreasing) or NULL.
+ * workspace: device, at least svdq_svd_split_workspace_bytes() bytes.
+ * An offline step: simple kernels, not tuned for speed. */
+svdq_status svdq_svd_split_workspace_bytes(int64_t N, int64_t K, int rank, int oversample, size_t* bytes);
+svdq_status svdq_svd_split(const void* W, const float* lambda, int64_t N, int64_t K, int rank,
+                           const float* omega, int oversample, int power_iters,
+                           void* R, void* L_down, void* L_up, float* singular_values,
+                           void* workspace, size_t workspace_bytes, svdq_stream_t stream);
+
 /* Synchronises the current device, then reads the device status word.
  * Returns SVDQ_OK, SVDQ_ERR_TIMEOUT (a kernel abandoned a wait; *site, if not
  * NULL, receives the id of the first wait that did) or SVDQ_ERR_CUDA.
@@ -207,14 +297,17 @@ svdq_status svdq_device_status(int clear, int* site);
  *  svdq_debug_override_capability: pretend the device has compute capability
  *    major.minor (major = -1 removes the override), to test the device check.
  *  svdq_debug_force_gemm_tiles: choose the nvfp4 GEMM kernel: 0 = automatic
- *    (M <= 128: 128 x 256 tiles on single CTAs; M > 128: 256 x 256 tiles on
- *    CTA pairs), 1 = always single CTAs, 2 = always 256 x 256 CTA-pair tiles,
- *    3 = 256 x 128 CTA-pair tiles with the weight scales resident in tensor
- *    memory where M > 128, K % 512 == 0 and K <= 3072 (a slower alternative,
- *    never chosen automatically), else as 2.  All kernels compute the same y;
- *    this exists so that tests can run each on the same inputs.  Any other
- *    value is SVDQ_ERR_INVALID_ARG. */
+ *    (M <= 128: 128 x 256 tiles on single CTAs; M > 128: CTA-pair tiles),
+ *    1 = always single CTAs, 2 = always CTA pairs.  Both kernels compute the
+ *    same y; this exists so that tests can run each on the same inputs.  Any
+ *    other value is SVDQ_ERR_INVALID_ARG. */
 svdq_status svdq_debug_set_wait_limit_ns(uint64_t ns);
+/* svdq_debug_force_quant_plan: how svdq_quantize_act adds the rank-r partials
+ *    of a K split: 0 = automatic, 1 = always through the workspace (global
+ *    memory, see svdq_quantize_act), 2 = always in one thread-block cluster
+ *    through distributed shared memory.  Results are the same; tests use it to
+ *    run both.  Any other value is SVDQ_ERR_INVALID_ARG. */
+svdq_status svdq_debug_force_quant_plan(int mode);
 svdq_status svdq_debug_timeout_probe(svdq_stream_t stream);
 void svdq_debug_override_capability(int major, int minor);
 svdq_status svdq_debug_force_gemm_tiles(int mode);

@@ -55,6 +55,13 @@ def _load():
         lib = ctypes.CDLL(build())
         P = ctypes.c_void_p
         L = ctypes.c_long
+        D = ctypes.c_double
+        lib.oracle_rms_norm_head.argtypes = [P, L, P, D]
+        lib.oracle_rms_norm_head.restype = None
+        lib.oracle_rope_head.argtypes = [P, L, P, P]
+        lib.oracle_rope_head.restype = None
+        lib.oracle_qkv_norm_rope.argtypes = [P, L, L, L, P, P, D, P, P, P, P]
+        lib.oracle_qkv_norm_rope.restype = None
         lib.oracle_bf16_to_double.argtypes = [ctypes.c_uint16]
         lib.oracle_bf16_to_double.restype = ctypes.c_double
         lib.oracle_bf16_from_double.argtypes = [ctypes.c_double]
@@ -237,6 +244,61 @@ def int4_linear(xc, xs, wc, ws, L, L_up_bits, bias_bits, rows=None):
     _load().oracle_int4_linear(_ptr(xc), _ptr(xs), _ptr(rows_arr), nrows, K, _ptr(wc), _ptr(ws), N,
                                _ptr(Lc), _ptr(Lu), r, _ptr(b), _ptr(y), _ptr(ybf))
     return y, ybf
+
+
+# --------------------------------------------- fused QKV + RMSNorm + RoPE
+def rms_norm_head(v: np.ndarray, w_bits: np.ndarray, eps: float) -> np.ndarray:
+    """RMSNorm of one head vector (fp64) with bf16 weights."""
+    out = np.ascontiguousarray(v, np.float64).copy()
+    _load().oracle_rms_norm_head(_ptr(out), out.shape[0], _ptr(_u16(w_bits)), float(eps))
+    return out
+
+
+def rope_head(v: np.ndarray, cos: np.ndarray, sin: np.ndarray) -> np.ndarray:
+    """Rotary embedding of one head vector (fp64): pair i rotates by (cos[i], sin[i])."""
+    out = np.ascontiguousarray(v, np.float64).copy()
+    _load().oracle_rope_head(_ptr(out), out.shape[0], _ptr(np.ascontiguousarray(cos, np.float64)),
+                             _ptr(np.ascontiguousarray(sin, np.float64)))
+    return out
+
+
+def qkv_norm_rope(y: np.ndarray, heads: int, head_dim: int, wq_bits, wk_bits, eps: float,
+                  cos: np.ndarray, sin: np.ndarray):
+    """Per-head RMSNorm and RoPE of the Q and K columns of a to_qkv output.
+
+    y [rows, 3 * heads * head_dim] fp64 (the linear layer's exact output);
+    cos, sin [rows, head_dim / 2] the tokens' rotary tables.  Returns the fp64
+    result and its bf16 bits (V columns pass through)."""
+    y = np.ascontiguousarray(y, np.float64)
+    rows, N = y.shape
+    assert N == 3 * heads * head_dim
+    out = np.zeros_like(y)
+    outb = np.zeros(y.shape, np.uint16)
+    _load().oracle_qkv_norm_rope(_ptr(y), rows, heads, head_dim, _ptr(_u16(wq_bits)), _ptr(_u16(wk_bits)),
+                                 float(eps), _ptr(np.ascontiguousarray(cos, np.float64)),
+                                 _ptr(np.ascontiguousarray(sin, np.float64)), _ptr(out), _ptr(outb))
+    return out, outb
+
+
+# ------------------------------------------------ offline SVDQuant split
+def svd_split(W_bits: np.ndarray, lam: np.ndarray, rank: int):
+    """The offline split of the SVDQuant paper that the Diffusers docs page
+    "Nunchaku Lite" builds on (introduction; the tutorial's quantize_hf.py
+    --rank 32 step): the smoothed weight W_hat = W diag(lambda) [N, K] is
+    split into its best rank-r approximation (the truncated SVD) and the
+    residual R = W_hat - L_up^T L_down^T, so that
+        x W^T = (x / lambda) W_hat^T = (x / lambda) R^T + ((x / lambda) L_down) L_up.
+    Returns (R [N, K], L_down [K, r], L_up [r, N], singular values), fp64;
+    the factors are unique up to the signs of singular-vector pairs, their
+    product and R are unique when s_r > s_{r+1}.  A library SVD (LAPACK
+    through numpy) is the step that computes the decomposition."""
+    W = bf16_to_float(_u16(W_bits)).astype(np.float64)
+    W_hat = W * np.asarray(lam, np.float64)[None, :]
+    U, s, Vt = np.linalg.svd(W_hat, full_matrices=False)
+    L_up = (U[:, :rank] * s[:rank]).T
+    L_down = Vt[:rank].T
+    R = W_hat - L_up.T @ L_down.T
+    return R, L_down, L_up, s
 
 
 # ------------------------------------------------------- whole layer

@@ -348,6 +348,68 @@ void oracle_int4_linear(const uint8_t* xc, const uint16_t* xs, const long* rows,
     }
 }
 
+/* ------------------------------------------- fused QKV + RMSNorm + RoPE */
+/*
+ * The fused attention-input path of the original Nunchaku engine (the
+ * tutorial page's "structural rewrite" section, the fused_qkv_norm_rottary
+ * operator on one to_qkv projection; the Diffusers docs page "Nunchaku Lite",
+ * section "Fused kernels": "QKV+norm+RoPE" fusion).  Readings (the pages name
+ * the fusion but fix none of its details; these follow the split path the
+ * tutorial prints -- norm_q / norm_k per head, then apply_rotary_emb -- with
+ * the FLUX-class DiT's choices):
+ *   - y [rows, N] is the to_qkv output with N = 3 * H * D: columns [0, HD) are
+ *     Q, [HD, 2HD) are K, [2HD, 3HD) are V; head h of Q (or K) is its columns
+ *     [hD, (h+1)D);
+ *   - RMSNorm per head of Q and of K: v / sqrt(mean_d(v^2) + eps) * w[d], with
+ *     its own weight w (D values) for Q and for K;
+ *   - RoPE on Q and K: the pairs (2i, 2i+1) of a head rotate by the token's
+ *     angle theta[i] (given as cos and sin, D/2 per token):
+ *         out[2i]   = v[2i] cos - v[2i+1] sin
+ *         out[2i+1] = v[2i+1] cos + v[2i] sin;
+ *   - V is passed through; everything in fp64, rounded once to bf16.
+ */
+
+/* RMSNorm of one head vector v[D] with weight w (bf16 bits), in place. */
+void oracle_rms_norm_head(double* v, long D, const uint16_t* w, double eps)
+{
+    double ss = 0.0;
+    for (long d = 0; d < D; ++d) ss += v[d] * v[d];
+    double inv = 1.0 / sqrt(ss / (double)D + eps);
+    for (long d = 0; d < D; ++d) v[d] = v[d] * inv * oracle_bf16_to_double(w[d]);
+}
+
+/* Rotary embedding of one head vector v[D] in place: pair i by (cos[i], sin[i]). */
+void oracle_rope_head(double* v, long D, const double* cs, const double* sn)
+{
+    for (long i = 0; i < D / 2; ++i) {
+        double a = v[2 * i], b = v[2 * i + 1];
+        v[2 * i] = a * cs[i] - b * sn[i];
+        v[2 * i + 1] = b * cs[i] + a * sn[i];
+    }
+}
+
+/* The whole epilogue on fp64 rows of y:
+ *   y, out [rows, N] (N = 3 H D); cs, sn [rows, D/2] per-token cos / sin;
+ *   wq, wk [D] bf16 norm weights; out_bf16 [rows, N] the bf16 rounding of out. */
+void oracle_qkv_norm_rope(const double* y, long rows, long H, long D, const uint16_t* wq, const uint16_t* wk,
+                          double eps, const double* cs, const double* sn, double* out, uint16_t* out_bf16)
+{
+    const long N = 3 * H * D;
+#pragma omp parallel for schedule(static)
+    for (long m = 0; m < rows; ++m) {
+        const double* yr = y + m * N;
+        double* o = out + m * N;
+        for (long n = 0; n < N; ++n) o[n] = yr[n];
+        for (long part = 0; part < 2; ++part)          /* Q, then K */
+            for (long h = 0; h < H; ++h) {
+                double* v = o + part * H * D + h * D;
+                oracle_rms_norm_head(v, D, part == 0 ? wq : wk, eps);
+                oracle_rope_head(v, D, cs + m * (D / 2), sn + m * (D / 2));
+            }
+        for (long n = 0; n < N; ++n) out_bf16[m * N + n] = oracle_bf16_from_double(o[n]);
+    }
+}
+
 int oracle_num_threads(void)
 {
 #ifdef _OPENMP

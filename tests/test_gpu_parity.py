@@ -45,7 +45,7 @@ def test_small_cases_full(case):
     check_case(case)
 
 
-@pytest.mark.parametrize("mode", [1, 2, 3], ids=["single_cta_tiles", "cta_pair_tiles", "cta_pair_256x128_tiles"])
+@pytest.mark.parametrize("mode", [1, 2], ids=["single_cta_tiles", "cta_pair_tiles"])
 @pytest.mark.parametrize("case", SMALL, ids=lambda c: c.name)
 def test_small_cases_each_gemm_kernel(case, mode):
     """Both nvfp4 GEMM kernels (128 x 256 tiles on one CTA, 256 x 256 tiles on
@@ -59,25 +59,27 @@ def test_small_cases_each_gemm_kernel(case, mode):
         _lib.svdq_debug_force_gemm_tiles(0)
 
 
-# shapes the 256 x 128 pair kernel takes (M > 128, K % 512 == 0, K <= 3072):
-# ragged M and N, K at its limit, a run of tiles crossing weight columns
-PAIR128 = [
-    W.scaled(W.QKV, M=300, K=1024, N=272, rank=32, name="p128_ragged"),
-    W.scaled(W.QKV, M=520, K=3072, N=384, rank=64, name="p128_k3072_r64"),
-    W.scaled(W.QKV, M=257, K=512, N=128, rank=0, name="p128_rank0"),
-    W.scaled(W.QKV, M=1100, K=1536, N=640, rank=128, name="p128_r128"),
+# the two ways the quantizer adds the rank-r partials of a K split: through
+# the workspace (global memory) and inside one thread-block cluster
+# (distributed shared memory); a ragged tail, the largest cluster, rank 128
+QUANT_PLAN_CASES = [
+    W.scaled(W.QKV, M=300, K=1024, N=512, rank=64, name="qp_ragged_r64"),
+    W.scaled(W.QKV, M=128, K=3072, N=256, rank=32, name="qp_one_block_k3072"),
+    W.scaled(W.QKV, M=520, K=1536, N=384, rank=128, name="qp_r128"),
+    W.scaled(W.INT4_QKV, M=200, K=1024, N=272, rank=16, name="qp_int4"),
 ]
 
 
-@pytest.mark.parametrize("case", PAIR128, ids=lambda c: c.name)
-def test_pair128_kernel(case):
+@pytest.mark.parametrize("mode", [1, 2], ids=["workspace", "cluster"])
+@pytest.mark.parametrize("case", QUANT_PLAN_CASES, ids=lambda c: c.name)
+def test_quantizer_split_modes(case, mode):
     from bit_w4a4_quantized_token_b200 import _lib
 
-    _lib.svdq_debug_force_gemm_tiles(3)
+    _lib.svdq_debug_force_quant_plan(mode)
     try:
         check_case(case)
     finally:
-        _lib.svdq_debug_force_gemm_tiles(0)
+        _lib.svdq_debug_force_quant_plan(0)
 
 
 def test_static_tensor_scale():

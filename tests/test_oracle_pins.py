@@ -384,3 +384,120 @@ def test_int4_ties_to_even(oracle_mod):
     assert np.all(scales == 0x3F80)
     q = O.int4_codes_to_int(codes)[0, :16]
     assert list(q) == [7, 0, 0, 2, -2, 2, -2, 4, -4, 4, -4, 6, -6, 6, -6, 0]
+
+
+# ------------------------------------------- fused QKV + RMSNorm + RoPE pins
+def _bf16_weights(rng, D):
+    return f32_to_bf16_bits(rng.uniform(0.5, 1.5, size=D).astype(np.float32))
+
+
+def test_rms_norm_closed_forms(oracle_mod):
+    """A constant head vector c normalises to c / sqrt(c^2 + eps) * w; an
+    alternating +-a vector to +-a / sqrt(a^2 + eps) * w."""
+    O = oracle_mod
+    rng = np.random.default_rng(11)
+    D, eps = 128, 1e-6
+    w = _bf16_weights(rng, D)
+    wv = bf16_bits_to_f64(w)
+    for c in (3.0, -0.25, 1e-2):
+        out = O.rms_norm_head(np.full(D, c), w, eps)
+        np.testing.assert_allclose(out, c / np.sqrt(c * c + eps) * wv, rtol=1e-14)
+    a = 2.5
+    v = np.where(np.arange(D) % 2 == 0, a, -a)
+    np.testing.assert_allclose(O.rms_norm_head(v, w, eps), v / np.sqrt(a * a + eps) * wv, rtol=1e-14)
+    # eps matters for a zero vector: no division by zero, result zero
+    assert not np.any(O.rms_norm_head(np.zeros(D), w, eps))
+
+
+def test_rope_identity_at_angle_zero(oracle_mod):
+    O = oracle_mod
+    rng = np.random.default_rng(12)
+    v = rng.standard_normal(128)
+    assert np.array_equal(O.rope_head(v, np.ones(64), np.zeros(64)), v)
+
+
+def test_rope_is_complex_rotation(oracle_mod):
+    """Pair (2i, 2i+1) read as the complex number v[2i] + j v[2i+1], multiplied
+    by exp(j theta_i): a sign or index mistake in either component fails."""
+    O = oracle_mod
+    rng = np.random.default_rng(13)
+    v = rng.standard_normal(128)
+    th = rng.uniform(-np.pi, np.pi, size=64)
+    out = O.rope_head(v, np.cos(th), np.sin(th))
+    z = (v[0::2] + 1j * v[1::2]) * np.exp(1j * th)
+    np.testing.assert_allclose(out[0::2], z.real, rtol=0, atol=1e-14)
+    np.testing.assert_allclose(out[1::2], z.imag, rtol=0, atol=1e-14)
+    # a quarter turn maps (a, b) to (-b, a)
+    q = O.rope_head(v, np.zeros(64), np.ones(64))
+    assert np.array_equal(q[0::2], -v[1::2]) and np.array_equal(q[1::2], v[0::2])
+
+
+def test_rope_preserves_pair_norms_and_composes(oracle_mod):
+    O = oracle_mod
+    rng = np.random.default_rng(14)
+    v = rng.standard_normal(128)
+    t1, t2 = rng.uniform(-3, 3, size=64), rng.uniform(-3, 3, size=64)
+    r1 = O.rope_head(v, np.cos(t1), np.sin(t1))
+    np.testing.assert_allclose(np.hypot(r1[0::2], r1[1::2]), np.hypot(v[0::2], v[1::2]), rtol=1e-14)
+    r12 = O.rope_head(r1, np.cos(t2), np.sin(t2))
+    r_sum = O.rope_head(v, np.cos(t1 + t2), np.sin(t1 + t2))
+    np.testing.assert_allclose(r12, r_sum, rtol=0, atol=1e-13)
+
+
+def test_qkv_norm_rope_layout(oracle_mod):
+    """Q is columns [0, HD), K [HD, 2HD), V [2HD, 3HD) and passes through; Q
+    heads take the Q weight, K heads the K weight, each row its own angles;
+    the bf16 output is the rounding of the fp64 one."""
+    O = oracle_mod
+    rng = np.random.default_rng(15)
+    H, D, rows, eps = 3, 128, 5, 1e-6
+    y = rng.standard_normal((rows, 3 * H * D)) * 4.0
+    wq, wk = _bf16_weights(rng, D), _bf16_weights(rng, D)
+    th = rng.uniform(-np.pi, np.pi, size=(rows, D // 2))
+    out, outb = O.qkv_norm_rope(y, H, D, wq, wk, eps, np.cos(th), np.sin(th))
+    assert np.array_equal(out[:, 2 * H * D:], y[:, 2 * H * D:])
+    for m in (0, rows - 1):
+        for part, w in ((0, wq), (1, wk)):
+            for h in (0, H - 1):
+                cols = slice(part * H * D + h * D, part * H * D + (h + 1) * D)
+                want = O.rope_head(O.rms_norm_head(y[m, cols], w, eps), np.cos(th[m]), np.sin(th[m]))
+                assert np.array_equal(out[m, cols], want)
+    assert all(outb[m, n] == O.bf16_from_double(float(out[m, n])) for m in range(rows) for n in range(0, 3 * H * D, 97))
+
+
+# ------------------------------------------------------- SVD split pins
+def test_svd_split_eckart_young(oracle_mod):
+    """The residual of the best rank-r approximation: ||R||_F^2 is the sum of
+    the squared singular values past r, ||R||_2 the (r+1)-th; W_hat is
+    reassembled exactly; L_down has orthonormal columns, L_up orthogonal rows
+    of norms s_i."""
+    O = oracle_mod
+    rng = np.random.default_rng(31)
+    N, K, r = 48, 40, 6
+    W = f32_to_bf16_bits(rng.standard_normal((N, K)).astype(np.float32))
+    lam = rng.uniform(0.5, 4.0, size=K).astype(np.float32)
+    R, Ld, Lu, s = O.svd_split(W, lam, r)
+    W_hat = bf16_bits_to_f64(W) * lam.astype(np.float64)[None, :]
+    np.testing.assert_allclose(R + Lu.T @ Ld.T, W_hat, rtol=0, atol=1e-12)
+    assert np.linalg.norm(R) ** 2 == pytest.approx(float(np.sum(s[r:] ** 2)), rel=1e-10)
+    assert np.linalg.norm(R, 2) == pytest.approx(float(s[r]), rel=1e-10)
+    np.testing.assert_allclose(Ld.T @ Ld, np.eye(r), atol=1e-12)
+    np.testing.assert_allclose(Lu @ Lu.T, np.diag(s[:r] ** 2), atol=1e-9 * s[0] ** 2)
+    assert np.all(np.diff(s) <= 0)
+
+
+def test_svd_split_low_rank_weight(oracle_mod):
+    """A weight that is rank r up to its bf16 rounding: the residual is no
+    larger than that rounding (the truncation is the best rank-r fit)."""
+    O = oracle_mod
+    rng = np.random.default_rng(32)
+    N, K, r = 64, 48, 5
+    exact = rng.standard_normal((N, r)) @ rng.standard_normal((r, K))
+    W = f32_to_bf16_bits(exact.astype(np.float32))
+    R, _, _, s = O.svd_split(W, np.ones(K, np.float32), r)
+    assert np.linalg.norm(R) <= np.linalg.norm(bf16_bits_to_f64(W) - exact) * (1 + 1e-9)
+    # rank 0 leaves the whole smoothed weight in R
+    lam = rng.uniform(0.5, 4.0, size=K).astype(np.float32)
+    R0, Ld0, Lu0, _ = O.svd_split(W, lam, 0)
+    assert np.array_equal(R0, bf16_bits_to_f64(W) * lam.astype(np.float64)[None, :])
+    assert Ld0.shape == (K, 0) and Lu0.shape == (0, N)
