@@ -455,6 +455,105 @@ def time_qkv_fusion(dev, stream, flush, steps: int) -> dict:
             "fused_step": "svdq_quantize_act + svdq_gemm_w4a4_qkv_norm_rope"}
 
 
+def _graph_time(fns, stream, dev, flush, steps: int) -> float:
+    """Seconds per replay of one CUDA graph of `fns` (L2 flushed before each
+    replay, outside the events on the launching stream)."""
+    import torch
+
+    with torch.cuda.stream(stream):
+        for i in range(3):
+            flush.fill_(i)
+            for fn in fns:
+                fn()
+    torch.cuda.synchronize(dev)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for fn in fns:
+            fn()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    torch.cuda.synchronize(dev)
+    with torch.cuda.stream(stream):
+        for i in range(steps):
+            flush.fill_(i & 0xFF)
+            evs[i][0].record(stream)
+            g.replay()
+            evs[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    del g
+    return sum(a.elapsed_time(b) for a, b in evs) / steps / 1e3
+
+
+def time_w4a16(dev, stream, flush, steps: int, peaks: dict) -> dict:
+    """The weight-only int4 GEMM (awq_w4a16, int4 group 64) at the QKV
+    projection shape: bf16 x, packed int4 weight, fp16 tensor-core MMA."""
+    import torch
+
+    from bit_w4a4_quantized_token_b200 import _lib, layer
+    from bit_w4a4_quantized_token_b200 import workloads as W
+
+    case = W.QKV
+    with torch.cuda.stream(stream):
+        inp = W.make_inputs(case)
+        x, Wt, b = inp["x"].to(dev), inp["R"].to(dev), inp["b"].to(dev)
+        ones = torch.ones(case.K, dtype=torch.float32, device=dev)
+        p = layer.pack_weight(Wt, ones, None, None, b, precision="int4", stream=stream)
+        y = torch.empty(case.M, case.N, dtype=torch.bfloat16, device=dev)
+
+    def run():
+        _lib.svdq_gemm_w4a16(x, case.M, p.w_codes, p.w_scales, case.N, case.K, p.bias, y, stream=stream)
+
+    t = _graph_time([run], stream, dev, flush, steps)
+    st, site = _lib.svdq_device_status(clear=True)
+    if st != 0:
+        raise RuntimeError(f"device status {st} at site {site} in the W4A16 leg")
+    tf = case.flops / t / 1e12
+    nbytes = case.M * case.K * 2 + case.N * case.K // 2 + case.N * (case.K // 64) * 2 + case.M * case.N * 2
+    return {"workload": "awq_w4a16 weight-only int4 g64 GEMM at the QKV shape, M=4608 K=3072 N=9216",
+            "value": round(tf, 2), "unit": "TFLOP/s", "us": round(t * 1e6, 2),
+            "roofline": {"bound": "tensor", "achieved": round(tf, 2), "peak": peaks["bf16_tflops"],
+                         "unit": "TFLOP/s", "frac": round(tf / peaks["bf16_tflops"], 4),
+                         "peak_source": f"{peaks['source']} bf16 burst (fp16 has the same nominal rate)",
+                         "hbm_frac": round(nbytes / t / 1e9 / peaks["hbm_gbs"], 4), "algorithmic_bytes": nbytes}}
+
+
+def time_svd_split(dev, stream, flush, steps: int) -> dict:
+    """The offline split of the QKV weight (9216 x 3072) at rank 32: randomized
+    range finder with 8 oversamples and 2 power iterations."""
+    import torch
+
+    from bit_w4a4_quantized_token_b200 import _lib
+    from bit_w4a4_quantized_token_b200 import workloads as W
+
+    N, K, r, p = W.QKV.N, W.QKV.K, 32, 8
+    with torch.cuda.stream(stream):
+        d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in W.svd_split_inputs(N, K, r, p).items()}
+        R = torch.empty(N, K, dtype=torch.bfloat16, device=dev)
+        Ld = torch.empty(K, r, dtype=torch.bfloat16, device=dev)
+        Lu = torch.empty(r, N, dtype=torch.bfloat16, device=dev)
+        sv = torch.empty(r + p, dtype=torch.float32, device=dev)
+        ws = torch.empty(_lib.svdq_svd_split_workspace_bytes(N, K, r, p), dtype=torch.uint8, device=dev)
+
+    def run():
+        _lib.svdq_svd_split(d["W"], d["lam"], N, K, r, d["omega"], p, 2, R, Ld, Lu, sv, ws, ws.numel(),
+                            stream=stream)
+
+    with torch.cuda.stream(stream):
+        run()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            run()
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    t = e0.elapsed_time(e1) / steps / 1e3
+    st, site = _lib.svdq_device_status(clear=True)
+    if st != 0:
+        raise RuntimeError(f"device status {st} at site {site} in the SVD split leg")
+    return {"workload": f"offline SVD split of a {N} x {K} weight, rank {r}, oversample {p}, 2 power iterations",
+            "ms": round(t * 1e3, 3)}
+
+
 def time_graphs(shape, gs, steps, flush, sampler=None):
     """Device time per step of each graph (CUDA events on the launching stream,
     L2 flushed before every replay, outside the events)."""
@@ -602,6 +701,10 @@ def run_cuda(args) -> dict | None:
             del g2, s2
             torch.cuda.empty_cache()
         extra["qkv_norm_rope"] = time_qkv_fusion(dev, stream, flush, max(3, min(args.steps, 10)))
+        torch.cuda.empty_cache()
+        extra["w4a16_qkv"] = time_w4a16(dev, stream, flush, max(3, min(args.steps, 10)), peaks)
+        torch.cuda.empty_cache()
+        extra["svd_split_qkv"] = time_svd_split(dev, stream, flush, 3)
         torch.cuda.empty_cache()
     if world > 1:
         dist.barrier()

@@ -88,6 +88,8 @@ def _load():
         lib.oracle_nvfp4_linear.restype = None
         lib.oracle_int4_linear.argtypes = [P, P, P, L, L, P, P, L, P, P, L, P, P, P]
         lib.oracle_int4_linear.restype = None
+        lib.oracle_w4a16_linear.argtypes = [P, P, L, L, P, P, L, P, P, P]
+        lib.oracle_w4a16_linear.restype = None
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = ctypes.c_int
         _lib = lib
@@ -243,6 +245,27 @@ def int4_linear(xc, xs, wc, ws, L, L_up_bits, bias_bits, rows=None):
     b = None if bias_bits is None else _u16(bias_bits)
     _load().oracle_int4_linear(_ptr(xc), _ptr(xs), _ptr(rows_arr), nrows, K, _ptr(wc), _ptr(ws), N,
                                _ptr(Lc), _ptr(Lu), r, _ptr(b), _ptr(y), _ptr(ybf))
+    return y, ybf
+
+
+def w4a16_linear(x_bits, wc, ws, bias_bits, rows=None):
+    """Weight-only int4: y = x . (q s)^T + b in fp64 and its bf16 bits.
+
+    x_bits [M, K] bf16 bits used as they are; wc [N, K/2] two's-complement
+    nibbles and ws [N, K/64] bf16 bits as ``int4_quantize`` returns them.
+    """
+    x_bits = _u16(x_bits)
+    wc = np.ascontiguousarray(wc, np.uint8)
+    ws = _u16(ws)
+    K = x_bits.shape[1]
+    N = wc.shape[0]
+    rows_arr = None if rows is None else np.ascontiguousarray(rows, np.int64)
+    nrows = x_bits.shape[0] if rows is None else len(rows_arr)
+    y = np.zeros((nrows, N), np.float64)
+    ybf = np.zeros((nrows, N), np.uint16)
+    b = None if bias_bits is None else _u16(bias_bits)
+    _load().oracle_w4a16_linear(_ptr(x_bits), _ptr(rows_arr), nrows, K, _ptr(wc), _ptr(ws), N, _ptr(b),
+                                _ptr(y), _ptr(ybf))
     return y, ybf
 
 

@@ -418,3 +418,29 @@ int oracle_num_threads(void)
     return 1;
 #endif
 }
+
+/* Weight-only int4 linear (the awq_w4a16 scheme of the Diffusers docs page
+ * "Nunchaku Lite", section "Supported quantization types"): the bf16
+ * activation is used as it is; each weight is its int4 code times its bf16
+ * group-64 scale; the products and their sum are taken in fp64, then the bias
+ * is added and the result rounded once to bf16. */
+void oracle_w4a16_linear(const uint16_t* x, const long* rows, long nrows, long K,
+                         const uint8_t* wc, const uint16_t* ws, long N,
+                         const uint16_t* bias, double* y, uint16_t* ybf)
+{
+    const long G = 64;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long i = 0; i < nrows; ++i) {
+        long m = rows ? rows[i] : i;
+        double* yr = y + i * N;
+        for (long n = 0; n < N; ++n) {
+            double acc = 0.0;
+            for (long k = 0; k < K; ++k) {
+                double w = (double)int4_code(wc, K, n, k) * oracle_bf16_to_double(ws[n * (K / G) + k / G]);
+                acc += oracle_bf16_to_double(x[m * K + k]) * w;
+            }
+            yr[n] = acc + (bias ? oracle_bf16_to_double(bias[n]) : 0.0);
+            ybf[i * N + n] = oracle_bf16_from_double(yr[n]);
+        }
+    }
+}

@@ -386,6 +386,66 @@ def test_int4_ties_to_even(oracle_mod):
     assert list(q) == [7, 0, 0, 2, -2, 2, -2, 4, -4, 4, -4, 6, -6, 6, -6, 0]
 
 
+# ------------------------------------------------- weight-only int4 (W4A16)
+def test_w4a16_exact_on_integer_grid(oracle_mod):
+    """Integer weights with amax 7 per group get scale 1, so y is the exact
+    integer product x . W^T (small integers are exact in bf16)."""
+    O = oracle_mod
+    rng = np.random.default_rng(21)
+    M, K, N = 4, 192, 6
+    xv = rng.integers(-20, 21, size=(M, K)).astype(np.float64)
+    wv = rng.integers(-7, 8, size=(N, K)).astype(np.float64)
+    wv[:, ::64] = 7
+    wc, ws = O.int4_quantize(f32_to_bf16_bits(wv), None)
+    assert np.all(ws == 0x3F80)
+    bias = rng.integers(-5, 6, size=N).astype(np.float64)
+    y, ybf = O.w4a16_linear(f32_to_bf16_bits(xv), wc, ws, f32_to_bf16_bits(bias))
+    assert np.array_equal(y, xv @ wv.T + bias)
+    assert np.array_equal(ybf, f32_to_bf16_bits(xv @ wv.T + bias))
+
+
+def test_w4a16_bruteforce_tiny(oracle_mod):
+    """Exact rational evaluation of sum_k x q s + b, then the nearest bf16."""
+    O = oracle_mod
+    rng = np.random.default_rng(22)
+    M, K, N = 2, 128, 3
+    x = f32_to_bf16_bits(rng.standard_normal((M, K)).astype(np.float32))
+    w = f32_to_bf16_bits(rng.standard_normal((N, K)).astype(np.float32) * 0.1)
+    b = f32_to_bf16_bits(rng.standard_normal(N).astype(np.float32))
+    wc, ws = O.int4_quantize(w, None)
+    y, ybf = O.w4a16_linear(x, wc, ws, b)
+    nib = [[(int(wc[n, k // 2]) >> (4 * (k & 1))) & 15 for k in range(K)] for n in range(N)]
+    for m in range(M):
+        for n in range(N):
+            acc = Fraction(float(bf16_bits_to_f64(b[n])))
+            for k in range(K):
+                q = nib[n][k] - 16 if nib[n][k] >= 8 else nib[n][k]
+                acc += Fraction(float(bf16_bits_to_f64(x[m, k]))) * q * Fraction(float(bf16_bits_to_f64(ws[n, k // 64])))
+            assert abs(Fraction(y[m, n]) - acc) <= abs(acc) * Fraction(1, 2 ** 45) + Fraction(1, 2 ** 80)
+            assert ybf[m, n] == brute_bf16(float(acc))
+
+
+def test_w4a16_is_linear_in_x_and_bias_free_at_zero(oracle_mod):
+    """y(2x) = 2 y(x) exactly (power-of-two scaling), y(0) = b, and the rows
+    are independent (a row subset equals the same rows of the full call)."""
+    O = oracle_mod
+    rng = np.random.default_rng(23)
+    M, K, N = 5, 256, 7
+    xf = rng.standard_normal((M, K)).astype(np.float32)
+    w = f32_to_bf16_bits(rng.standard_normal((N, K)).astype(np.float32))
+    b = f32_to_bf16_bits(rng.standard_normal(N).astype(np.float32))
+    wc, ws = O.int4_quantize(w, None)
+    y1, _ = O.w4a16_linear(f32_to_bf16_bits(xf), wc, ws, None)
+    y2, _ = O.w4a16_linear(f32_to_bf16_bits(2 * xf), wc, ws, None)
+    assert np.array_equal(y2, 2 * y1)
+    y0, y0bf = O.w4a16_linear(np.zeros((M, K), np.uint16), wc, ws, b)
+    assert np.array_equal(y0bf, np.broadcast_to(b, (M, N)))
+    rows = np.array([4, 1])
+    ys, _ = O.w4a16_linear(f32_to_bf16_bits(xf), wc, ws, b, rows=rows)
+    yf, _ = O.w4a16_linear(f32_to_bf16_bits(xf), wc, ws, b)
+    assert np.array_equal(ys, yf[rows])
+
+
 # ------------------------------------------- fused QKV + RMSNorm + RoPE pins
 def _bf16_weights(rng, D):
     return f32_to_bf16_bits(rng.uniform(0.5, 1.5, size=D).astype(np.float32))
