@@ -90,6 +90,10 @@ def _load():
         lib.oracle_int4_linear.restype = None
         lib.oracle_w4a16_linear.argtypes = [P, P, L, L, P, P, L, P, P, P]
         lib.oracle_w4a16_linear.restype = None
+        lib.oracle_gelu.argtypes = [D, ctypes.c_int]
+        lib.oracle_gelu.restype = D
+        lib.oracle_gelu_bf16.argtypes = [P, L, ctypes.c_int, P]
+        lib.oracle_gelu_bf16.restype = None
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = ctypes.c_int
         _lib = lib
@@ -267,6 +271,39 @@ def w4a16_linear(x_bits, wc, ws, bias_bits, rows=None):
     _load().oracle_w4a16_linear(_ptr(x_bits), _ptr(rows_arr), nrows, K, _ptr(wc), _ptr(ws), N, _ptr(b),
                                 _ptr(y), _ptr(ybf))
     return y, ybf
+
+
+# ------------------------------------------------------------- GELU MLP
+def gelu(x: float, approx: int = 0) -> float:
+    """GELU of one value in fp64 (approx 0: x Phi(x); 1: the tanh form)."""
+    return float(_load().oracle_gelu(float(x), int(approx)))
+
+
+def gelu_bf16(x_bits: np.ndarray, approx: int = 0) -> np.ndarray:
+    """bf16 bits -> GELU in fp64 -> bf16 bits (one rounding)."""
+    x_bits = _u16(x_bits)
+    out = np.zeros_like(x_bits)
+    _load().oracle_gelu_bf16(_ptr(x_bits), x_bits.size, int(approx), _ptr(out))
+    return out
+
+
+def gelu_mlp(x_bits, fc1: dict, fc2: dict, S_x1: float, S_x2: float, approx: int = 0, rows=None):
+    """The DiT MLP block fc1 -> GELU -> fc2 with both linears SVDQ W4A4 nvfp4
+    layers: y1 = fc1(x) rounded to bf16, h = bf16(GELU(y1)), and fc2 applied
+    to h with its static activation tensor scale S_x2 (the fused kernel of the
+    Diffusers docs page "Nunchaku Lite", section "Fused kernels", hands the
+    same h to fc2's quantizer without writing it out).
+
+    fc1, fc2: dicts of bf16 bits / arrays with keys lam, R, L_down, L_up, b.
+    rows: optional subset of token rows (the MLP is row-wise).
+    Returns (fc1 result, h bits, fc2 result) for the chosen rows."""
+    x_bits = _u16(x_bits)
+    if rows is not None:
+        x_bits = np.ascontiguousarray(x_bits[np.asarray(rows)])
+    r1 = svdq_linear("nvfp4", x_bits, fc1["lam"], fc1["R"], fc1["L_down"], fc1["L_up"], fc1["b"], S_x=S_x1)
+    h = gelu_bf16(r1.y_bf16, approx)
+    r2 = svdq_linear("nvfp4", h, fc2["lam"], fc2["R"], fc2["L_down"], fc2["L_up"], fc2["b"], S_x=S_x2)
+    return r1, h, r2
 
 
 # --------------------------------------------- fused QKV + RMSNorm + RoPE

@@ -444,3 +444,24 @@ void oracle_w4a16_linear(const uint16_t* x, const long* rows, long nrows, long K
         }
     }
 }
+
+/* GELU, the activation between the two linear layers of the DiT MLP that the
+ * fused GELU-MLP kernel of the Diffusers docs page "Nunchaku Lite" (section
+ * "Fused kernels") targets.  approx = 0: the exact form x Phi(x), written
+ * with erfc so that the tail for negative x keeps its relative accuracy;
+ * approx = 1: the tanh form 0.5 x (1 + tanh(u)), u = sqrt(2/pi)(x + 0.044715
+ * x^3), written as x / (1 + exp(-2u)), the same function without the
+ * cancellation of 1 + tanh(u) for negative u. */
+double oracle_gelu(double x, int approx)
+{
+    if (approx == 0) return 0.5 * x * erfc(-x / sqrt(2.0));
+    const double u = sqrt(2.0 / 3.14159265358979323846) * (x + 0.044715 * x * x * x);
+    return x / (1.0 + exp(-2.0 * u));
+}
+
+/* bf16 in -> GELU in fp64 -> one rounding to bf16. */
+void oracle_gelu_bf16(const uint16_t* in, long n, int approx, uint16_t* out)
+{
+#pragma omp parallel for schedule(static)
+    for (long i = 0; i < n; ++i) out[i] = oracle_bf16_from_double(oracle_gelu(oracle_bf16_to_double(in[i]), approx));
+}

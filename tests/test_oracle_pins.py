@@ -446,6 +446,82 @@ def test_w4a16_is_linear_in_x_and_bias_free_at_zero(oracle_mod):
     assert np.array_equal(ys, yf[rows])
 
 
+# ------------------------------------------------------------ GELU MLP pins
+# Standard normal CDF values (textbook tables): Phi(1), Phi(-3), Phi(2).
+PHI_1, PHI_M3, PHI_2 = 0.8413447460685429, 0.0013498980316300946, 0.9772498680518208
+
+
+def test_gelu_exact_form_table_values(oracle_mod):
+    """GELU(x) = x Phi(x): checked against tabulated Phi and its limits."""
+    O = oracle_mod
+    assert O.gelu(0.0, 0) == 0.0
+    assert abs(O.gelu(1.0, 0) - PHI_1) <= 1e-15
+    assert abs(O.gelu(-3.0, 0) - (-3.0 * PHI_M3)) <= 1e-17
+    assert abs(O.gelu(2.0, 0) - 2.0 * PHI_2) <= 4e-16
+    assert O.gelu(10.0, 0) == 10.0                       # Phi(10) rounds to 1
+    v = O.gelu(-10.0, 0)                                 # -10 Phi(-10) = -7.6e-23: the tail keeps its digits
+    assert v < 0 and abs(v / -7.619853024160527e-23 - 1) < 1e-9
+
+
+def test_gelu_odd_part_identity(oracle_mod):
+    """Phi(x) + Phi(-x) = 1 gives GELU(x) - GELU(-x) = x, for both forms
+    (the tanh form's sigmoid obeys the same symmetry)."""
+    O = oracle_mod
+    rng = np.random.default_rng(31)
+    for x in rng.uniform(-6, 6, 200):
+        for approx in (0, 1):
+            d = O.gelu(float(x), approx) - O.gelu(float(-x), approx)
+            assert abs(d - x) <= 4e-15 * max(1.0, abs(x)), (x, approx)
+
+
+def test_gelu_tanh_form_is_close_to_exact_form(oracle_mod):
+    """The tanh form approximates x Phi(x) to a few 1e-4 over the real line;
+    a wrong constant (sqrt(2/pi), 0.044715) moves it well beyond."""
+    O = oracle_mod
+    xs = np.linspace(-8, 8, 3201)
+    err = max(abs(O.gelu(float(x), 1) - O.gelu(float(x), 0)) for x in xs)
+    assert 1e-5 < err < 5e-4
+    # at x = 1 the tanh form is 0.5 (1 + tanh(sqrt(2/pi) 1.044715))
+    assert abs(O.gelu(1.0, 1) - 0.5 * (1 + np.tanh(np.sqrt(2 / np.pi) * 1.044715))) <= 1e-15
+
+
+def test_gelu_bf16_rounds_once(oracle_mod):
+    O = oracle_mod
+    rng = np.random.default_rng(32)
+    x = f32_to_bf16_bits(np.concatenate([rng.standard_normal(300) * 3, [0.0, -0.0, 40.0, -40.0]]).astype(np.float32))
+    for approx in (0, 1):
+        out = O.gelu_bf16(x, approx)
+        for i in range(0, x.size, 7):
+            assert out[i] == brute_bf16(O.gelu(float(bf16_bits_to_f64(x[i])), approx)), (i, approx)
+
+
+def test_gelu_mlp_saturated_negative_gives_fc2_bias(oracle_mod):
+    """fc1 outputs near -100 make h = GELU(y1) = -0 exactly, so fc2 quantizes an
+    all-zero activation (codes 0x88, zero scales, no rank-r term) and its
+    output is its bias, bit for bit."""
+    O = oracle_mod
+    rng = np.random.default_rng(33)
+    M, D, Hd, r = 4, 64, 128, 16
+
+    def layer(N, K, bias):
+        return {"lam": rng.uniform(0.5, 2, K).astype(np.float32),
+                "R": f32_to_bf16_bits(rng.standard_normal((N, K)).astype(np.float32) * 1e-3),
+                "L_down": f32_to_bf16_bits(rng.standard_normal((K, r)).astype(np.float32) * 1e-3),
+                "L_up": f32_to_bf16_bits(rng.standard_normal((r, N)).astype(np.float32) * 1e-3),
+                "b": f32_to_bf16_bits(bias.astype(np.float32))}
+
+    fc1 = layer(Hd, D, np.full(Hd, -100.0))
+    fc2 = layer(D, Hd, rng.standard_normal(D))
+    x = f32_to_bf16_bits(rng.standard_normal((M, D)).astype(np.float32))
+    r1, h, r2 = O.gelu_mlp(x, fc1, fc2, S_x1=0.01, S_x2=0.01)
+    assert np.all(h == 0x8000)
+    assert np.all(r2.x_codes == 0x88) and np.all(r2.x_scales == 0)
+    assert np.array_equal(r2.y_bf16, np.broadcast_to(fc2["b"], (M, D)))
+    # rows are independent
+    _, h1, r2b = O.gelu_mlp(x, fc1, fc2, S_x1=0.01, S_x2=0.01, rows=[3, 1])
+    assert np.array_equal(r2b.y_bf16, r2.y_bf16[[3, 1]])
+
+
 # ------------------------------------------- fused QKV + RMSNorm + RoPE pins
 def _bf16_weights(rng, D):
     return f32_to_bf16_bits(rng.uniform(0.5, 1.5, size=D).astype(np.float32))
