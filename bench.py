@@ -483,6 +483,72 @@ def _graph_time(fns, stream, dev, flush, steps: int) -> float:
     return sum(a.elapsed_time(b) for a, b in evs) / steps / 1e3
 
 
+def time_gelu_mlp(dev, stream, flush, steps: int) -> dict:
+    """The DiT MLP block (3072 -> 12288 -> GELU -> 3072, rank 32, 4608 tokens):
+    fc1's GEMM with the fused GELU + fc2-activation epilogue against the
+    unfused path (fc1 GEMM -> bf16 -> GELU pass -> fc2's quantizer)."""
+    import torch
+
+    from bit_w4a4_quantized_token_b200 import _lib, layer
+    from bit_w4a4_quantized_token_b200 import workloads as W
+
+    c1, c2 = W.FC1, W.FC2
+    M, Hd = c1.M, c1.N
+    with torch.cuda.stream(stream):
+        s1, s2 = Shape(c1, dev, stream), Shape(c2, dev, stream)
+        p1, q1, p2 = s1.packed, s1.q, s2.packed
+        y1 = torch.empty(M, Hd, dtype=torch.bfloat16, device=dev)
+        h = torch.empty_like(y1)
+        y2 = torch.empty(M, c2.N, dtype=torch.bfloat16, device=dev)
+        # fc2's static activation scale: the amax pre-pass on this h, once
+        layer.gemm(q1, p1, y1, stream=stream)
+        _lib.svdq_gelu(y1, h, M * Hd, 0, stream=stream)
+        qu = layer.quantize_act(h, p2, stream=stream)
+        qf = layer.alloc_act(p2, M, dev)
+        qf.x_tensor_scale.copy_(qu.x_tensor_scale)
+        ws = torch.zeros(_lib.svdq_gelu_mlp_workspace_bytes(M, c2.rank) // 4, dtype=torch.float32, device=dev)
+    torch.cuda.synchronize(dev)
+
+    def fused_fc1():
+        _lib.svdq_gemm_w4a4_gelu_quant("nvfp4", 16, q1.x_codes, q1.x_scales, q1.x_tensor_scale, M, p1.w_codes,
+                                       p1.w_scales, p1.w_tensor_scale, Hd, c1.K, q1.lowrank_act, p1.L_up_t, c1.rank,
+                                       p1.bias, 0, p2.inv_lambda, p2.L_down_t, c2.rank, qf.x_tensor_scale,
+                                       p2.w_tensor_scale, qf.x_codes, qf.x_scales, qf.lowrank_act, ws, stream=stream)
+
+    def fc2_fused():
+        layer.gemm(qf, p2, y2, stream=stream)
+
+    def fc1_plain():
+        layer.gemm(q1, p1, y1, stream=stream)
+
+    def gelu():
+        _lib.svdq_gelu(y1, h, M * Hd, 0, stream=stream)
+
+    def quant2():   # static scale (compute flag 0)
+        _lib.svdq_quantize_act("nvfp4", 16, h, M, Hd, p2.inv_lambda, qu.x_tensor_scale, 0, p2.w_tensor_scale,
+                               p2.L_down_t, c2.rank, qu.x_codes, qu.x_scales, qu.lowrank_act, qu.workspace,
+                               stream=stream)
+
+    def fc2_unfused():
+        layer.gemm(qu, p2, y2, stream=stream)
+
+    t_f = _graph_time([s1.quant, fused_fc1, fc2_fused], stream, dev, flush, steps)
+    t_u = _graph_time([s1.quant, fc1_plain, gelu, quant2, fc2_unfused], stream, dev, flush, steps)
+    t_f1 = _graph_time([fused_fc1], stream, dev, flush, steps)
+    t_p1 = _graph_time([fc1_plain], stream, dev, flush, steps)
+    st, site = _lib.svdq_device_status(clear=True)
+    if st != 0:
+        raise RuntimeError(f"device status {st} at site {site} in the GELU MLP leg")
+    flops = c1.flops + c2.flops
+    return {"workload": "DiT MLP 3072 -> 12288 -> GELU -> 3072, rank 32 both layers, M=4608",
+            "step_us": {"fused": round(t_f * 1e6, 2), "unfused": round(t_u * 1e6, 2)},
+            "speedup": round(t_u / t_f, 3),
+            "fc1_us": {"gelu_quant_epilogue": round(t_f1 * 1e6, 2), "plain_epilogue": round(t_p1 * 1e6, 2)},
+            "value": round(flops / t_f / 1e12, 2), "unit": UNIT,
+            "fused_step": "quantize_act(fc1) + gemm_w4a4_gelu_quant(fc1) + gemm_w4a4(fc2)",
+            "unfused_step": "quantize_act(fc1) + gemm_w4a4(fc1) + gelu + quantize_act(fc2) + gemm_w4a4(fc2)"}
+
+
 def time_w4a16(dev, stream, flush, steps: int, peaks: dict) -> dict:
     """The weight-only int4 GEMM (awq_w4a16, int4 group 64) at the QKV
     projection shape: bf16 x, packed int4 weight, fp16 tensor-core MMA."""
@@ -701,6 +767,8 @@ def run_cuda(args) -> dict | None:
             del g2, s2
             torch.cuda.empty_cache()
         extra["qkv_norm_rope"] = time_qkv_fusion(dev, stream, flush, max(3, min(args.steps, 10)))
+        torch.cuda.empty_cache()
+        extra["gelu_mlp"] = time_gelu_mlp(dev, stream, flush, max(3, min(args.steps, 10)))
         torch.cuda.empty_cache()
         extra["w4a16_qkv"] = time_w4a16(dev, stream, flush, max(3, min(args.steps, 10)), peaks)
         torch.cuda.empty_cache()

@@ -30,7 +30,8 @@ GROUP_SIZES = {"nvfp4": 16, "int4": 64}
 EXPORTS = (
     "svdq_status_string", "svdq_abi_version", "svdq_last_error", "svdq_buffer_sizes", "svdq_pack_weight",
     "svdq_quantize_act_workspace_bytes", "svdq_quantize_act", "svdq_quantize_act_noalloc", "svdq_gemm_w4a4",
-    "svdq_gemm_w4a4_qkv_norm_rope", "svdq_qkv_norm_rope", "svdq_gemm_w4a16", "svdq_svd_split_workspace_bytes",
+    "svdq_gemm_w4a4_qkv_norm_rope", "svdq_qkv_norm_rope", "svdq_gelu_mlp_workspace_bytes",
+    "svdq_gemm_w4a4_gelu_quant", "svdq_gelu", "svdq_gemm_w4a16", "svdq_svd_split_workspace_bytes",
     "svdq_svd_split",
     "svdq_device_status",
     "svdq_debug_set_wait_limit_ns", "svdq_debug_timeout_probe", "svdq_debug_override_capability",
@@ -82,6 +83,13 @@ def _load():
     lib.svdq_gemm_w4a4_qkv_norm_rope.restype = I
     lib.svdq_qkv_norm_rope.argtypes = [P, P, I64, I, I, P, P, F, P, P, P]
     lib.svdq_qkv_norm_rope.restype = I
+    lib.svdq_gelu_mlp_workspace_bytes.argtypes = [I64, I, ctypes.POINTER(ctypes.c_size_t)]
+    lib.svdq_gelu_mlp_workspace_bytes.restype = I
+    lib.svdq_gemm_w4a4_gelu_quant.argtypes = [I, I, P, P, P, I64, P, P, P, I64, I64, P, P, I, P, I, P, P, I, P, P, P,
+                                              P, P, P, ctypes.c_size_t, P]
+    lib.svdq_gemm_w4a4_gelu_quant.restype = I
+    lib.svdq_gelu.argtypes = [P, P, I64, I, P]
+    lib.svdq_gelu.restype = I
     lib.svdq_gemm_w4a16.argtypes = [P, I64, P, P, I64, I64, P, P, P]
     lib.svdq_gemm_w4a16.restype = I
     lib.svdq_svd_split_workspace_bytes.argtypes = [I64, I64, I, I, ctypes.POINTER(ctypes.c_size_t)]
@@ -209,6 +217,31 @@ def svdq_qkv_norm_rope(y_in, y_out, M, heads, head_dim, norm_q, norm_k, eps, rop
     _check(lib.svdq_qkv_norm_rope(_ptr(y_in), _ptr(y_out), int(M), int(heads), int(head_dim), _ptr(norm_q),
                                   _ptr(norm_k), float(eps), _ptr(rope_cos), _ptr(rope_sin), _stream(stream)),
            "svdq_qkv_norm_rope")
+
+
+def svdq_gelu_mlp_workspace_bytes(M, next_rank) -> int:
+    out = ctypes.c_size_t(0)
+    _check(lib.svdq_gelu_mlp_workspace_bytes(int(M), int(next_rank), ctypes.byref(out)),
+           "svdq_gelu_mlp_workspace_bytes")
+    return int(out.value)
+
+
+def svdq_gemm_w4a4_gelu_quant(precision, group_size, x_codes, x_scales, x_tensor_scale, M, w_codes, w_scales,
+                              w_tensor_scale, N, K, lowrank_act, L_up_t, rank, bias, gelu_approx, next_inv_lambda,
+                              next_L_down_t, next_rank, next_x_tensor_scale, next_w_tensor_scale, next_x_codes,
+                              next_x_scales, next_lowrank_act, workspace, workspace_bytes=0, stream=None) -> None:
+    if workspace is not None and not isinstance(workspace, int) and not workspace_bytes:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    _check(lib.svdq_gemm_w4a4_gelu_quant(
+        _prec(precision), int(group_size), _ptr(x_codes), _ptr(x_scales), _ptr(x_tensor_scale), int(M),
+        _ptr(w_codes), _ptr(w_scales), _ptr(w_tensor_scale), int(N), int(K), _ptr(lowrank_act), _ptr(L_up_t),
+        int(rank), _ptr(bias), int(gelu_approx), _ptr(next_inv_lambda), _ptr(next_L_down_t), int(next_rank),
+        _ptr(next_x_tensor_scale), _ptr(next_w_tensor_scale), _ptr(next_x_codes), _ptr(next_x_scales),
+        _ptr(next_lowrank_act), _ptr(workspace), int(workspace_bytes), _stream(stream)), "svdq_gemm_w4a4_gelu_quant")
+
+
+def svdq_gelu(x, y, n, approx=0, stream=None) -> None:
+    _check(lib.svdq_gelu(_ptr(x), _ptr(y), int(n), int(approx), _stream(stream)), "svdq_gelu")
 
 
 def svdq_gemm_w4a16(x, M, w_codes, w_scales, N, K, bias, y, stream=None) -> None:

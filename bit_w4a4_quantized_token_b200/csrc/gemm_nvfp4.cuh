@@ -64,6 +64,18 @@ struct GemmArgs {
     const float* rope_sin;
     float eps;
     int q_cols, qk_cols;
+    // Fused GELU + next-layer activation epilogue (pair kernel, kEpiGelu):
+    // h = bf16(GELU(y)) is not stored; the next layer's activation step is
+    // done on it instead (gelu_mlp.cuh).
+    int gelu_approx;                 // 0: x Phi(x); 1: tanh form
+    const float* nx_inv_lambda;      // [N] 1 / lambda of the next layer
+    const __nv_bfloat16* nx_ldt;     // [2, nx_rank, N] hi/lo planes of L_down / lambda (next layer)
+    int nx_rank;                     // 0, 16 or 32
+    const float* nx_x_scale;         // the next layer's static activation tensor scale
+    uint8_t* nx_codes;               // [M, N / 2] nvfp4 codes of h / lambda
+    uint8_t* nx_scales;              // their E4M3 group scales, tensor-core layout, K = N
+    float* nx_acc;                   // [M, nx_rank] fp32 sums of h (L_down / lambda), zero on entry
+    int nx_rows_pad;                 // rows of nx_scales: M rounded up to 128
 };
 
 enum : uint32_t { kSiteGmEmpty = 16, kSiteGmFull = 17, kSiteGmAcc = 18, kSiteGmDrain = 19, kSiteGmAccEmpty = 20 };

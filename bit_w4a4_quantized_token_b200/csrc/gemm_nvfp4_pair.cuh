@@ -35,9 +35,13 @@
 // cycles, whatever the box size, and a stage of four K-steps lasts 512 cycles
 // of MMA; so each producer role runs on two lanes that take alternate stages.
 //
-// With the fused QKV epilogue (kQkv, GemmArgs.qk_cols > 0) the warps whose 128
-// columns are a Q or K head apply that head's RMSNorm and rotary embedding
-// (qkv_norm_rope.cuh) to the fp32 results before the bf16 store.
+// With the fused QKV epilogue (kEpiQkv, GemmArgs.qk_cols > 0) the warps whose
+// 128 columns are a Q or K head apply that head's RMSNorm and rotary embedding
+// (qkv_norm_rope.cuh) to the fp32 results before the bf16 store.  With the
+// fused GELU epilogue (kEpiGelu) nothing is stored for y: each row's
+// h = bf16(GELU(bf16(y))) is quantized for the next layer and its rank-r
+// down-projection partial sums are added into a global fp32 buffer
+// (gp_gelu_epilogue below, gelu_mlp.cuh).
 //
 // Measured alternative, not kept: four extra warps writing the scale factors
 // into TMEM with tcgen05.st (so that the MMA thread issues MMAs only) ran the
@@ -45,6 +49,7 @@
 // their shared-memory reads of the staged scale blocks slowed the TMA fill of
 // the ring, whose stages then landed 3-5 us after issue.
 #pragma once
+#include "gelu_mlp.cuh"
 #include "gemm_nvfp4.cuh"
 #include "qkv_norm_rope.cuh"
 
@@ -86,7 +91,15 @@ constexpr int kLanesPerRole = 2;               // producer lanes per role, takin
 constexpr uint32_t kAccEmptyArrivals = 2 * kEpiWarps;
 constexpr size_t SMEM_BYTES = 1024 + (size_t)kStages * STAGE_BYTES + 256;
 static_assert(SMEM_BYTES <= 227 * 1024, "stage ring does not fit in shared memory");
+// kEpiGelu: a 2 KB transpose buffer per epilogue warp (32 rows x 32 bf16)
+constexpr int kGeluScratch = 2048;
+constexpr size_t SMEM_BYTES_GELU = SMEM_BYTES + (size_t)kEpiWarps * kGeluScratch;
+static_assert(SMEM_BYTES_GELU <= 227 * 1024, "GELU epilogue buffers do not fit in shared memory");
 }  // namespace gp
+
+// Epilogue variants of the pair kernel (separate instantiations, so that the
+// plain kernel keeps its registers).
+enum : int { kEpiPlain = 0, kEpiQkv = 1, kEpiGelu = 2 };
 
 enum : uint32_t {
     kSiteGpEmpty = 24,
@@ -119,9 +132,149 @@ __device__ __forceinline__ void gp_issue_stage(uint32_t acc, uint64_t da, uint64
     }
 }
 
-// kQkv: the fused QKV + RMSNorm + RoPE epilogue is compiled in (a separate
-// instantiation, so that the plain kernel keeps its registers).
-template <bool kQkv>
+// The fused GELU epilogue of one thread's row (grow) over one warp's 128
+// columns [nbase, nbase + 128) of a tile; acc holds the fp32 accumulators.
+//  1. y = S acc + b rounded to bf16 (what the plain epilogue stores), then
+//     h = bf16(GELU(y)): the next layer's input, never written out;
+//  2. the next layer's nvfp4 step on h, with the arithmetic of the activation
+//     quantizer (quantize_act.cuh): v = h * (1 / lambda), per 16 columns the
+//     E4M3 scale of amax(v) / (6 S2) and the E2M1 codes of v / (scale S2);
+//     codes go to row grow of nx_codes, scales to the tensor-core layout
+//     (rows between M and the 128-row padding get scale 0, as the quantizer
+//     writes them);
+//  3. the next layer's rank-r down-projection over these 128 columns,
+//     h [32 rows x 128] (L_down / lambda) [128 x r], on the warp's tensor
+//     cores (m16n8k16 bf16 MMAs; h is exact in bf16, L_down / lambda enters
+//     as its hi and lo bf16 planes), added into nx_acc with fp32 atomics.
+// Every lane takes part in step 3 (warp-wide MMAs), whatever its row.
+__device__ __forceinline__ void gp_gelu_epilogue(const uint32_t (&acc)[128], const GemmArgs& a, float S, float S2,
+                                                 float six_s2, int64_t grow, int nbase, uint32_t scr,
+                                                 uint32_t lane) {
+    const bool row_ok = grow < a.M;
+    const int64_t half_k = (int64_t)a.N / 2;
+    const int64_t kg4n = a.N / 64;
+    uint32_t hpk[64];
+    uint32_t cw[4] = {0u, 0u, 0u, 0u};
+    uint32_t sword = 0u;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        const int n = nbase + 16 * c;
+        uint32_t bw[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+        if (a.bias) {
+            const uint4 w0 = __ldg(reinterpret_cast<const uint4*>(a.bias + n));
+            const uint4 w1 = __ldg(reinterpret_cast<const uint4*>(a.bias + n) + 1);
+            bw[0] = w0.x, bw[1] = w0.y, bw[2] = w0.z, bw[3] = w0.w;
+            bw[4] = w1.x, bw[5] = w1.y, bw[6] = w1.z, bw[7] = w1.w;
+        }
+        float h[16];
+#pragma unroll
+        for (int p = 0; p < 8; ++p) {
+            const float o0 = fmaf(__uint_as_float(acc[16 * c + 2 * p]), S, bf16lo_to_f32(bw[p]));
+            const float o1 = fmaf(__uint_as_float(acc[16 * c + 2 * p + 1]), S, bf16hi_to_f32(bw[p]));
+            const __nv_bfloat162 y2 = __floats2bfloat162_rn(o0, o1);
+            const __nv_bfloat162 h2 = __floats2bfloat162_rn(gelu_f32(__low2float(y2), a.gelu_approx),
+                                                            gelu_f32(__high2float(y2), a.gelu_approx));
+            hpk[8 * c + p] = *reinterpret_cast<const uint32_t*>(&h2);
+            h[2 * p] = __low2float(h2);
+            h[2 * p + 1] = __high2float(h2);
+        }
+        const float4* il = reinterpret_cast<const float4*>(a.nx_inv_lambda + n);
+        float v[16];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float4 l = __ldg(il + q);
+            fmul2_rn(h[4 * q], h[4 * q + 1], l.x, l.y, v[4 * q], v[4 * q + 1]);
+            fmul2_rn(h[4 * q + 2], h[4 * q + 3], l.z, l.w, v[4 * q + 2], v[4 * q + 3]);
+        }
+        uint32_t lo, hi;
+        const uint32_t eb = quant_group16(v, S2, six_s2, lo, hi);
+        cw[2 * (c & 1)] = lo;
+        cw[2 * (c & 1) + 1] = hi;
+        sword |= eb << (8 * (c & 3));
+        if (c & 1) {
+            if (row_ok)
+                *reinterpret_cast<uint4*>(a.nx_codes + grow * half_k + (n - 16) / 2) =
+                    make_uint4(cw[0], cw[1], cw[2], cw[3]);
+        }
+        if ((c & 3) == 3) {
+            const int64_t g0 = (n - 48) / 16;   // the first of these four groups (a multiple of 4)
+            if (grow < a.nx_rows_pad)
+                *reinterpret_cast<uint32_t*>(a.nx_scales + sf_offset(grow, g0, kg4n)) = row_ok ? sword : 0u;
+            sword = 0u;
+        }
+    }
+    if (a.nx_rank == 0) return;
+    // ---- rank-r down-projection of the next layer over these 128 columns
+    const int g = (int)(lane >> 2), t = (int)(lane & 3);
+    const int nj = a.nx_rank / 8;                     // 2 or 4 column blocks of 8
+    const int64_t plane = (int64_t)a.nx_rank * a.N;   // hi plane, then lo plane
+    float lacc[2][4][4];
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) lacc[mt][j][e] = 0.0f;
+    const uint32_t my_row = scr + 64u * lane;
+#pragma unroll
+    for (int kc = 0; kc < 4; ++kc) {
+        // this lane's row, columns 32 kc .. 32 kc + 31, in four 16-byte pieces
+        // placed at piece ^ ((row / 2) % 4) so that neither these stores nor
+        // the ldmatrix reads below meet a bank twice
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch)
+            st_shared_v4(my_row + ((uint32_t)(ch ^ ((lane >> 1) & 3)) << 4), hpk[16 * kc + 4 * ch],
+                         hpk[16 * kc + 4 * ch + 1], hpk[16 * kc + 4 * ch + 2], hpk[16 * kc + 4 * ch + 3]);
+        __syncwarp();
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks) {
+            uint32_t af[2][4];
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt) {
+                const uint32_t rr = 16u * mt + ((lane >> 3) & 1u) * 8u + (lane & 7u);
+                const uint32_t kch = 2u * ks + (lane >> 4);
+                ldmatrix_x4(af[mt], scr + 64u * rr + ((kch ^ ((rr >> 1) & 3u)) << 4));
+            }
+            const int64_t k = nbase + 32 * kc + 16 * ks + 2 * t;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                if (j < nj) {
+                    const __nv_bfloat16* bp = a.nx_ldt + (int64_t)(8 * j + g) * a.N + k;
+                    const uint32_t bh0 = __ldg(reinterpret_cast<const unsigned int*>(bp));
+                    const uint32_t bh1 = __ldg(reinterpret_cast<const unsigned int*>(bp + 8));
+                    const uint32_t bl0 = __ldg(reinterpret_cast<const unsigned int*>(bp + plane));
+                    const uint32_t bl1 = __ldg(reinterpret_cast<const unsigned int*>(bp + plane + 8));
+#pragma unroll
+                    for (int mt = 0; mt < 2; ++mt) {
+                        mma_16816_bf16(lacc[mt][j], af[mt], bh0, bh1);
+                        mma_16816_bf16(lacc[mt][j], af[mt], bl0, bl1);
+                    }
+                }
+            }
+        }
+        __syncwarp();
+    }
+    const int64_t row0 = grow - (int64_t)lane;   // the warp's first row
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            if (j < nj) {
+                const int64_t r0 = row0 + 16 * mt + g, r1 = r0 + 8;
+                const int col = 8 * j + 2 * t;
+                if (r0 < a.M)
+                    atomicAdd(reinterpret_cast<float2*>(a.nx_acc + r0 * a.nx_rank + col),
+                              make_float2(lacc[mt][j][0], lacc[mt][j][1]));
+                if (r1 < a.M)
+                    atomicAdd(reinterpret_cast<float2*>(a.nx_acc + r1 * a.nx_rank + col),
+                              make_float2(lacc[mt][j][2], lacc[mt][j][3]));
+            }
+        }
+}
+
+// kEpi: kEpiPlain, kEpiQkv (the fused QKV + RMSNorm + RoPE epilogue) or
+// kEpiGelu (the fused GELU + next-layer activation epilogue).
+template <int kEpi>
 __global__ void __launch_bounds__(gp::kThreads, 1)
     gemm_nvfp4_pair_kernel(const __grid_constant__ CUtensorMap tm_xc, const __grid_constant__ CUtensorMap tm_wc,
                            const __grid_constant__ CUtensorMap tm_sfa, const __grid_constant__ CUtensorMap tm_sfb,
@@ -331,6 +484,13 @@ __global__ void __launch_bounds__(gp::kThreads, 1)
         const int row = (int)(32u * q + lane);
         const float S = __fmul_rn(*a.x_scale, *a.w_scale);
         const uint32_t acc_empty_leader = cluster_addr(acc_empty, 0);
+        float gelu_s2 = 1.0f, gelu_six_s2 = 6.0f;
+        uint32_t gelu_scr = 0u;
+        if (kEpi == kEpiGelu) {
+            gelu_s2 = *a.nx_x_scale;
+            gelu_six_s2 = __fmul_rn(6.0f, gelu_s2);
+            gelu_scr = smem_u32(smem + (size_t)kStages * STAGE_BYTES + 256);
+        }
         int local = 0;
         for (int tile = t_begin; tile < t_end; ++tile, ++local) {
             const int m_tile = tile / a.n_tiles, n_tile = tile - m_tile * a.n_tiles;
@@ -354,9 +514,16 @@ __global__ void __launch_bounds__(gp::kThreads, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(acc_empty_leader);   // this half of the pair is drained
+            if (kEpi == kEpiGelu) {
+                // warp-uniform: with N % 128 == 0 a warp's columns are all in or all out
+                if (nbase < a.N)
+                    gp_gelu_epilogue(acc, a, S, gelu_s2, gelu_six_s2, grow, nbase,
+                                     gelu_scr + (uint32_t)(warp - kEpiWarp0) * (uint32_t)kGeluScratch, lane);
+                continue;
+            }
             if (grow >= a.M) continue;
             __nv_bfloat16* yrow = a.y + grow * (int64_t)a.N;
-            if (kQkv && nbase < a.qk_cols) {
+            if (kEpi == kEpiQkv && nbase < a.qk_cols) {
                 // this warp's 128 columns are one Q or K head of a to_qkv
                 // projection (qkv_norm_rope.cuh): RMSNorm over them, then the
                 // rotary pairs, on the fp32 values before the single bf16 rounding

@@ -126,10 +126,12 @@ svdq_status check_device() {
                                  (int)i4::SMEM_BYTES) != cudaSuccess ||
             cudaFuncSetAttribute(gemm_w4a16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)aw::SMEM_BYTES) != cudaSuccess ||
-            cudaFuncSetAttribute(gemm_nvfp4_pair_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            cudaFuncSetAttribute(gemm_nvfp4_pair_kernel<kEpiPlain>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)gp::SMEM_BYTES) != cudaSuccess ||
-            cudaFuncSetAttribute(gemm_nvfp4_pair_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)gp::SMEM_BYTES) != cudaSuccess)
+            cudaFuncSetAttribute(gemm_nvfp4_pair_kernel<kEpiQkv>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)gp::SMEM_BYTES) != cudaSuccess ||
+            cudaFuncSetAttribute(gemm_nvfp4_pair_kernel<kEpiGelu>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)gp::SMEM_BYTES_GELU) != cudaSuccess)
             return cuda_fail("setting kernel shared-memory limits");
         g_device_ready[dev] = true;
     }
@@ -520,7 +522,7 @@ int pair_clusters() {
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         int n = 0;
-        if (cudaOccupancyMaxActiveClusters(&n, gemm_nvfp4_pair_kernel<false>, &cfg) != cudaSuccess || n <= 0) {
+        if (cudaOccupancyMaxActiveClusters(&n, gemm_nvfp4_pair_kernel<kEpiPlain>, &cfg) != cudaSuccess || n <= 0) {
             cudaGetLastError();
             n = num_sms() / 2;
         }
@@ -540,10 +542,24 @@ struct QkvEpilogue {
     const float* rope_sin = nullptr;
 };
 
+// The fused GELU + next-layer activation epilogue's arguments (next_x_scale ==
+// nullptr: not used).
+struct GeluEpilogue {
+    int approx = 0;
+    const float* next_inv_lambda = nullptr;
+    const void* next_L_down_t = nullptr;
+    int next_rank = 0;
+    const float* next_x_scale = nullptr;
+    void* next_codes = nullptr;
+    void* next_scales = nullptr;
+    float* next_acc = nullptr;
+};
+
 svdq_status gemm_nvfp4_pair(const void* x_codes, const void* x_scales, const float* x_scale, int64_t M,
                             const void* w_codes, const void* w_scales, const float* w_scale, int64_t N, int64_t K,
                             const void* lowrank, const void* L_up_t, int rank, const void* bias, void* y,
-                            cudaStream_t st, const QkvEpilogue& qkv = QkvEpilogue()) {
+                            cudaStream_t st, const QkvEpilogue& qkv = QkvEpilogue(),
+                            const GeluEpilogue& gelu = GeluEpilogue()) {
     CUtensorMap tm_xc, tm_wc, tm_sfa, tm_sfb, tm_L, tm_Lup;
     const int64_t kg4 = K / 64;
     if (!make_map(&tm_xc, CU_TENSOR_MAP_DATA_TYPE_UINT8, x_codes, (uint64_t)K / 2, (uint64_t)M, (uint64_t)K / 2,
@@ -585,6 +601,17 @@ svdq_status gemm_nvfp4_pair(const void* x_codes, const void* x_scales, const flo
         a.q_cols = qkv.heads * 128;
         a.qk_cols = 2 * qkv.heads * 128;
     }
+    if (gelu.next_x_scale) {
+        a.gelu_approx = gelu.approx;
+        a.nx_inv_lambda = gelu.next_inv_lambda;
+        a.nx_ldt = reinterpret_cast<const __nv_bfloat16*>(gelu.next_L_down_t);
+        a.nx_rank = gelu.next_rank;
+        a.nx_x_scale = gelu.next_x_scale;
+        a.nx_codes = reinterpret_cast<uint8_t*>(gelu.next_codes);
+        a.nx_scales = reinterpret_cast<uint8_t*>(gelu.next_scales);
+        a.nx_acc = gelu.next_acc;
+        a.nx_rows_pad = (int)round_up(M, 128);
+    }
     const int64_t mt = (M + gp::BM - 1) / gp::BM, nt = (N + gp::BN - 1) / gp::BN;
     if (mt * nt > (int64_t(1) << 30)) return SVDQ_ERR_UNSUPPORTED_SHAPE;
     a.m_tiles = (int)mt;
@@ -592,11 +619,17 @@ svdq_status gemm_nvfp4_pair(const void* x_codes, const void* x_scales, const flo
     const int clusters = (int)std::min<int64_t>(mt * nt, pair_clusters());
     // programmatic dependent launch: the kernel's prologue overlaps the tail of
     // the activation quantizer, which releases its dependents early
-    const cudaError_t e =
-        qkv.heads > 0 ? launch_ex(gemm_nvfp4_pair_kernel<true>, dim3(2 * (unsigned)clusters), dim3(gp::kThreads),
-                                  gp::SMEM_BYTES, st, 2u, tm_xc, tm_wc, tm_sfa, tm_sfb, tm_L, tm_Lup, a)
-                      : launch_ex(gemm_nvfp4_pair_kernel<false>, dim3(2 * (unsigned)clusters), dim3(gp::kThreads),
-                                  gp::SMEM_BYTES, st, 2u, tm_xc, tm_wc, tm_sfa, tm_sfb, tm_L, tm_Lup, a);
+    const dim3 grid(2 * (unsigned)clusters), block(gp::kThreads);
+    cudaError_t e;
+    if (gelu.next_x_scale)
+        e = launch_ex(gemm_nvfp4_pair_kernel<kEpiGelu>, grid, block, gp::SMEM_BYTES_GELU, st, 2u, tm_xc, tm_wc,
+                      tm_sfa, tm_sfb, tm_L, tm_Lup, a);
+    else if (qkv.heads > 0)
+        e = launch_ex(gemm_nvfp4_pair_kernel<kEpiQkv>, grid, block, gp::SMEM_BYTES, st, 2u, tm_xc, tm_wc, tm_sfa,
+                      tm_sfb, tm_L, tm_Lup, a);
+    else
+        e = launch_ex(gemm_nvfp4_pair_kernel<kEpiPlain>, grid, block, gp::SMEM_BYTES, st, 2u, tm_xc, tm_wc, tm_sfa,
+                      tm_sfb, tm_L, tm_Lup, a);
     if (e != cudaSuccess) return cuda_fail("gemm_nvfp4_pair_kernel launch");
     return launch_status("gemm_nvfp4_pair_kernel launch");
 }
@@ -959,6 +992,92 @@ svdq_status svdq_qkv_norm_rope(const void* y_in, void* y_out, int64_t M, int hea
         SVDQ_TRY(launch_status("copy_v_kernel launch"));
     }
     return SVDQ_OK;
+}
+
+svdq_status svdq_gelu_mlp_workspace_bytes(int64_t M, int next_rank, size_t* bytes) {
+    if (!bytes) return SVDQ_ERR_INVALID_ARG;
+    SVDQ_TRY(check_rank(next_rank));
+    if (next_rank > 32 || M < 1 || M >= (int64_t(1) << 31)) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+    *bytes = (size_t)M * (size_t)next_rank * sizeof(float);
+    return SVDQ_OK;
+}
+
+svdq_status svdq_gemm_w4a4_gelu_quant(svdq_precision p, int group_size, const void* x_codes, const void* x_scales,
+                                      const float* x_tensor_scale, int64_t M, const void* w_codes,
+                                      const void* w_scales, const float* w_tensor_scale, int64_t N, int64_t K,
+                                      const void* lowrank_act, const void* L_up_t, int rank, const void* bias,
+                                      int gelu_approx, const float* next_inv_lambda, const void* next_L_down_t,
+                                      int next_rank, const float* next_x_tensor_scale,
+                                      const float* next_w_tensor_scale, void* next_x_codes, void* next_x_scales,
+                                      void* next_lowrank_act, void* workspace, size_t workspace_bytes,
+                                      svdq_stream_t stream) {
+    SVDQ_TRY(check_precision(p, group_size));
+    if (p != SVDQ_NVFP4) return SVDQ_ERR_INVALID_ARG;   // the fused epilogue belongs to the nvfp4 GEMM
+    SVDQ_TRY(check_rank(rank));
+    SVDQ_TRY(check_rank(next_rank));
+    if (next_rank > 32) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+    if (gelu_approx != 0 && gelu_approx != 1) return SVDQ_ERR_INVALID_ARG;
+    SVDQ_TRY(check_dims(M, K));
+    SVDQ_TRY(check_dims(N, K));
+    if (N % 128 != 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;   // N is the next layer's K
+    SVDQ_TRY(check_ptr(x_codes));
+    SVDQ_TRY(check_ptr(x_scales));
+    SVDQ_TRY(check_ptr(w_codes));
+    SVDQ_TRY(check_ptr(w_scales));
+    SVDQ_TRY(check_ptr(x_tensor_scale));
+    SVDQ_TRY(check_ptr(w_tensor_scale));
+    SVDQ_TRY(check_opt_ptr(bias));
+    if (rank > 0) {
+        SVDQ_TRY(check_ptr(lowrank_act));
+        SVDQ_TRY(check_ptr(L_up_t));
+    }
+    SVDQ_TRY(check_ptr(next_inv_lambda));
+    SVDQ_TRY(check_ptr(next_x_tensor_scale));
+    SVDQ_TRY(check_ptr(next_x_codes));
+    SVDQ_TRY(check_ptr(next_x_scales));
+    if (next_rank > 0) {
+        SVDQ_TRY(check_ptr(next_L_down_t));
+        SVDQ_TRY(check_ptr(next_w_tensor_scale));
+        SVDQ_TRY(check_ptr(next_lowrank_act));
+        SVDQ_TRY(check_ptr(workspace));
+        if (workspace_bytes < (size_t)M * (size_t)next_rank * sizeof(float)) return SVDQ_ERR_INVALID_ARG;
+    }
+    SVDQ_TRY(check_device());
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    GeluEpilogue g;
+    g.approx = gelu_approx;
+    g.next_inv_lambda = next_inv_lambda;
+    g.next_L_down_t = next_L_down_t;
+    g.next_rank = next_rank;
+    g.next_x_scale = next_x_tensor_scale;
+    g.next_codes = next_x_codes;
+    g.next_scales = next_x_scales;
+    g.next_acc = reinterpret_cast<float*>(workspace);
+    SVDQ_TRY(gemm_nvfp4_pair(x_codes, x_scales, x_tensor_scale, M, w_codes, w_scales, w_tensor_scale, N, K,
+                             lowrank_act, L_up_t, rank, bias, nullptr, st, QkvEpilogue(), g));
+    if (next_rank > 0) {
+        const int64_t count = M * next_rank;
+        const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((count + 255) / 256, 2LL * num_sms()));
+        if (launch_ex(lowrank_finalize_kernel, dim3((unsigned)grid), dim3(256), 0, st, 1u,
+                      reinterpret_cast<float*>(workspace), count, next_x_tensor_scale, next_w_tensor_scale,
+                      reinterpret_cast<__nv_bfloat16*>(next_lowrank_act)) != cudaSuccess)
+            return cuda_fail("lowrank_finalize_kernel launch");
+        SVDQ_TRY(launch_status("lowrank_finalize_kernel launch"));
+    }
+    return SVDQ_OK;
+}
+
+svdq_status svdq_gelu(const void* x, void* y, int64_t n, int approx, svdq_stream_t stream) {
+    SVDQ_TRY(check_ptr(x));
+    SVDQ_TRY(check_ptr(y));
+    if (approx != 0 && approx != 1) return SVDQ_ERR_INVALID_ARG;
+    if (n < 1 || n >= (int64_t(1) << 40)) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+    SVDQ_TRY(check_device());
+    const int64_t n8 = n / 8;
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((n8 + 255) / 256, 8LL * num_sms()));
+    gelu_bf16_kernel<<<grid, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        reinterpret_cast<const __nv_bfloat16*>(x), reinterpret_cast<__nv_bfloat16*>(y), n, approx);
+    return launch_status("gelu_bf16_kernel launch");
 }
 
 svdq_status svdq_gemm_w4a16(const void* x, int64_t M, const void* w_codes, const void* w_scales, int64_t N,

@@ -239,6 +239,54 @@ svdq_status svdq_qkv_norm_rope(const void* y_in, void* y_out, int64_t M, int hea
                                const void* norm_q, const void* norm_k, float eps,
                                const float* rope_cos, const float* rope_sin, svdq_stream_t stream);
 
+/* The fused GELU MLP (the "fused GELU kernel" for the MLP of the original
+ * Nunchaku engine; the Diffusers docs page "Nunchaku Lite", section "Fused
+ * kernels", GELU-MLP row): the W4A4 GEMM of fc1 whose epilogue applies GELU
+ * and performs fc2's activation step itself, so that the [M, N]
+ * intermediate is never written:
+ *     y  = bf16(fc1 linear output)              (as svdq_gemm_w4a4 computes it)
+ *     h  = bf16(GELU(y))                         GELU: gelu_approx 0 = x Phi(x),
+ *                                                1 = 0.5 x (1 + tanh(sqrt(2/pi)(x + 0.044715 x^3)))
+ *     next_x_codes, next_x_scales = svdq_quantize_act's nvfp4 step on h with
+ *                                   fc2's 1/lambda and the static tensor scale S2
+ *     next_lowrank_act = (h / lambda2) L_down2 / (S2 S_w2) as a hi/lo bf16 pair
+ * after which svdq_gemm_w4a4 with fc2's packed weight and these three
+ * buffers (x_tensor_scale = next_x_tensor_scale) computes fc2.  nvfp4 only.
+ * Arguments up to bias are fc1's, as in svdq_gemm_w4a4 (N = fc2's K,
+ * N % 128 == 0).  fc2's side, from svdq_pack_weight of fc2 and the caller:
+ *   next_inv_lambda      device fp32 [N]  (pack output inv_lambda)
+ *   next_L_down_t        device bf16 [2, next_rank, N] (pack output L_down_t)
+ *   next_rank            0, 16 or 32
+ *   next_x_tensor_scale  device fp32 [1]: S2, fc2's static (calibrated) activation
+ *                        tensor scale; a dynamic scale needs all of h first
+ *   next_w_tensor_scale  device fp32 [1]: fc2's S_w (pack output w_tensor_scale)
+ *   next_x_codes, next_x_scales, next_lowrank_act   outputs, sized as
+ *                        svdq_buffer_sizes(NVFP4, M, N, next_rank) gives for
+ *                        svdq_quantize_act
+ *   workspace            device fp32 [M, next_rank] partial sums: zero-filled once
+ *                        by the caller; every successful call leaves it zeroed
+ *                        (NULL when next_rank == 0)
+ * Two kernels on `stream`: the GEMM, then (next_rank > 0) the finalisation of
+ * the rank-r sums.  Errors: as svdq_gemm_w4a4; INVALID_ARG for int4, a bad
+ * gelu_approx or rank, a short workspace; UNSUPPORTED_SHAPE when N % 128 != 0
+ * or next_rank > 32. */
+svdq_status svdq_gelu_mlp_workspace_bytes(int64_t M, int next_rank, size_t* bytes);
+svdq_status svdq_gemm_w4a4_gelu_quant(svdq_precision precision, int group_size,
+                                      const void* x_codes, const void* x_scales, const float* x_tensor_scale,
+                                      int64_t M, const void* w_codes, const void* w_scales,
+                                      const float* w_tensor_scale, int64_t N, int64_t K,
+                                      const void* lowrank_act, const void* L_up_t, int rank, const void* bias,
+                                      int gelu_approx, const float* next_inv_lambda, const void* next_L_down_t,
+                                      int next_rank, const float* next_x_tensor_scale,
+                                      const float* next_w_tensor_scale, void* next_x_codes, void* next_x_scales,
+                                      void* next_lowrank_act, void* workspace, size_t workspace_bytes,
+                                      svdq_stream_t stream);
+
+/* The unfused activation pass of the same MLP: y[i] = bf16(GELU(x[i])) over n
+ * bf16 elements (device pointers, 16-byte aligned; y may equal x).
+ * Errors: INVALID_ARG for a bad pointer or approx; UNSUPPORTED_SHAPE for n < 1. */
+svdq_status svdq_gelu(const void* x, void* y, int64_t n, int approx, svdq_stream_t stream);
+
 /* The weight-only int4 GEMM of the `awq_w4a16` scheme (the "INT4 weight-only
  * AWQ-style kernel", int4 with group 64, of the Diffusers docs page "Nunchaku
  * Lite", section "Supported quantization types"; its targets are listed in
