@@ -23,18 +23,60 @@ namespace svdq {
 // GELU in fp32.  approx = 0: x Phi(x) = 0.5 x erfc(-x / sqrt(2)) (erfc keeps
 // the relative accuracy of the tail for negative x); approx = 1: the tanh
 // form 0.5 x (1 + tanh(u)), u = sqrt(2/pi)(x + 0.044715 x^3), evaluated as
-// x / (1 + exp(-2u)), the same function without the cancellation of
-// 1 + tanh(u) for negative u.
+// x / (1 + e^(-2u)) for u >= 0 and x e^(2u) / (1 + e^(2u)) for u < 0: the
+// same function without the cancellation of 1 + tanh(u) and without an
+// exponential that overflows while the result is still a bf16 subnormal.
 __device__ __forceinline__ float gelu_f32(float x, int approx) {
     if (approx == 0) return 0.5f * x * erfcf(-x * 0.70710678118654752f);
     const float u = 0.79788456080286536f * fmaf(0.044715f * x, x * x, x);
-    return x / (1.0f + expf(-2.0f * u));
+    const float e = expf(-2.0f * fabsf(u));   // in [0, 1]
+    return u >= 0.0f ? x / (1.0f + e) : x * e / (1.0f + e);
+}
+
+// bf16 -> bf16 GELU as both the fused epilogue and the unfused pass compute
+// it, so that the two hand fc2 the same h bit for bit.  The input has only
+// 65536 values, and for most of them the result is a table entry:
+//  * |x| in [2^-10, 16) (biased exponent 117 .. 130, both signs): a table of
+//    bf16(gelu_f32(x)), 3584 entries (7 KB) built once per CTA;
+//  * |x| < 2^-10: GELU(x) = x/2 + x^2/sqrt(2 pi) + O(x^4) (both forms), and
+//    the x^2 term is below a quarter of a bf16 ulp of x/2, so the result is
+//    bf16(x / 2) (computed in fp32: exact, then rounded to bf16);
+//  * |x| >= 16: Phi(x) rounds to 1 (x > 0: the result is x) or x Phi(x)
+//    underflows fp32 (x < 0: -0), for both forms, as gelu_f32 gives them.
+constexpr int kGeluTabE0 = 117;                     // biased exponent of 2^-10
+constexpr int kGeluTabNE = 14;                      // exponents 117 .. 130
+constexpr int kGeluTabEntries = 2 * kGeluTabNE * 128;
+constexpr int kGeluTabBytes = kGeluTabEntries * 2;
+
+// Fills the table (threads tid, tid + nthreads, ...); the caller syncs.
+__device__ __forceinline__ void gelu_table_fill(uint16_t* tab, int tid, int nthreads, int approx) {
+    for (int i = tid; i < kGeluTabEntries; i += nthreads) {
+        const uint32_t sign = (uint32_t)(i / (kGeluTabNE * 128));
+        const uint32_t e = (uint32_t)kGeluTabE0 + (uint32_t)((i / 128) % kGeluTabNE);
+        const uint32_t bits = (sign << 15) | (e << 7) | (uint32_t)(i & 127);
+        tab[i] = __bfloat16_as_ushort(__float2bfloat16_rn(gelu_f32(__uint_as_float(bits << 16), approx)));
+    }
+}
+
+// GELU of one bf16 (bits in the low 16 of b) -> bf16 bits.  The table holds
+// the magnitudes 117 * 128 .. 131 * 128 - 1 (exponent and mantissa bits) of
+// the positive values, then the same of the negative ones.
+__device__ __forceinline__ uint32_t gelu_bf16_bits(uint32_t b, const uint16_t* tab) {
+    constexpr uint32_t kSpan = (uint32_t)kGeluTabNE << 7;
+    const uint32_t off = (b & 0x7FFFu) - ((uint32_t)kGeluTabE0 << 7);   // wraps below the table
+    if (off < kSpan) return tab[off + ((b & 0x8000u) ? kSpan : 0u)];
+    if (((b >> 7) & 0xFFu) < (uint32_t)kGeluTabE0)
+        return __bfloat16_as_ushort(__float2bfloat16_rn(0.5f * __uint_as_float(b << 16)));
+    return (b & 0x8000u) ? 0x8000u : b;
 }
 
 // The unfused activation pass: y[i] = bf16(GELU(x[i])) over n elements
 // (eight per thread per step, grid-stride).
 __global__ void __launch_bounds__(256) gelu_bf16_kernel(const __nv_bfloat16* __restrict__ x,
                                                         __nv_bfloat16* __restrict__ y, int64_t n, int approx) {
+    __shared__ uint16_t tab[kGeluTabEntries];
+    gelu_table_fill(tab, (int)threadIdx.x, (int)blockDim.x, approx);
+    __syncthreads();
     const int64_t n8 = n / 8;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8; i += stride) {
@@ -42,16 +84,13 @@ __global__ void __launch_bounds__(256) gelu_bf16_kernel(const __nv_bfloat16* __r
         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
         uint32_t o[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const __nv_bfloat162 h =
-                __floats2bfloat162_rn(gelu_f32(bf16lo_to_f32(w[e]), approx), gelu_f32(bf16hi_to_f32(w[e]), approx));
-            o[e] = *reinterpret_cast<const uint32_t*>(&h);
-        }
+        for (int e = 0; e < 4; ++e)
+            o[e] = gelu_bf16_bits(w[e] & 0xFFFFu, tab) | (gelu_bf16_bits(w[e] >> 16, tab) << 16);
         reinterpret_cast<uint4*>(y)[i] = make_uint4(o[0], o[1], o[2], o[3]);
     }
     if (blockIdx.x == 0 && threadIdx.x < (unsigned)(n - 8 * n8)) {
         const int64_t i = 8 * n8 + threadIdx.x;
-        y[i] = __float2bfloat16_rn(gelu_f32(__bfloat162float(x[i]), approx));
+        y[i] = __ushort_as_bfloat16((uint16_t)gelu_bf16_bits(__bfloat16_as_ushort(x[i]), tab));
     }
 }
 

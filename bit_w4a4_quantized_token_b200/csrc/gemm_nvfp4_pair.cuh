@@ -88,18 +88,30 @@ constexpr uint32_t SFB_RES = SFA_RES + 4 * kResidentKSteps;   // 448: two sets o
 static_assert(SFB_RES + 64 <= TMEM_COLS, "resident scale-factor columns do not fit in TMEM");
 constexpr uint32_t kFullArrivals = 3;          // CTA 0's three producer roles, for both CTAs' bytes
 constexpr int kLanesPerRole = 2;               // producer lanes per role, taking alternate stages
-constexpr uint32_t kAccEmptyArrivals = 2 * kEpiWarps;
 constexpr size_t SMEM_BYTES = 1024 + (size_t)kStages * STAGE_BYTES + 256;
 static_assert(SMEM_BYTES <= 227 * 1024, "stage ring does not fit in shared memory");
-// kEpiGelu: a 2 KB transpose buffer per epilogue warp (32 rows x 32 bf16)
-constexpr int kGeluScratch = 2048;
-constexpr size_t SMEM_BYTES_GELU = SMEM_BYTES + (size_t)kEpiWarps * kGeluScratch;
+// kEpiGelu: twice the epilogue warps (four per TMEM lane quadrant, 64
+// columns each: the GELU epilogue is latency-bound, and more warps hide more
+// of it), a 1 KB transpose buffer per warp (32 rows x 16 bf16), the GELU
+// table and the 128 reciprocals of the next layer's decoded group scales.
+constexpr int kEpiWarpsGelu = 16;
+constexpr int kThreadsGelu = 32 * (kEpiWarp0 + kEpiWarpsGelu);
+constexpr int kGeluScratch = 1024;
+constexpr size_t SMEM_BYTES_GELU = SMEM_BYTES + (size_t)kEpiWarpsGelu * kGeluScratch + kGeluTabBytes + 128 * 4;
 static_assert(SMEM_BYTES_GELU <= 227 * 1024, "GELU epilogue buffers do not fit in shared memory");
 }  // namespace gp
 
 // Epilogue variants of the pair kernel (separate instantiations, so that the
 // plain kernel keeps its registers).
 enum : int { kEpiPlain = 0, kEpiQkv = 1, kEpiGelu = 2 };
+template <int kEpi>
+__host__ __device__ constexpr int gp_epi_warps() {
+    return kEpi == kEpiGelu ? gp::kEpiWarpsGelu : gp::kEpiWarps;
+}
+template <int kEpi>
+__host__ __device__ constexpr int gp_threads() {
+    return 32 * (gp::kEpiWarp0 + gp_epi_warps<kEpi>());
+}
 
 enum : uint32_t {
     kSiteGpEmpty = 24,
@@ -132,32 +144,35 @@ __device__ __forceinline__ void gp_issue_stage(uint32_t acc, uint64_t da, uint64
     }
 }
 
-// The fused GELU epilogue of one thread's row (grow) over one warp's 128
-// columns [nbase, nbase + 128) of a tile; acc holds the fp32 accumulators.
+// The fused GELU epilogue of one thread's row (grow) over one warp's NC
+// columns [nbase, nbase + NC) of a tile; acc holds the fp32 accumulators.
 //  1. y = S acc + b rounded to bf16 (what the plain epilogue stores), then
-//     h = bf16(GELU(y)): the next layer's input, never written out;
+//     h = bf16(GELU(y)) by gelu_bf16_bits (the per-CTA table): the next
+//     layer's input, never written out;
 //  2. the next layer's nvfp4 step on h, with the arithmetic of the activation
 //     quantizer (quantize_act.cuh): v = h * (1 / lambda), per 16 columns the
-//     E4M3 scale of amax(v) / (6 S2) and the E2M1 codes of v / (scale S2);
-//     codes go to row grow of nx_codes, scales to the tensor-core layout
-//     (rows between M and the 128-row padding get scale 0, as the quantizer
-//     writes them);
-//  3. the next layer's rank-r down-projection over these 128 columns,
-//     h [32 rows x 128] (L_down / lambda) [128 x r], on the warp's tensor
+//     E4M3 scale e of amax(v) / (6 S2) and the E2M1 codes of v * inv_tab[e],
+//     inv_tab[e] = 1 / (e S2); codes go to row grow of nx_codes, scales to
+//     the tensor-core layout (rows between M and the 128-row padding get
+//     scale 0, as the quantizer writes them);
+//  3. the next layer's rank-r down-projection over these NC columns,
+//     h [32 rows x NC] (L_down / lambda) [NC x r], on the warp's tensor
 //     cores (m16n8k16 bf16 MMAs; h is exact in bf16, L_down / lambda enters
 //     as its hi and lo bf16 planes), added into nx_acc with fp32 atomics.
 // Every lane takes part in step 3 (warp-wide MMAs), whatever its row.
-__device__ __forceinline__ void gp_gelu_epilogue(const uint32_t (&acc)[128], const GemmArgs& a, float S, float S2,
-                                                 float six_s2, int64_t grow, int nbase, uint32_t scr,
-                                                 uint32_t lane) {
+template <int NC>
+__device__ __forceinline__ void gp_gelu_epilogue(const uint32_t (&acc)[NC], const GemmArgs& a, float S,
+                                                 float six_s2, const float* inv_tab, int64_t grow, int nbase,
+                                                 uint32_t scr, const uint16_t* gelu_tab, uint32_t lane) {
+    static_assert(NC % 64 == 0, "a warp covers whole groups of four scale bytes");
     const bool row_ok = grow < a.M;
     const int64_t half_k = (int64_t)a.N / 2;
     const int64_t kg4n = a.N / 64;
-    uint32_t hpk[64];
+    uint32_t hpk[NC / 2];
     uint32_t cw[4] = {0u, 0u, 0u, 0u};
     uint32_t sword = 0u;
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
+    for (int c = 0; c < NC / 16; ++c) {
         const int n = nbase + 16 * c;
         uint32_t bw[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
         if (a.bias) {
@@ -172,11 +187,11 @@ __device__ __forceinline__ void gp_gelu_epilogue(const uint32_t (&acc)[128], con
             const float o0 = fmaf(__uint_as_float(acc[16 * c + 2 * p]), S, bf16lo_to_f32(bw[p]));
             const float o1 = fmaf(__uint_as_float(acc[16 * c + 2 * p + 1]), S, bf16hi_to_f32(bw[p]));
             const __nv_bfloat162 y2 = __floats2bfloat162_rn(o0, o1);
-            const __nv_bfloat162 h2 = __floats2bfloat162_rn(gelu_f32(__low2float(y2), a.gelu_approx),
-                                                            gelu_f32(__high2float(y2), a.gelu_approx));
-            hpk[8 * c + p] = *reinterpret_cast<const uint32_t*>(&h2);
-            h[2 * p] = __low2float(h2);
-            h[2 * p + 1] = __high2float(h2);
+            const uint32_t yb = *reinterpret_cast<const uint32_t*>(&y2);
+            const uint32_t hb = gelu_bf16_bits(yb & 0xFFFFu, gelu_tab) | (gelu_bf16_bits(yb >> 16, gelu_tab) << 16);
+            hpk[8 * c + p] = hb;
+            h[2 * p] = __uint_as_float(hb << 16);
+            h[2 * p + 1] = __uint_as_float(hb & 0xFFFF0000u);
         }
         const float4* il = reinterpret_cast<const float4*>(a.nx_inv_lambda + n);
         float v[16];
@@ -186,10 +201,21 @@ __device__ __forceinline__ void gp_gelu_epilogue(const uint32_t (&acc)[128], con
             fmul2_rn(h[4 * q], h[4 * q + 1], l.x, l.y, v[4 * q], v[4 * q + 1]);
             fmul2_rn(h[4 * q + 2], h[4 * q + 3], l.z, l.w, v[4 * q + 2], v[4 * q + 3]);
         }
-        uint32_t lo, hi;
-        const uint32_t eb = quant_group16(v, S2, six_s2, lo, hi);
-        cw[2 * (c & 1)] = lo;
-        cw[2 * (c & 1) + 1] = hi;
+        float m0 = fmaxf(fabsf(v[0]), fabsf(v[1])), m1 = fmaxf(fabsf(v[2]), fabsf(v[3]));
+#pragma unroll
+        for (int i = 4; i < 16; i += 4) {
+            m0 = fmaxf(m0, fmaxf(fabsf(v[i]), fabsf(v[i + 1])));
+            m1 = fmaxf(m1, fmaxf(fabsf(v[i + 2]), fabsf(v[i + 3])));
+        }
+        const uint32_t eb = cvt_e4m3(__fdiv_rn(fmaxf(m0, m1), six_s2));
+        const float inv = inv_tab[eb];
+        float qv[8];
+#pragma unroll
+        for (int i = 0; i < 8; i += 2) fmul2_rn(v[i], v[i + 1], inv, inv, qv[i], qv[i + 1]);
+        cw[2 * (c & 1)] = cvt_e2m1x8(qv);
+#pragma unroll
+        for (int i = 0; i < 8; i += 2) fmul2_rn(v[8 + i], v[9 + i], inv, inv, qv[i], qv[i + 1]);
+        cw[2 * (c & 1) + 1] = cvt_e2m1x8(qv);
         sword |= eb << (8 * (c & 3));
         if (c & 1) {
             if (row_ok)
@@ -204,7 +230,7 @@ __device__ __forceinline__ void gp_gelu_epilogue(const uint32_t (&acc)[128], con
         }
     }
     if (a.nx_rank == 0) return;
-    // ---- rank-r down-projection of the next layer over these 128 columns
+    // ---- rank-r down-projection of the next layer over these NC columns
     const int g = (int)(lane >> 2), t = (int)(lane & 3);
     const int nj = a.nx_rank / 8;                     // 2 or 4 column blocks of 8
     const int64_t plane = (int64_t)a.nx_rank * a.N;   // hi plane, then lo plane
@@ -215,40 +241,47 @@ __device__ __forceinline__ void gp_gelu_epilogue(const uint32_t (&acc)[128], con
         for (int j = 0; j < 4; ++j)
 #pragma unroll
             for (int e = 0; e < 4; ++e) lacc[mt][j][e] = 0.0f;
-    const uint32_t my_row = scr + 64u * lane;
+    const uint32_t my_row = scr + 32u * lane;
 #pragma unroll
-    for (int kc = 0; kc < 4; ++kc) {
-        // this lane's row, columns 32 kc .. 32 kc + 31, in four 16-byte pieces
-        // placed at piece ^ ((row / 2) % 4) so that neither these stores nor
-        // the ldmatrix reads below meet a bank twice
+    for (int kb = 0; kb < NC / 16; ++kb) {
+        // Within a block of 16 K values the MMA's K slots are taken in the
+        // order 0 1 4 5 8 9 12 13 | 2 3 6 7 10 11 14 15 (the same permutation
+        // for A and B leaves the product unchanged): a lane's two B registers
+        // then hold four consecutive K values, one 8-byte load per plane,
+        // issued ahead of the transposition so that their latency overlaps it.
+        uint2 bf[4][2];
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch)
-            st_shared_v4(my_row + ((uint32_t)(ch ^ ((lane >> 1) & 3)) << 4), hpk[16 * kc + 4 * ch],
-                         hpk[16 * kc + 4 * ch + 1], hpk[16 * kc + 4 * ch + 2], hpk[16 * kc + 4 * ch + 3]);
-        __syncwarp();
-#pragma unroll
-        for (int ks = 0; ks < 2; ++ks) {
-            uint32_t af[2][4];
-#pragma unroll
-            for (int mt = 0; mt < 2; ++mt) {
-                const uint32_t rr = 16u * mt + ((lane >> 3) & 1u) * 8u + (lane & 7u);
-                const uint32_t kch = 2u * ks + (lane >> 4);
-                ldmatrix_x4(af[mt], scr + 64u * rr + ((kch ^ ((rr >> 1) & 3u)) << 4));
+        for (int j = 0; j < 4; ++j) {
+            bf[j][0] = bf[j][1] = make_uint2(0u, 0u);
+            if (j < nj) {
+                const __nv_bfloat16* bp = a.nx_ldt + (int64_t)(8 * j + g) * a.N + (nbase + 16 * kb + 4 * t);
+                bf[j][0] = __ldg(reinterpret_cast<const uint2*>(bp));
+                bf[j][1] = __ldg(reinterpret_cast<const uint2*>(bp + plane));
             }
-            const int64_t k = nbase + 32 * kc + 16 * ks + 2 * t;
+        }
+        // this lane's row of the block: pairs (0 1)(4 5)(8 9)(12 13), then
+        // (2 3)(6 7)(10 11)(14 15), as two 16-byte pieces placed at
+        // piece ^ ((row / 4) % 2) so that neither these stores nor the
+        // ldmatrix reads below meet a bank twice
+        const uint32_t sw = (lane >> 2) & 1u;
+        st_shared_v4(my_row + (sw << 4), hpk[8 * kb], hpk[8 * kb + 2], hpk[8 * kb + 4], hpk[8 * kb + 6]);
+        st_shared_v4(my_row + ((sw ^ 1u) << 4), hpk[8 * kb + 1], hpk[8 * kb + 3], hpk[8 * kb + 5],
+                     hpk[8 * kb + 7]);
+        __syncwarp();
+        uint32_t af[2][4];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                if (j < nj) {
-                    const __nv_bfloat16* bp = a.nx_ldt + (int64_t)(8 * j + g) * a.N + k;
-                    const uint32_t bh0 = __ldg(reinterpret_cast<const unsigned int*>(bp));
-                    const uint32_t bh1 = __ldg(reinterpret_cast<const unsigned int*>(bp + 8));
-                    const uint32_t bl0 = __ldg(reinterpret_cast<const unsigned int*>(bp + plane));
-                    const uint32_t bl1 = __ldg(reinterpret_cast<const unsigned int*>(bp + plane + 8));
+        for (int mt = 0; mt < 2; ++mt) {
+            const uint32_t rr = 16u * mt + ((lane >> 3) & 1u) * 8u + (lane & 7u);
+            const uint32_t kch = lane >> 4;
+            ldmatrix_x4(af[mt], scr + 32u * rr + ((kch ^ ((rr >> 2) & 1u)) << 4));
+        }
 #pragma unroll
-                    for (int mt = 0; mt < 2; ++mt) {
-                        mma_16816_bf16(lacc[mt][j], af[mt], bh0, bh1);
-                        mma_16816_bf16(lacc[mt][j], af[mt], bl0, bl1);
-                    }
+        for (int j = 0; j < 4; ++j) {
+            if (j < nj) {
+#pragma unroll
+                for (int mt = 0; mt < 2; ++mt) {
+                    mma_16816_bf16(lacc[mt][j], af[mt], bf[j][0].x, bf[j][0].y);
+                    mma_16816_bf16(lacc[mt][j], af[mt], bf[j][1].x, bf[j][1].y);
                 }
             }
         }
@@ -275,7 +308,7 @@ __device__ __forceinline__ void gp_gelu_epilogue(const uint32_t (&acc)[128], con
 // kEpi: kEpiPlain, kEpiQkv (the fused QKV + RMSNorm + RoPE epilogue) or
 // kEpiGelu (the fused GELU + next-layer activation epilogue).
 template <int kEpi>
-__global__ void __launch_bounds__(gp::kThreads, 1)
+__global__ void __launch_bounds__(gp_threads<kEpi>(), 1)
     gemm_nvfp4_pair_kernel(const __grid_constant__ CUtensorMap tm_xc, const __grid_constant__ CUtensorMap tm_wc,
                            const __grid_constant__ CUtensorMap tm_sfa, const __grid_constant__ CUtensorMap tm_sfb,
                            const __grid_constant__ CUtensorMap tm_L, const __grid_constant__ CUtensorMap tm_Lup,
@@ -310,7 +343,7 @@ __global__ void __launch_bounds__(gp::kThreads, 1)
             mbar_init(&empty[s], 1);
         }
         mbar_init(acc_full, 1);
-        mbar_init(acc_empty, kAccEmptyArrivals);
+        mbar_init(acc_empty, 2u * (uint32_t)gp_epi_warps<kEpi>());   // both CTAs' epilogue warps
         for (int s = 0; s < kStages; ++s) s_issued[s] = 0;
         s_failed = 0;
         fence_barrier_init();
@@ -329,6 +362,10 @@ __global__ void __launch_bounds__(gp::kThreads, 1)
         tmem_alloc_pair(tmem_slot, TMEM_COLS);
         tmem_relinquish_pair();
     }
+    if (kEpi == kEpiGelu)     // the bf16 GELU table (gelu_mlp.cuh), once per CTA
+        gelu_table_fill(reinterpret_cast<uint16_t*>(smem + (size_t)kStages * STAGE_BYTES + 256 +
+                                                    (size_t)kEpiWarpsGelu * kGeluScratch),
+                        (int)threadIdx.x, gp_threads<kEpi>(), a.gelu_approx);
     tc_fence_before();
     cluster_sync_all();       // barriers of both CTAs initialised, TMEM address written
     tc_fence_after();
@@ -484,12 +521,24 @@ __global__ void __launch_bounds__(gp::kThreads, 1)
         const int row = (int)(32u * q + lane);
         const float S = __fmul_rn(*a.x_scale, *a.w_scale);
         const uint32_t acc_empty_leader = cluster_addr(acc_empty, 0);
-        float gelu_s2 = 1.0f, gelu_six_s2 = 6.0f;
+        float gelu_six_s2 = 6.0f;
         uint32_t gelu_scr = 0u;
+        uint8_t* gelu_base = smem + (size_t)kStages * STAGE_BYTES + 256;
+        const uint16_t* gelu_tab =
+            reinterpret_cast<const uint16_t*>(gelu_base + (size_t)kEpiWarpsGelu * kGeluScratch);
+        float* gelu_inv = reinterpret_cast<float*>(gelu_base + (size_t)kEpiWarpsGelu * kGeluScratch + kGeluTabBytes);
         if (kEpi == kEpiGelu) {
-            gelu_s2 = *a.nx_x_scale;
-            gelu_six_s2 = __fmul_rn(6.0f, gelu_s2);
-            gelu_scr = smem_u32(smem + (size_t)kStages * STAGE_BYTES + 256);
+            const float S2 = *a.nx_x_scale;
+            gelu_six_s2 = __fmul_rn(6.0f, S2);
+            gelu_scr = smem_u32(gelu_base);
+            // reciprocals of the 128 decoded group scales e * S2, as the
+            // activation quantizer tabulates them
+            const int t = (int)threadIdx.x - 32 * kEpiWarp0;
+            if (t < 128) {
+                const float dec = __fmul_rn(e4m3_to_f32((uint32_t)t), S2);
+                gelu_inv[t] = (dec == 0.0f) ? 0.0f : __frcp_rn(dec);
+            }
+            named_bar_sync(1, 32 * kEpiWarpsGelu);
         }
         int local = 0;
         for (int tile = t_begin; tile < t_end; ++tile, ++local) {
@@ -501,6 +550,26 @@ __global__ void __launch_bounds__(gp::kThreads, 1)
                 break;
             }
             tc_fence_after();
+            if (kEpi == kEpiGelu) {
+                // four warps per lane quadrant: this warp's 64 columns
+                const int part = (int)(warp - kEpiWarp0) >> 2;
+                const int gbase = n_tile * BN + 64 * part;
+                uint32_t acc[64];
+                tmem_ld_32x32b_x32(tmem + ((32u * q) << 16) + ACC_COL + 64u * part + 0u,
+                                   *reinterpret_cast<uint32_t(*)[32]>(acc + 0));
+                tmem_ld_32x32b_x32(tmem + ((32u * q) << 16) + ACC_COL + 64u * part + 32u,
+                                   *reinterpret_cast<uint32_t(*)[32]>(acc + 32));
+                tmem_ld_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
+                // warp-uniform: with N % 128 == 0 a warp's columns are all in or all out
+                if (gbase < a.N)
+                    gp_gelu_epilogue<64>(acc, a, S, gelu_six_s2, gelu_inv, grow, gbase,
+                                         gelu_scr + (uint32_t)(warp - kEpiWarp0) * (uint32_t)kGeluScratch,
+                                         gelu_tab, lane);
+                continue;
+            }
             uint32_t acc[128];
             tmem_ld_32x32b_x32(tmem + ((32u * q) << 16) + ACC_COL + 128u * half + 0u,
                                *reinterpret_cast<uint32_t(*)[32]>(acc + 0));
@@ -514,13 +583,6 @@ __global__ void __launch_bounds__(gp::kThreads, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(acc_empty_leader);   // this half of the pair is drained
-            if (kEpi == kEpiGelu) {
-                // warp-uniform: with N % 128 == 0 a warp's columns are all in or all out
-                if (nbase < a.N)
-                    gp_gelu_epilogue(acc, a, S, gelu_s2, gelu_six_s2, grow, nbase,
-                                     gelu_scr + (uint32_t)(warp - kEpiWarp0) * (uint32_t)kGeluScratch, lane);
-                continue;
-            }
             if (grow >= a.M) continue;
             __nv_bfloat16* yrow = a.y + grow * (int64_t)a.N;
             if (kEpi == kEpiQkv && nbase < a.qk_cols) {

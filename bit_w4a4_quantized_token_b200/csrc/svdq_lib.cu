@@ -622,8 +622,8 @@ svdq_status gemm_nvfp4_pair(const void* x_codes, const void* x_scales, const flo
     const dim3 grid(2 * (unsigned)clusters), block(gp::kThreads);
     cudaError_t e;
     if (gelu.next_x_scale)
-        e = launch_ex(gemm_nvfp4_pair_kernel<kEpiGelu>, grid, block, gp::SMEM_BYTES_GELU, st, 2u, tm_xc, tm_wc,
-                      tm_sfa, tm_sfb, tm_L, tm_Lup, a);
+        e = launch_ex(gemm_nvfp4_pair_kernel<kEpiGelu>, grid, dim3(gp::kThreadsGelu), gp::SMEM_BYTES_GELU, st, 2u,
+                      tm_xc, tm_wc, tm_sfa, tm_sfb, tm_L, tm_Lup, a);
     else if (qkv.heads > 0)
         e = launch_ex(gemm_nvfp4_pair_kernel<kEpiQkv>, grid, block, gp::SMEM_BYTES, st, 2u, tm_xc, tm_wc, tm_sfa,
                       tm_sfb, tm_L, tm_Lup, a);

@@ -283,7 +283,9 @@ svdq_status svdq_gemm_w4a4_gelu_quant(svdq_precision precision, int group_size,
                                       svdq_stream_t stream);
 
 /* The unfused activation pass of the same MLP: y[i] = bf16(GELU(x[i])) over n
- * bf16 elements (device pointers, 16-byte aligned; y may equal x).
+ * finite bf16 elements (device pointers, 16-byte aligned; y may equal x);
+ * the same bf16 -> bf16 function the fused epilogue applies, so both paths
+ * give fc2 the same h.
  * Errors: INVALID_ARG for a bad pointer or approx; UNSUPPORTED_SHAPE for n < 1. */
 svdq_status svdq_gelu(const void* x, void* y, int64_t n, int approx, svdq_stream_t stream);
 
