@@ -17,7 +17,11 @@
 //   * every load of either CTA completes on CTA 0's stage barrier, CTA 0's
 //     commits arrive on both CTAs' "stage free" and "accumulator full"
 //     barriers, and both CTAs' epilogue warps hand the accumulator back on
-//     CTA 0's barrier.
+//     CTA 0's barrier;
+//   * a fourth warp of CTA 0 waits on the stage and accumulator barriers and
+//     meets the MMA warp at named barriers, so that the thread issuing the
+//     copies never touches shared memory while they are in flight (3-5 %
+//     faster than testing the mbarriers itself).
 // Against 128 x 256 tiles on single CTAs this halves the weight-code bytes
 // each SM loads per FLOP and the number of scale-block copies per FLOP; with
 // the activation scales resident in TMEM (K <= 3072, below) two copies per
@@ -68,6 +72,10 @@ constexpr int kEpiWarps = 8;
 constexpr int kEpiWarp0 = 4;
 constexpr int kThreads = 32 * (kEpiWarp0 + kEpiWarps);
 constexpr uint32_t kMmaWarp = 2;
+constexpr uint32_t kWaitWarp = 3;              // waits on the mbarriers for the MMA warp
+constexpr uint32_t kBarStage0 = 2;             // named barriers 2 .. 2 + kStages - 1: stage s ready
+constexpr uint32_t kBarAcc = 7;                // named barrier: accumulator free
+static_assert(kBarStage0 + kStages <= kBarAcc, "named barriers overlap");   // 0: __syncthreads, 1: GELU epilogue
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COL = 0;
 // Scale factors in TMEM.  Stages alternate between two "scale sets"; one of
@@ -90,6 +98,13 @@ constexpr uint32_t kFullArrivals = 3;          // CTA 0's three producer roles, 
 constexpr int kLanesPerRole = 2;               // producer lanes per role, taking alternate stages
 constexpr size_t SMEM_BYTES = 1024 + (size_t)kStages * STAGE_BYTES + 256;
 static_assert(SMEM_BYTES <= 227 * 1024, "stage ring does not fit in shared memory");
+// kEpiPlain: y leaves through TMA stores of 32 x 32 boxes staged per
+// epilogue warp in two 2 KB buffers (64-byte swizzle), 1 KB aligned after
+// the barriers.
+constexpr int kYStageBytes = 2048;
+constexpr size_t Y_STAGE_OFF = (size_t)kStages * STAGE_BYTES + 1024;
+constexpr size_t SMEM_BYTES_PLAIN = 1024 + Y_STAGE_OFF + (size_t)kEpiWarps * 2 * kYStageBytes;
+static_assert(SMEM_BYTES_PLAIN <= 227 * 1024, "y staging buffers do not fit in shared memory");
 // kEpiGelu: twice the epilogue warps (four per TMEM lane quadrant, 64
 // columns each: the GELU epilogue is latency-bound, and more warps hide more
 // of it), a 1 KB transpose buffer per warp (32 rows x 16 bf16), the GELU
@@ -104,6 +119,11 @@ static_assert(SMEM_BYTES_GELU <= 227 * 1024, "GELU epilogue buffers do not fit i
 // Epilogue variants of the pair kernel (separate instantiations, so that the
 // plain kernel keeps its registers).
 enum : int { kEpiPlain = 0, kEpiQkv = 1, kEpiGelu = 2 };
+// The GELU epilogue runs four warps per TMEM lane quadrant (64 columns
+// each): its chain is latency-bound, and more warps hide more of it.  The
+// plain and QKV epilogues keep two (128 columns per warp; a QKV head's
+// RMSNorm needs all of its 128 columns in one thread); four measured no
+// faster for the plain one.
 template <int kEpi>
 __host__ __device__ constexpr int gp_epi_warps() {
     return kEpi == kEpiGelu ? gp::kEpiWarpsGelu : gp::kEpiWarps;
@@ -305,6 +325,49 @@ __device__ __forceinline__ void gp_gelu_epilogue(const uint32_t (&acc)[NC], cons
         }
 }
 
+// The plain epilogue of one thread's row over NC columns from nbase:
+// y = bf16(S acc + b), 16-byte stores.
+template <int NC>
+__device__ __forceinline__ void gp_store_plain(const uint32_t (&acc)[NC], const GemmArgs& a, float S,
+                                               __nv_bfloat16* yrow, int nbase) {
+#pragma unroll
+    for (int c = 0; c < NC / 16; ++c) {
+        const int n = nbase + 16 * c;
+        if (n >= a.N) break;   // N % 16 == 0
+        uint32_t bw[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+        if (a.bias) {
+            const uint4 w0 = __ldg(reinterpret_cast<const uint4*>(a.bias + n));
+            const uint4 w1 = __ldg(reinterpret_cast<const uint4*>(a.bias + n) + 1);
+            bw[0] = w0.x, bw[1] = w0.y, bw[2] = w0.z, bw[3] = w0.w;
+            bw[4] = w1.x, bw[5] = w1.y, bw[6] = w1.z, bw[7] = w1.w;
+        }
+        uint32_t packed[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float o0 = fmaf(__uint_as_float(acc[16 * c + 2 * i]), S, bf16lo_to_f32(bw[i]));
+            const float o1 = fmaf(__uint_as_float(acc[16 * c + 2 * i + 1]), S, bf16hi_to_f32(bw[i]));
+            const __nv_bfloat162 h = __floats2bfloat162_rn(o0, o1);
+            packed[i] = *reinterpret_cast<const uint32_t*>(&h);
+        }
+        uint4* dst = reinterpret_cast<uint4*>(yrow + n);
+        dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+        dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+    }
+}
+
+// The MMA warp and the barrier-waiting warp meet at named barrier `id` (64
+// threads); returns the OR of their flags (the waiter's "gave up").
+__device__ __forceinline__ bool gp_meet(uint32_t id, uint32_t flag) {
+    uint32_t out;
+    asm volatile(
+        "{\n\t.reg .pred q, p;\n\tsetp.ne.u32 q, %1, 0;\n\tbar.red.or.pred p, %2, 64, q;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(out)
+        : "r"(flag), "r"(id)
+        : "memory");
+    return out != 0;
+}
+
 // kEpi: kEpiPlain, kEpiQkv (the fused QKV + RMSNorm + RoPE epilogue) or
 // kEpiGelu (the fused GELU + next-layer activation epilogue).
 template <int kEpi>
@@ -312,7 +375,7 @@ __global__ void __launch_bounds__(gp_threads<kEpi>(), 1)
     gemm_nvfp4_pair_kernel(const __grid_constant__ CUtensorMap tm_xc, const __grid_constant__ CUtensorMap tm_wc,
                            const __grid_constant__ CUtensorMap tm_sfa, const __grid_constant__ CUtensorMap tm_sfb,
                            const __grid_constant__ CUtensorMap tm_L, const __grid_constant__ CUtensorMap tm_Lup,
-                           GemmArgs a) {
+                           const __grid_constant__ CUtensorMap tm_y, GemmArgs a) {
     using namespace gp;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -437,7 +500,12 @@ __global__ void __launch_bounds__(gp_threads<kEpi>(), 1)
         }
     } else if (warp == kMmaWarp) {
         // ------------------------------------------ copies + MMAs (CTA 0 only)
-        if (rank == 0 && lane == 0) {
+        // The whole warp walks the stages and meets the waiting warp at a
+        // named barrier per stage; lane 0 issues the copies and MMAs.  The
+        // issuing thread never tests an mbarrier itself: a shared-memory
+        // access by a thread with scale-block copies in flight waits for
+        // them, which drained the tensor pipe at every stage.
+        if (rank == 0) {
             const uint32_t idesc_fp4 = idesc_m(idesc_nvfp4(BN), BM);
             const uint32_t idesc_lr = idesc_m(idesc_bf16_f32(BN), BM);
             const uint32_t smem0 = smem_u32(smem);
@@ -448,44 +516,46 @@ __global__ void __launch_bounds__(gp_threads<kEpi>(), 1)
             for (int tile = t_begin; tile < t_end && ok; ++tile, ++local) {
                 const int n_tile = tile % a.n_tiles;
                 const bool need_sfa = !sfa_res || tile == t_begin || n_tile == 0;
-                if (!mbar_wait(acc_empty, ((uint32_t)local & 1u) ^ 1u, kSiteGpAccEmpty)) {
+                if (gp_meet(kBarAcc, 0u)) {
                     s_failed = 1;
                     break;
                 }
-                tc_fence_after();
+                if (lane == 0) tc_fence_after();
                 // FP4 stages
                 for (int kk = 0; kk < n_kb; ++kk, ++it) {
-                    if (!mbar_wait(&full[s], ph, kSiteGpFull)) {
+                    if (gp_meet(kBarStage0 + (uint32_t)s, 0u)) {
                         ok = false;
                         s_failed = 1;
                         break;
                     }
-                    tc_fence_after();
-                    const uint32_t sa = smem0 + (uint32_t)s * STAGE_BYTES;
-                    const uint64_t da = desc_sw128(sa), db = desc_sw128(sa + A_BYTES);   // + 2 per 32-byte K-step
-                    const uint64_t dfa = desc_sf_block(sa + A_BYTES + B_BYTES);         // + 32 per 512 bytes
-                    const uint64_t dfb = dfa + (uint64_t)(SFA_BYTES >> 4);
-                    // activation-scale columns of this stage's K-steps, weight-scale set
-                    const uint32_t ta = sfa_res ? tmem + SFA_RES + 16u * (uint32_t)kk
-                                                : tmem + SF_COL + SF_SET_COLS * (uint32_t)(it & 1);
-                    const uint32_t tb = sfa_res ? tmem + SFB_RES + 32u * (uint32_t)(it & 1) : ta + 16u;
-                    const uint32_t acc0 = kk > 0 ? 1u : 0u;
-                    if (kk + 1 < n_kb || nks_last == 4) {
-                        if (need_sfa)
-                            gp_issue_stage<true>(tmem + ACC_COL, da, db, dfa, dfb, ta, tb, idesc_fp4, acc0);
-                        else
-                            gp_issue_stage<false>(tmem + ACC_COL, da, db, dfa, dfb, ta, tb, idesc_fp4, acc0);
-                    } else {
-                        // a last stage of fewer than four K-steps
-                        for (int j = 0; j < nks_last; ++j) {
-                            if (need_sfa) tmem_cp_32x128b_x4_pair(ta + 4u * j, dfa + 32u * j);
-                            tmem_cp_32x128b_x4_pair(tb + 8u * j, dfb + 32u * j);
-                            tmem_cp_32x128b_x4_pair(tb + 8u * j + 4u, dfb + 128u + 32u * j);
-                            mma_nvfp4_pair(tmem + ACC_COL, da + 2u * j, db + 2u * j, idesc_fp4, ta + 4u * j,
-                                           tb + 8u * j, (kk > 0 || j > 0) ? 1u : 0u);
+                    if (lane == 0) {
+                        tc_fence_after();
+                        const uint32_t sa = smem0 + (uint32_t)s * STAGE_BYTES;
+                        const uint64_t da = desc_sw128(sa), db = desc_sw128(sa + A_BYTES);   // + 2 per 32-byte K-step
+                        const uint64_t dfa = desc_sf_block(sa + A_BYTES + B_BYTES);         // + 32 per 512 bytes
+                        const uint64_t dfb = dfa + (uint64_t)(SFA_BYTES >> 4);
+                        // activation-scale columns of this stage's K-steps, weight-scale set
+                        const uint32_t ta = sfa_res ? tmem + SFA_RES + 16u * (uint32_t)kk
+                                                    : tmem + SF_COL + SF_SET_COLS * (uint32_t)(it & 1);
+                        const uint32_t tb = sfa_res ? tmem + SFB_RES + 32u * (uint32_t)(it & 1) : ta + 16u;
+                        const uint32_t acc0 = kk > 0 ? 1u : 0u;
+                        if (kk + 1 < n_kb || nks_last == 4) {
+                            if (need_sfa)
+                                gp_issue_stage<true>(tmem + ACC_COL, da, db, dfa, dfb, ta, tb, idesc_fp4, acc0);
+                            else
+                                gp_issue_stage<false>(tmem + ACC_COL, da, db, dfa, dfb, ta, tb, idesc_fp4, acc0);
+                        } else {
+                            // a last stage of fewer than four K-steps
+                            for (int j = 0; j < nks_last; ++j) {
+                                if (need_sfa) tmem_cp_32x128b_x4_pair(ta + 4u * j, dfa + 32u * j);
+                                tmem_cp_32x128b_x4_pair(tb + 8u * j, dfb + 32u * j);
+                                tmem_cp_32x128b_x4_pair(tb + 8u * j + 4u, dfb + 128u + 32u * j);
+                                mma_nvfp4_pair(tmem + ACC_COL, da + 2u * j, db + 2u * j, idesc_fp4, ta + 4u * j,
+                                               tb + 8u * j, (kk > 0 || j > 0) ? 1u : 0u);
+                            }
                         }
+                        tc_commit_pair(&empty[s], 0x3);
                     }
-                    tc_commit_pair(&empty[s], 0x3);
                     if (++s == kStages) {
                         s = 0;
                         ph ^= 1u;
@@ -493,25 +563,55 @@ __global__ void __launch_bounds__(gp_threads<kEpi>(), 1)
                 }
                 // rank-r stages: bf16 MMAs of the hi and lo parts into the same accumulator
                 for (int kk = n_kb; kk < per_tile && ok; ++kk, ++it) {
-                    if (!mbar_wait(&full[s], ph, kSiteGpFull)) {
+                    if (gp_meet(kBarStage0 + (uint32_t)s, 0u)) {
                         ok = false;
                         s_failed = 1;
                         break;
                     }
-                    tc_fence_after();
-                    const uint32_t sa = smem0 + (uint32_t)s * STAGE_BYTES;
-                    const uint64_t da = desc_sw128(sa), db = desc_sw128(sa + A_BYTES);
-                    const int c = (kk - n_kb) >> 1;
-                    const int nks = min(4, (a.rank - 64 * c + 15) / 16);
-                    for (int j = 0; j < nks; ++j)
-                        mma_bf16_pair(tmem + ACC_COL, da + 2u * j, db + 2u * j, idesc_lr, 1u);
-                    tc_commit_pair(&empty[s], 0x3);
+                    if (lane == 0) {
+                        tc_fence_after();
+                        const uint32_t sa = smem0 + (uint32_t)s * STAGE_BYTES;
+                        const uint64_t da = desc_sw128(sa), db = desc_sw128(sa + A_BYTES);
+                        const int c = (kk - n_kb) >> 1;
+                        const int nks = min(4, (a.rank - 64 * c + 15) / 16);
+                        for (int j = 0; j < nks; ++j)
+                            mma_bf16_pair(tmem + ACC_COL, da + 2u * j, db + 2u * j, idesc_lr, 1u);
+                        tc_commit_pair(&empty[s], 0x3);
+                    }
                     if (++s == kStages) {
                         s = 0;
                         ph ^= 1u;
                     }
                 }
-                if (ok) tc_commit_pair(acc_full, 0x3);
+                if (ok && lane == 0) tc_commit_pair(acc_full, 0x3);
+            }
+        }
+    } else if (warp == kWaitWarp) {
+        // ------------------------- barrier waiter for the MMA warp (CTA 0 only)
+        // The same walk over tiles and stages: wait on the accumulator and
+        // stage barriers, then meet the MMA warp (which goes on only then).
+        if (rank == 0) {
+            bool ok = true;
+            int local = 0, s = 0, it = 0;
+            uint32_t ph = 0;
+            for (int tile = t_begin; tile < t_end && ok; ++tile, ++local) {
+                bool f = !mbar_wait(acc_empty, ((uint32_t)local & 1u) ^ 1u, kSiteGpAccEmpty);
+                if (gp_meet(kBarAcc, f ? 1u : 0u)) {
+                    s_failed = 1;
+                    break;
+                }
+                for (int kk = 0; kk < per_tile; ++kk, ++it) {
+                    f = !mbar_wait(&full[s], ph, kSiteGpFull);
+                    if (gp_meet(kBarStage0 + (uint32_t)s, f ? 1u : 0u)) {
+                        ok = false;
+                        s_failed = 1;
+                        break;
+                    }
+                    if (++s == kStages) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                }
             }
         }
     } else if (warp >= (uint32_t)kEpiWarp0) {
@@ -583,6 +683,54 @@ __global__ void __launch_bounds__(gp_threads<kEpi>(), 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(acc_empty_leader);   // this half of the pair is drained
+            if (kEpi == kEpiPlain) {
+                // 32 columns at a time: bf16 into this warp's staging buffer
+                // (16-byte piece j of row `lane` at j ^ ((lane / 2) % 4), the
+                // 64-byte swizzle), then one TMA store of the 32 x 32 box; rows
+                // past M and columns past N are not written
+                const uint32_t stage0 =
+                    smem_u32(smem + Y_STAGE_OFF) + (uint32_t)(warp - kEpiWarp0) * (2u * kYStageBytes);
+                const int row0 = (int)(grow - lane);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const int n = nbase + 32 * c;
+                    if (n >= a.N) break;   // warp-uniform
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        uint32_t bw[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+                        if (a.bias && n + 16 * h < a.N) {
+                            const uint4 w0 = __ldg(reinterpret_cast<const uint4*>(a.bias + n + 16 * h));
+                            const uint4 w1 = __ldg(reinterpret_cast<const uint4*>(a.bias + n + 16 * h) + 1);
+                            bw[0] = w0.x, bw[1] = w0.y, bw[2] = w0.z, bw[3] = w0.w;
+                            bw[4] = w1.x, bw[5] = w1.y, bw[6] = w1.z, bw[7] = w1.w;
+                        }
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const float o0 =
+                                fmaf(__uint_as_float(acc[32 * c + 16 * h + 2 * i]), S, bf16lo_to_f32(bw[i]));
+                            const float o1 =
+                                fmaf(__uint_as_float(acc[32 * c + 16 * h + 2 * i + 1]), S, bf16hi_to_f32(bw[i]));
+                            const __nv_bfloat162 hv = __floats2bfloat162_rn(o0, o1);
+                            pk[8 * h + i] = *reinterpret_cast<const uint32_t*>(&hv);
+                        }
+                    }
+                    const uint32_t buf = stage0 + (uint32_t)(c & 1) * kYStageBytes;
+                    if (lane == 0) bulk_wait_group_read<1>();   // the previous store from this buffer has read it
+                    __syncwarp();
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        st_shared_v4(buf + 64u * lane + ((uint32_t)(j ^ ((lane >> 1) & 3)) << 4), pk[4 * j],
+                                     pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0 && row0 < a.M) {   // a box wholly past M is not stored at all
+                        tma_store_2d(&tm_y, buf, n, row0);
+                        bulk_commit_group();
+                    }
+                }
+                continue;
+            }
             if (grow >= a.M) continue;
             __nv_bfloat16* yrow = a.y + grow * (int64_t)a.N;
             if (kEpi == kEpiQkv && nbase < a.qk_cols) {
@@ -636,39 +784,12 @@ __global__ void __launch_bounds__(gp_threads<kEpi>(), 1)
                 }
                 continue;
             }
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                const int n = nbase + 16 * c;
-                if (n >= a.N) break;
-                float bv[16];
-                if (a.bias) {
-                    const uint4 w0 = __ldg(reinterpret_cast<const uint4*>(a.bias + n));
-                    const uint4 w1 = __ldg(reinterpret_cast<const uint4*>(a.bias + n) + 1);
-                    const uint32_t ws[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-#pragma unroll
-                    for (int p = 0; p < 8; ++p) {
-                        bv[2 * p] = bf16lo_to_f32(ws[p]);
-                        bv[2 * p + 1] = bf16hi_to_f32(ws[p]);
-                    }
-                } else {
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) bv[i] = 0.0f;
-                }
-                uint32_t packed[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const float o0 = fmaf(__uint_as_float(acc[16 * c + 2 * i]), S, bv[2 * i]);
-                    const float o1 = fmaf(__uint_as_float(acc[16 * c + 2 * i + 1]), S, bv[2 * i + 1]);
-                    const __nv_bfloat162 h = __floats2bfloat162_rn(o0, o1);
-                    packed[i] = *reinterpret_cast<const uint32_t*>(&h);
-                }
-                uint4* dst = reinterpret_cast<uint4*>(yrow + n);
-                dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-                dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
-            }
+            gp_store_plain<128>(acc, a, S, yrow, nbase);
         }
     }
 
+    if (kEpi == kEpiPlain && warp >= (uint32_t)kEpiWarp0 && lane == 0)
+        bulk_wait_group<0>();   // this warp's y stores are done with shared memory and written
     __syncthreads();
     if (s_failed && rank == 0 && warp == 0 && lane == 0) {
         // after a timeout, let the loads already issued land before either CTA

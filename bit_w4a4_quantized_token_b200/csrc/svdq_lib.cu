@@ -127,7 +127,7 @@ svdq_status check_device() {
             cudaFuncSetAttribute(gemm_w4a16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)aw::SMEM_BYTES) != cudaSuccess ||
             cudaFuncSetAttribute(gemm_nvfp4_pair_kernel<kEpiPlain>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)gp::SMEM_BYTES) != cudaSuccess ||
+                                 (int)gp::SMEM_BYTES_PLAIN) != cudaSuccess ||
             cudaFuncSetAttribute(gemm_nvfp4_pair_kernel<kEpiQkv>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)gp::SMEM_BYTES) != cudaSuccess ||
             cudaFuncSetAttribute(gemm_nvfp4_pair_kernel<kEpiGelu>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -517,8 +517,8 @@ int pair_clusters() {
         attr[0].val.clusterDim.y = 1;
         attr[0].val.clusterDim.z = 1;
         cfg.gridDim = dim3(2 * (unsigned)num_sms(), 1, 1);
-        cfg.blockDim = dim3(gp::kThreads, 1, 1);
-        cfg.dynamicSmemBytes = gp::SMEM_BYTES;
+        cfg.blockDim = dim3(gp_threads<kEpiPlain>(), 1, 1);
+        cfg.dynamicSmemBytes = gp::SMEM_BYTES_PLAIN;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         int n = 0;
@@ -619,17 +619,23 @@ svdq_status gemm_nvfp4_pair(const void* x_codes, const void* x_scales, const flo
     const int clusters = (int)std::min<int64_t>(mt * nt, pair_clusters());
     // programmatic dependent launch: the kernel's prologue overlaps the tail of
     // the activation quantizer, which releases its dependents early
-    const dim3 grid(2 * (unsigned)clusters), block(gp::kThreads);
+    const dim3 grid(2 * (unsigned)clusters), block(gp_threads<kEpiPlain>());   // the QKV variant's too
     cudaError_t e;
     if (gelu.next_x_scale)
         e = launch_ex(gemm_nvfp4_pair_kernel<kEpiGelu>, grid, dim3(gp::kThreadsGelu), gp::SMEM_BYTES_GELU, st, 2u,
-                      tm_xc, tm_wc, tm_sfa, tm_sfb, tm_L, tm_Lup, a);
+                      tm_xc, tm_wc, tm_sfa, tm_sfb, tm_L, tm_Lup, tm_xc, a);
     else if (qkv.heads > 0)
         e = launch_ex(gemm_nvfp4_pair_kernel<kEpiQkv>, grid, block, gp::SMEM_BYTES, st, 2u, tm_xc, tm_wc, tm_sfa,
-                      tm_sfb, tm_L, tm_Lup, a);
-    else
-        e = launch_ex(gemm_nvfp4_pair_kernel<kEpiPlain>, grid, block, gp::SMEM_BYTES, st, 2u, tm_xc, tm_wc, tm_sfa,
-                      tm_sfb, tm_L, tm_Lup, a);
+                      tm_sfb, tm_L, tm_Lup, tm_xc, a);
+    else {
+        // y leaves through TMA stores of 32 x 32 boxes (64-byte swizzle)
+        CUtensorMap tm_y;
+        if (!make_map(&tm_y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, (uint64_t)N, (uint64_t)M, (uint64_t)N * 2, 32, 32,
+                      CU_TENSOR_MAP_SWIZZLE_64B))
+            return SVDQ_ERR_CUDA;
+        e = launch_ex(gemm_nvfp4_pair_kernel<kEpiPlain>, grid, block, gp::SMEM_BYTES_PLAIN, st, 2u, tm_xc, tm_wc,
+                      tm_sfa, tm_sfb, tm_L, tm_Lup, tm_y, a);
+    }
     if (e != cudaSuccess) return cuda_fail("gemm_nvfp4_pair_kernel launch");
     return launch_status("gemm_nvfp4_pair_kernel launch");
 }
