@@ -1,0 +1,323 @@
+// gemm_dq16.cuh -- the two int4 GEMMs of the Diffusers docs page "Nunchaku
+// Lite" ("Supported quantization types" table), on fp16 tensor-core MMAs
+// (sm_100a):
+//
+//  * W4A16, the `awq_w4a16` scheme (int4 weights, group 64; the AWQ scaling
+//    folded into the weights offline, x used as it comes):
+//        y[m, n] = bf16( sum_k x[m, k] (q_w[n, k] s_w[n, k / 64]) + b[n] )
+//  * the int4 W4A4 variant of the SVDQ layer (`svdq_w4a4` with precision
+//    int4, group 64, with the rank-r correction):
+//        y[m, n] = bf16( sum_k (q_x[m, k] s_x[m, k / 64]) (q_w[n, k] s_w[n, k / 64])
+//                        + sum_j L[m, j] L_up[j, n] + b[n] )
+//
+// Every product q s of a signed 4-bit code and a bf16 group scale is exact in
+// fp16 (at most 3 + 8 significant bits, for scales in fp16's normal range),
+// and a bf16 activation converts exactly to fp16 in fp16's normal range.  So
+// both operands are expanded into fp16 tiles in shared memory and multiplied
+// with kind::f16 MMAs (fp16 x fp16, fp32 accumulation): the group scales are
+// applied before the MMA instead of on the accumulators, and no per-group
+// rescale is left for the CUDA cores.  The rank-r term runs as bf16 MMAs
+// (the hi and lo parts of L against L_up) into the same accumulator.
+//
+// One CTA per 128 x 256 output tile.  Warp 0 loads, per 64 columns of K, the
+// activation tile (bf16 x, or int4 codes and their group scales), the packed
+// weight tile (256 rows x 32 bytes) and its 256 group scales; warps 4..11
+// expand both into fp16 tiles in the MMA's swizzled layout (x converted in
+// place); warp 1 issues four M = 128, N = 256, K = 16 MMAs per stage into
+// TMEM; warps 12..19 add the bias and store bf16.
+#pragma once
+#include "sm100_ptx.cuh"
+
+namespace svdq {
+namespace dq {
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int kStages = 3;
+constexpr int A_BYTES = 128 * 128;            // fp16 A: 128 rows x 64 values (x arrives here as bf16)
+constexpr int WF_BYTES = 256 * 128;           // fp16 weights: 256 rows x 64 values
+constexpr int WP_BYTES = 256 * 32;            // packed int4 weights: 256 rows x 64 codes
+constexpr int AP_BYTES = 128 * 32;            // packed int4 activations: 128 rows x 64 codes
+constexpr int WS_BYTES = 256 * 2;             // bf16 group scales of the 256 weight rows
+constexpr int AS_BYTES = 128 * 2;             // bf16 group scales of the 128 activation rows
+constexpr int OFF_WF = A_BYTES;
+constexpr int OFF_WP = OFF_WF + WF_BYTES;
+constexpr int OFF_AP = OFF_WP + WP_BYTES;
+constexpr int OFF_WS = OFF_AP + AP_BYTES;
+constexpr int OFF_AS = OFF_WS + WS_BYTES;
+constexpr int STAGE_BYTES = ((OFF_AS + AS_BYTES + 1023) / 1024) * 1024;
+constexpr int kConvWarp0 = 4, kConvWarps = 8;
+constexpr int kEpiWarp0 = 12, kEpiWarps = 8;
+constexpr int kThreads = 32 * (kEpiWarp0 + kEpiWarps);
+constexpr size_t SMEM_BYTES = 1024 + (size_t)kStages * STAGE_BYTES + 256;
+static_assert(SMEM_BYTES <= 227 * 1024, "stage ring does not fit in shared memory");
+}  // namespace dq
+
+struct Dq16Args {
+    const __nv_bfloat16* bias;   // may be null
+    __nv_bfloat16* y;
+    int M, N, K;
+    int rank;                    // int4 W4A4: rank-r chunks appended to the K loop
+};
+
+enum : uint32_t { kSiteDqEmpty = 40, kSiteDqFull = 41, kSiteDqConv = 42, kSiteDqAcc = 43, kSiteDqDrain = 44 };
+
+__host__ __device__ constexpr uint32_t idesc_f16_f32(uint32_t n) {
+    return (1u << 4)            // D format f32; A and B format f16 (0)
+           | ((n >> 3) << 17)   // N / 8
+           | ((128u >> 4) << 24);  // M / 16
+}
+
+// 8 int4 codes (two's complement, element i in bits 4i+3..4i) times the fp16
+// scale pair s2 -> 8 fp16 values in element order (four fp16x2 words).  The
+// nibble n is q + 8 after flipping its top bit, and the fp16 with bits
+// 0x6400 | (q + 8) is 1024 + q + 8; subtracting 1032 leaves q exactly.
+__device__ __forceinline__ void int4x8_to_f16(uint32_t w, __half2 s2, uint32_t (&out)[4]) {
+    const uint32_t u = w ^ 0x88888888u;
+    const __half2 bias2 = __halves2half2(__ushort_as_half(0x6408), __ushort_as_half(0x6408));   // 1032
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+        // elements 2p (bits 8p..8p+3) and 2p+1 (bits 8p+4..8p+7)
+        const uint32_t lo = (u >> (8 * p)) & 0xFu, hi = (u >> (8 * p + 4)) & 0xFu;
+        const uint32_t bits = (0x6400u | lo) | ((0x6400u | hi) << 16);
+        __half2 v = *reinterpret_cast<const __half2*>(&bits);
+        v = __hmul2(__hsub2(v, bias2), s2);
+        out[p] = *reinterpret_cast<const uint32_t*>(&v);
+    }
+}
+
+__device__ __forceinline__ __half2 bf16_scale_to_h2(uint16_t sbits) {
+    const __half sh = __float2half_rn(__bfloat162float(__ushort_as_bfloat16(sbits)));
+    return __halves2half2(sh, sh);
+}
+
+// kInt4A: the activations are int4 codes with bf16 group scales (the int4
+// W4A4 layer); otherwise bf16 (W4A16).  tm_a: x [M, K] bf16 (box 64 x 128,
+// 128-byte swizzle) or the activation codes [M, K/2] (box 32 x 128);
+// tm_as: activation scales [K/64, rows_pad] (box 128 x 1; int4 only);
+// tm_L, tm_Lup: the rank-r operands (int4 W4A4 with rank > 0 only).
+template <bool kInt4A>
+__global__ void __launch_bounds__(dq::kThreads, 1)
+    gemm_dq16_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_as,
+                     const __grid_constant__ CUtensorMap tm_wc, const __grid_constant__ CUtensorMap tm_ws,
+                     const __grid_constant__ CUtensorMap tm_L, const __grid_constant__ CUtensorMap tm_Lup,
+                     Dq16Args a) {
+    using namespace dq;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)kStages * STAGE_BYTES);
+    uint64_t* conv = full + kStages;
+    uint64_t* empty = conv + kStages;
+    uint64_t* acc_full = empty + kStages;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
+    __shared__ int s_failed;
+    __shared__ int s_issued[dq::kStages];
+
+    const uint32_t warp = warp_id(), lane = lane_id();
+    const int m0 = blockIdx.x * BM, n0 = blockIdx.y * BN;
+    const int n_kc = a.K / 64;
+    const int n_lr = (kInt4A && a.rank > 0) ? 2 * ((a.rank + 63) / 64) : 0;   // hi and lo per 64 of rank
+    const int n_st = n_kc + n_lr;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&conv[s], kConvWarps);
+            mbar_init(&empty[s], 1);
+            s_issued[s] = 0;
+        }
+        mbar_init(acc_full, 1);
+        s_failed = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tensormap(&tm_a);
+        prefetch_tensormap(&tm_wc);
+        prefetch_tensormap(&tm_ws);
+        if (kInt4A) prefetch_tensormap(&tm_as);
+        if (n_lr > 0) {
+            prefetch_tensormap(&tm_L);
+            prefetch_tensormap(&tm_Lup);
+        }
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 256);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            for (int it = 0; it < n_st; ++it) {
+                const int s = it % kStages;
+                const uint32_t ph = (uint32_t)(it / kStages) & 1u;
+                if (!mbar_wait(&empty[s], ph ^ 1u, kSiteDqEmpty)) {
+                    s_failed = 1;
+                    break;
+                }
+                uint8_t* st = smem + (size_t)s * STAGE_BYTES;
+                if (it < n_kc) {
+                    const int kc = it;
+                    if (kInt4A) {
+                        mbar_arrive_expect_tx(&full[s], AP_BYTES + AS_BYTES + WP_BYTES + WS_BYTES);
+                        tma_load_2d(st + OFF_AP, &tm_a, &full[s], kc * 32, m0);
+                        tma_load_2d(st + OFF_AS, &tm_as, &full[s], m0, kc);
+                    } else {
+                        mbar_arrive_expect_tx(&full[s], A_BYTES + WP_BYTES + WS_BYTES);
+                        tma_load_2d(st, &tm_a, &full[s], kc * 64, m0);
+                    }
+                    tma_load_2d(st + OFF_WP, &tm_wc, &full[s], kc * 32, n0);
+                    tma_load_2d(st + OFF_WS, &tm_ws, &full[s], n0, kc);
+                } else {
+                    // rank-r chunk: an L tile (hi or lo plane) and an L_up tile, already bf16
+                    const int c = (it - n_kc) >> 1, part = (it - n_kc) & 1;
+                    mbar_arrive_expect_tx(&full[s], A_BYTES + WF_BYTES);
+                    tma_load_3d(st, &tm_L, &full[s], c * 64, m0, part);
+                    tma_load_2d(st + OFF_WF, &tm_Lup, &full[s], c * 64, n0);
+                }
+                reinterpret_cast<volatile int*>(s_issued)[s] += 1;
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc = idesc_m(idesc_f16_f32(BN), BM);
+            const uint32_t idesc_lr = idesc_m(idesc_bf16_f32(BN), BM);
+            bool ok = true;
+            for (int it = 0; it < n_st; ++it) {
+                const int s = it % kStages;
+                if (!mbar_wait(&conv[s], (uint32_t)(it / kStages) & 1u, kSiteDqConv)) {
+                    ok = false;
+                    s_failed = 1;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t sx = smem_u32(smem + (size_t)s * STAGE_BYTES), sw = sx + OFF_WF;
+                if (it < n_kc) {
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        mma_bf16(tmem, desc_sw128(sx + 32u * j), desc_sw128(sw + 32u * j), idesc,
+                                 (it > 0 || j > 0) ? 1u : 0u);
+                } else {
+                    const int c = (it - n_kc) >> 1;
+                    const int nks = min(4, (a.rank - 64 * c + 15) / 16);
+                    for (int j = 0; j < nks; ++j)
+                        mma_bf16(tmem, desc_sw128(sx + 32u * j), desc_sw128(sw + 32u * j), idesc_lr, 1u);
+                }
+                tc_commit(&empty[s]);
+            }
+            if (ok) tc_commit(acc_full);
+        }
+    } else if (warp >= (uint32_t)kConvWarp0 && warp < (uint32_t)kConvWarp0 + kConvWarps) {
+        // ----------------------------------- activations and weights -> fp16
+        const int t = (int)threadIdx.x - 32 * kConvWarp0;   // 0..255: weight row t
+        for (int it = 0; it < n_st; ++it) {
+            const int s = it % kStages;
+            if (!mbar_wait(&full[s], (uint32_t)(it / kStages) & 1u, kSiteDqFull)) {
+                s_failed = 1;
+                break;
+            }
+            uint8_t* st = smem + (size_t)s * STAGE_BYTES;
+            if (it < n_kc) {
+                if (kInt4A) {
+                    // activation row t / 2, values 32 (t % 2) .. + 31: codes -> fp16 (q s_x)
+                    const int r = t >> 1, h = t & 1;
+                    const __half2 s2 = bf16_scale_to_h2(*reinterpret_cast<const uint16_t*>(st + OFF_AS + 2 * r));
+                    const uint4 c4 = *reinterpret_cast<const uint4*>(st + OFF_AP + 32 * r + 16 * h);
+                    const uint32_t cw[4] = {c4.x, c4.y, c4.z, c4.w};
+                    uint8_t* arow = st + r * 128;
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {   // 16-byte chunk 4h + c: values 8 (4h + c) .. + 7
+                        uint32_t o[4];
+                        int4x8_to_f16(cw[c], s2, o);
+                        *reinterpret_cast<uint4*>(arow + (((4 * h + c) ^ (r & 7)) << 4)) =
+                            make_uint4(o[0], o[1], o[2], o[3]);
+                    }
+                } else {
+                    // x: 16 KB of bf16 in place, 64 bytes per thread (position-preserving)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        uint4* p = reinterpret_cast<uint4*>(st + 16 * (t + 256 * i));
+                        const uint4 v = *p;
+                        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+                        uint32_t o[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const __half2 hv = __floats2half2_rn(bf16lo_to_f32(w[e]), bf16hi_to_f32(w[e]));
+                            o[e] = *reinterpret_cast<const uint32_t*>(&hv);
+                        }
+                        *p = make_uint4(o[0], o[1], o[2], o[3]);
+                    }
+                }
+                // weight row t: 64 codes -> 64 fp16 (q s_w) in the swizzled 128-byte row
+                const uint8_t* wp = st + OFF_WP + 32 * t;
+                const __half2 s2 = bf16_scale_to_h2(*reinterpret_cast<const uint16_t*>(st + OFF_WS + 2 * t));
+                const uint4 c0 = *reinterpret_cast<const uint4*>(wp), c1 = *reinterpret_cast<const uint4*>(wp + 16);
+                const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+                uint8_t* wrow = st + OFF_WF + t * 128;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {   // 16-byte chunk c: K values 8c .. 8c + 7
+                    uint32_t o[4];
+                    int4x8_to_f16(cw[c], s2, o);
+                    *reinterpret_cast<uint4*>(wrow + ((c ^ (t & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+                }
+                fence_proxy_async_smem();   // both tiles are read by the tensor core
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&conv[s]);
+        }
+    } else if (warp >= (uint32_t)kEpiWarp0) {
+        // ------------------------------------------------------------ epilogue
+        const uint32_t q = warp & 3u;
+        const int half = (int)(warp - kEpiWarp0) >> 2;
+        const int64_t grow = (int64_t)m0 + 32 * q + lane;
+        const bool ok = mbar_wait(acc_full, 0, kSiteDqAcc);
+        if (!ok) s_failed = 1;
+        tc_fence_after();
+        if (ok) {
+            __nv_bfloat16* yrow = a.y + grow * (int64_t)a.N;
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+                uint32_t acc[32];
+                tmem_ld_32x32b_x32(tmem + ((32u * q) << 16) + 128u * half + 32u * c, acc);
+                tmem_ld_wait();
+                const int n = n0 + 128 * half + 32 * c;
+#pragma unroll
+                for (int p = 0; p < 4; ++p) {
+                    if (n + 8 * p >= a.N) break;   // N % 16 == 0
+                    uint4 bw = make_uint4(0u, 0u, 0u, 0u);
+                    if (a.bias) bw = __ldg(reinterpret_cast<const uint4*>(a.bias + n + 8 * p));
+                    const uint32_t ws[4] = {bw.x, bw.y, bw.z, bw.w};
+                    uint32_t pk[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const float o0 = __fadd_rn(__uint_as_float(acc[8 * p + 2 * i]), bf16lo_to_f32(ws[i]));
+                        const float o1 = __fadd_rn(__uint_as_float(acc[8 * p + 2 * i + 1]), bf16hi_to_f32(ws[i]));
+                        const __nv_bfloat162 h2 = __floats2bfloat162_rn(o0, o1);
+                        pk[i] = *reinterpret_cast<const uint32_t*>(&h2);
+                    }
+                    if (grow < a.M) *reinterpret_cast<uint4*>(yrow + n + 8 * p) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                }
+            }
+        }
+    }
+
+    __syncthreads();
+    if (s_failed && warp == 0 && lane == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            const int n = reinterpret_cast<volatile int*>(s_issued)[s];
+            if (n > 0) mbar_wait(&full[s], (uint32_t)(n - 1) & 1u, kSiteDqDrain);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 256);
+    }
+}
+
+}  // namespace svdq

@@ -98,9 +98,9 @@ constexpr uint32_t kFullArrivals = 3;          // CTA 0's three producer roles, 
 constexpr int kLanesPerRole = 2;               // producer lanes per role, taking alternate stages
 constexpr size_t SMEM_BYTES = 1024 + (size_t)kStages * STAGE_BYTES + 256;
 static_assert(SMEM_BYTES <= 227 * 1024, "stage ring does not fit in shared memory");
-// kEpiPlain: y leaves through TMA stores of 32 x 32 boxes staged per
-// epilogue warp in two 2 KB buffers (64-byte swizzle), 1 KB aligned after
-// the barriers.
+// kEpiPlain, kEpiQkv: y leaves through TMA stores of 32 x 32 boxes staged
+// per epilogue warp in two 2 KB buffers (64-byte swizzle), 1 KB aligned
+// after the barriers.
 constexpr int kYStageBytes = 2048;
 constexpr size_t Y_STAGE_OFF = (size_t)kStages * STAGE_BYTES + 1024;
 constexpr size_t SMEM_BYTES_PLAIN = 1024 + Y_STAGE_OFF + (size_t)kEpiWarps * 2 * kYStageBytes;
@@ -325,33 +325,47 @@ __device__ __forceinline__ void gp_gelu_epilogue(const uint32_t (&acc)[NC], cons
         }
 }
 
-// The plain epilogue of one thread's row over NC columns from nbase:
-// y = bf16(S acc + b), 16-byte stores.
-template <int NC>
-__device__ __forceinline__ void gp_store_plain(const uint32_t (&acc)[NC], const GemmArgs& a, float S,
-                                               __nv_bfloat16* yrow, int nbase) {
+// bf16(S acc + b) of one thread's row for the 32 columns n .. n + 31
+// (chunk c2 of its 128 accumulators), as 16 packed words.
+__device__ __forceinline__ void gp_pack32(const uint32_t (&acc)[128], int c2, const GemmArgs& a, float S, int n,
+                                          uint32_t (&pk)[16]) {
 #pragma unroll
-    for (int c = 0; c < NC / 16; ++c) {
-        const int n = nbase + 16 * c;
-        if (n >= a.N) break;   // N % 16 == 0
+    for (int h = 0; h < 2; ++h) {
         uint32_t bw[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-        if (a.bias) {
-            const uint4 w0 = __ldg(reinterpret_cast<const uint4*>(a.bias + n));
-            const uint4 w1 = __ldg(reinterpret_cast<const uint4*>(a.bias + n) + 1);
+        if (a.bias && n + 16 * h < a.N) {   // N % 16 == 0
+            const uint4 w0 = __ldg(reinterpret_cast<const uint4*>(a.bias + n + 16 * h));
+            const uint4 w1 = __ldg(reinterpret_cast<const uint4*>(a.bias + n + 16 * h) + 1);
             bw[0] = w0.x, bw[1] = w0.y, bw[2] = w0.z, bw[3] = w0.w;
             bw[4] = w1.x, bw[5] = w1.y, bw[6] = w1.z, bw[7] = w1.w;
         }
-        uint32_t packed[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            const float o0 = fmaf(__uint_as_float(acc[16 * c + 2 * i]), S, bf16lo_to_f32(bw[i]));
-            const float o1 = fmaf(__uint_as_float(acc[16 * c + 2 * i + 1]), S, bf16hi_to_f32(bw[i]));
-            const __nv_bfloat162 h = __floats2bfloat162_rn(o0, o1);
-            packed[i] = *reinterpret_cast<const uint32_t*>(&h);
+            const float o0 = fmaf(__uint_as_float(acc[32 * c2 + 16 * h + 2 * i]), S, bf16lo_to_f32(bw[i]));
+            const float o1 = fmaf(__uint_as_float(acc[32 * c2 + 16 * h + 2 * i + 1]), S, bf16hi_to_f32(bw[i]));
+            const __nv_bfloat162 hv = __floats2bfloat162_rn(o0, o1);
+            pk[8 * h + i] = *reinterpret_cast<const uint32_t*>(&hv);
         }
-        uint4* dst = reinterpret_cast<uint4*>(yrow + n);
-        dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-        dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+    }
+}
+
+// One warp's 32 rows x 32 columns of y through a 2 KB staging buffer: each
+// lane writes its row (16-byte piece j at j ^ ((lane / 2) % 4), the 64-byte
+// swizzle of the y tensor map), then lane 0 stores the box at (n, row0) with
+// TMA.  Before writing, lane 0 waits until at most one earlier store of this
+// thread still reads shared memory (the warp alternates two buffers).
+__device__ __forceinline__ void gp_stage_store(const uint32_t (&pk)[16], uint32_t buf, uint32_t lane,
+                                               const CUtensorMap* tm_y, int n, int row0, int M) {
+    if (lane == 0) bulk_wait_group_read<1>();
+    __syncwarp();
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+        st_shared_v4(buf + 64u * lane + ((uint32_t)(j ^ ((lane >> 1) & 3)) << 4), pk[4 * j], pk[4 * j + 1],
+                     pk[4 * j + 2], pk[4 * j + 3]);
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0 && row0 < M) {   // a box wholly past M is not stored at all
+        tma_store_2d(tm_y, buf, n, row0);
+        bulk_commit_group();
     }
 }
 
@@ -683,56 +697,12 @@ __global__ void __launch_bounds__(gp_threads<kEpi>(), 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(acc_empty_leader);   // this half of the pair is drained
-            if (kEpi == kEpiPlain) {
-                // 32 columns at a time: bf16 into this warp's staging buffer
-                // (16-byte piece j of row `lane` at j ^ ((lane / 2) % 4), the
-                // 64-byte swizzle), then one TMA store of the 32 x 32 box; rows
-                // past M and columns past N are not written
-                const uint32_t stage0 =
-                    smem_u32(smem + Y_STAGE_OFF) + (uint32_t)(warp - kEpiWarp0) * (2u * kYStageBytes);
-                const int row0 = (int)(grow - lane);
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const int n = nbase + 32 * c;
-                    if (n >= a.N) break;   // warp-uniform
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        uint32_t bw[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-                        if (a.bias && n + 16 * h < a.N) {
-                            const uint4 w0 = __ldg(reinterpret_cast<const uint4*>(a.bias + n + 16 * h));
-                            const uint4 w1 = __ldg(reinterpret_cast<const uint4*>(a.bias + n + 16 * h) + 1);
-                            bw[0] = w0.x, bw[1] = w0.y, bw[2] = w0.z, bw[3] = w0.w;
-                            bw[4] = w1.x, bw[5] = w1.y, bw[6] = w1.z, bw[7] = w1.w;
-                        }
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            const float o0 =
-                                fmaf(__uint_as_float(acc[32 * c + 16 * h + 2 * i]), S, bf16lo_to_f32(bw[i]));
-                            const float o1 =
-                                fmaf(__uint_as_float(acc[32 * c + 16 * h + 2 * i + 1]), S, bf16hi_to_f32(bw[i]));
-                            const __nv_bfloat162 hv = __floats2bfloat162_rn(o0, o1);
-                            pk[8 * h + i] = *reinterpret_cast<const uint32_t*>(&hv);
-                        }
-                    }
-                    const uint32_t buf = stage0 + (uint32_t)(c & 1) * kYStageBytes;
-                    if (lane == 0) bulk_wait_group_read<1>();   // the previous store from this buffer has read it
-                    __syncwarp();
-#pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        st_shared_v4(buf + 64u * lane + ((uint32_t)(j ^ ((lane >> 1) & 3)) << 4), pk[4 * j],
-                                     pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0 && row0 < a.M) {   // a box wholly past M is not stored at all
-                        tma_store_2d(&tm_y, buf, n, row0);
-                        bulk_commit_group();
-                    }
-                }
-                continue;
-            }
-            if (grow >= a.M) continue;
-            __nv_bfloat16* yrow = a.y + grow * (int64_t)a.N;
+            // y leaves 32 columns at a time through this warp's staging
+            // buffers and a TMA store (gp_stage_store); rows past M and
+            // columns past N are not written
+            const uint32_t stage0 =
+                smem_u32(smem + Y_STAGE_OFF) + (uint32_t)(warp - kEpiWarp0) * (2u * kYStageBytes);
+            const int row0 = (int)(grow - lane);
             if (kEpi == kEpiQkv && nbase < a.qk_cols) {
                 // this warp's 128 columns are one Q or K head of a to_qkv
                 // projection (qkv_norm_rope.cuh): RMSNorm over them, then the
@@ -759,36 +729,49 @@ __global__ void __launch_bounds__(gp_threads<kEpi>(), 1)
                 }
                 const float r = rsqrtf(ss * (1.0f / 128.0f) + a.eps);
                 const __nv_bfloat16* w = nbase < a.q_cols ? a.norm_q : a.norm_k;
-                const float4* cs4 = reinterpret_cast<const float4*>(a.rope_cos + grow * 64);
-                const float4* sn4 = reinterpret_cast<const float4*>(a.rope_sin + grow * 64);
+                // rows past M read the last row's rotary table (their results are not stored)
+                const int64_t trow = grow < a.M ? grow : (int64_t)a.M - 1;
+                const float4* cs4 = reinterpret_cast<const float4*>(a.rope_cos + trow * 64);
+                const float4* sn4 = reinterpret_cast<const float4*>(a.rope_sin + trow * 64);
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {   // 16 columns = 8 rotary pairs
-                    const uint4 g0 = __ldg(reinterpret_cast<const uint4*>(w + 16 * c));
-                    const uint4 g1 = __ldg(reinterpret_cast<const uint4*>(w + 16 * c) + 1);
-                    const uint32_t gs[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-                    const float4 c0 = __ldg(cs4 + 2 * c), c1 = __ldg(cs4 + 2 * c + 1);
-                    const float4 s0 = __ldg(sn4 + 2 * c), s1 = __ldg(sn4 + 2 * c + 1);
-                    const float cc[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-                    const float sc[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-                    uint32_t packed[8];
+                for (int c2 = 0; c2 < 4; ++c2) {
+                    uint32_t pk[16];
 #pragma unroll
-                    for (int p = 0; p < 8; ++p) {
-                        const float v0 = __uint_as_float(acc[16 * c + 2 * p]) * r * bf16lo_to_f32(gs[p]);
-                        const float v1 = __uint_as_float(acc[16 * c + 2 * p + 1]) * r * bf16hi_to_f32(gs[p]);
-                        const __nv_bfloat162 h = __floats2bfloat162_rn(v0 * cc[p] - v1 * sc[p], v1 * cc[p] + v0 * sc[p]);
-                        packed[p] = *reinterpret_cast<const uint32_t*>(&h);
+                    for (int h = 0; h < 2; ++h) {   // 16 columns = 8 rotary pairs
+                        const int c = 2 * c2 + h;
+                        const uint4 g0 = __ldg(reinterpret_cast<const uint4*>(w + 16 * c));
+                        const uint4 g1 = __ldg(reinterpret_cast<const uint4*>(w + 16 * c) + 1);
+                        const uint32_t gs[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+                        const float4 c0 = __ldg(cs4 + 2 * c), c1 = __ldg(cs4 + 2 * c + 1);
+                        const float4 s0 = __ldg(sn4 + 2 * c), s1 = __ldg(sn4 + 2 * c + 1);
+                        const float cc[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+                        const float sc[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+#pragma unroll
+                        for (int p = 0; p < 8; ++p) {
+                            const float v0 = __uint_as_float(acc[16 * c + 2 * p]) * r * bf16lo_to_f32(gs[p]);
+                            const float v1 = __uint_as_float(acc[16 * c + 2 * p + 1]) * r * bf16hi_to_f32(gs[p]);
+                            const __nv_bfloat162 hv =
+                                __floats2bfloat162_rn(v0 * cc[p] - v1 * sc[p], v1 * cc[p] + v0 * sc[p]);
+                            pk[8 * h + p] = *reinterpret_cast<const uint32_t*>(&hv);
+                        }
                     }
-                    uint4* dst = reinterpret_cast<uint4*>(yrow + nbase + 16 * c);
-                    dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-                    dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+                    gp_stage_store(pk, stage0 + (uint32_t)(c2 & 1) * kYStageBytes, lane, &tm_y, nbase + 32 * c2,
+                                   row0, a.M);
                 }
                 continue;
             }
-            gp_store_plain<128>(acc, a, S, yrow, nbase);
+#pragma unroll
+            for (int c2 = 0; c2 < 4; ++c2) {
+                const int n = nbase + 32 * c2;
+                if (n >= a.N) break;   // warp-uniform
+                uint32_t pk[16];
+                gp_pack32(acc, c2, a, S, n, pk);
+                gp_stage_store(pk, stage0 + (uint32_t)(c2 & 1) * kYStageBytes, lane, &tm_y, n, row0, a.M);
+            }
         }
     }
 
-    if (kEpi == kEpiPlain && warp >= (uint32_t)kEpiWarp0 && lane == 0)
+    if (kEpi != kEpiGelu && warp >= (uint32_t)kEpiWarp0 && lane == 0)
         bulk_wait_group<0>();   // this warp's y stores are done with shared memory and written
     __syncthreads();
     if (s_failed && rank == 0 && warp == 0 && lane == 0) {

@@ -20,8 +20,7 @@
 #include "gemm_nvfp4_pair.cuh"
 #include "qkv_norm_rope.cuh"
 #include "svd_split.cuh"
-#include "gemm_w4a16.cuh"
-#include "int4.cuh"
+#include "gemm_dq16.cuh"
 
 namespace svdq {
 namespace {
@@ -122,14 +121,14 @@ svdq_status check_device() {
                                  kQuantSmemBudget) != cudaSuccess ||
             cudaFuncSetAttribute(quantize_act_kernel<kPrecInt4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kQuantSmemBudget) != cudaSuccess ||
-            cudaFuncSetAttribute(gemm_int4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)i4::SMEM_BYTES) != cudaSuccess ||
-            cudaFuncSetAttribute(gemm_w4a16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)aw::SMEM_BYTES) != cudaSuccess ||
+            cudaFuncSetAttribute(gemm_dq16_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)dq::SMEM_BYTES) != cudaSuccess ||
+            cudaFuncSetAttribute(gemm_dq16_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)dq::SMEM_BYTES) != cudaSuccess ||
             cudaFuncSetAttribute(gemm_nvfp4_pair_kernel<kEpiPlain>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)gp::SMEM_BYTES_PLAIN) != cudaSuccess ||
             cudaFuncSetAttribute(gemm_nvfp4_pair_kernel<kEpiQkv>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)gp::SMEM_BYTES) != cudaSuccess ||
+                                 (int)gp::SMEM_BYTES_PLAIN) != cudaSuccess ||
             cudaFuncSetAttribute(gemm_nvfp4_pair_kernel<kEpiGelu>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)gp::SMEM_BYTES_GELU) != cudaSuccess)
             return cuda_fail("setting kernel shared-memory limits");
@@ -624,57 +623,71 @@ svdq_status gemm_nvfp4_pair(const void* x_codes, const void* x_scales, const flo
     if (gelu.next_x_scale)
         e = launch_ex(gemm_nvfp4_pair_kernel<kEpiGelu>, grid, dim3(gp::kThreadsGelu), gp::SMEM_BYTES_GELU, st, 2u,
                       tm_xc, tm_wc, tm_sfa, tm_sfb, tm_L, tm_Lup, tm_xc, a);
-    else if (qkv.heads > 0)
-        e = launch_ex(gemm_nvfp4_pair_kernel<kEpiQkv>, grid, block, gp::SMEM_BYTES, st, 2u, tm_xc, tm_wc, tm_sfa,
-                      tm_sfb, tm_L, tm_Lup, tm_xc, a);
     else {
         // y leaves through TMA stores of 32 x 32 boxes (64-byte swizzle)
         CUtensorMap tm_y;
         if (!make_map(&tm_y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, (uint64_t)N, (uint64_t)M, (uint64_t)N * 2, 32, 32,
                       CU_TENSOR_MAP_SWIZZLE_64B))
             return SVDQ_ERR_CUDA;
-        e = launch_ex(gemm_nvfp4_pair_kernel<kEpiPlain>, grid, block, gp::SMEM_BYTES_PLAIN, st, 2u, tm_xc, tm_wc,
-                      tm_sfa, tm_sfb, tm_L, tm_Lup, tm_y, a);
+        if (qkv.heads > 0)
+            e = launch_ex(gemm_nvfp4_pair_kernel<kEpiQkv>, grid, block, gp::SMEM_BYTES_PLAIN, st, 2u, tm_xc, tm_wc,
+                          tm_sfa, tm_sfb, tm_L, tm_Lup, tm_y, a);
+        else
+            e = launch_ex(gemm_nvfp4_pair_kernel<kEpiPlain>, grid, block, gp::SMEM_BYTES_PLAIN, st, 2u, tm_xc, tm_wc,
+                          tm_sfa, tm_sfb, tm_L, tm_Lup, tm_y, a);
     }
     if (e != cudaSuccess) return cuda_fail("gemm_nvfp4_pair_kernel launch");
     return launch_status("gemm_nvfp4_pair_kernel launch");
 }
 
-svdq_status int4_gemm(const void* x_codes, const void* x_scales, int64_t M, const void* w_codes, const void* w_scales,
-                      int64_t N, int64_t K, const void* lowrank, const void* L_up_t, int rank, const void* bias, void* y,
-                      cudaStream_t st) {
-    CUtensorMap tm_xc, tm_wc, tm_L, tm_Lup;
-    if (!make_map(&tm_xc, CU_TENSOR_MAP_DATA_TYPE_UINT8, x_codes, (uint64_t)K / 2, (uint64_t)M, (uint64_t)K / 2, 128,
-                  i4::BM) ||
-        !make_map(&tm_wc, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_codes, (uint64_t)K / 2, (uint64_t)N, (uint64_t)K / 2, 128,
-                  i4::BN))
-        return SVDQ_ERR_CUDA;
-    if (rank > 0) {
-        if (!make_map_3d(&tm_L, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, lowrank, (uint64_t)rank, (uint64_t)M, 2,
-                         (uint64_t)rank * 2, 64, i4::BM, 1) ||
-            !make_map(&tm_Lup, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L_up_t, (uint64_t)rank, (uint64_t)N,
-                      (uint64_t)rank * 2, 64, i4::BN))
-            return SVDQ_ERR_CUDA;
-    } else {
-        tm_L = tm_xc;
+// The int4 GEMMs on fp16 MMAs (gemm_dq16.cuh): int4 W4A4 (a_codes, a_scales:
+// the activation's int4 codes and bf16 group scales; rank-r operands) or
+// W4A16 (x bf16 in a_codes, a_scales null, rank 0).
+svdq_status dq16_gemm(bool int4_a, const void* a_codes, const void* a_scales, int64_t M, const void* w_codes,
+                      const void* w_scales, int64_t N, int64_t K, const void* lowrank, const void* L_up_t, int rank,
+                      const void* bias, void* y, cudaStream_t st) {
+    const int64_t mt = (M + dq::BM - 1) / dq::BM, nt = (N + dq::BN - 1) / dq::BN;
+    if (mt > 0x7FFFFFFF || nt > 65535) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+    CUtensorMap tm_a, tm_as, tm_wc, tm_ws, tm_L, tm_Lup;
+    const int64_t n_pad = round_up(N, 128), m_pad = round_up(M, 128);
+    bool ok;
+    if (int4_a)
+        ok = make_map(&tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_codes, (uint64_t)K / 2, (uint64_t)M, (uint64_t)K / 2, 32,
+                      128, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+             make_map(&tm_as, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a_scales, (uint64_t)m_pad, (uint64_t)(K / 64),
+                      (uint64_t)m_pad * 2, 128, 1, CU_TENSOR_MAP_SWIZZLE_NONE);
+    else
+        ok = make_map(&tm_a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a_codes, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, 64,
+                      128);
+    ok = ok &&
+         make_map(&tm_wc, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_codes, (uint64_t)K / 2, (uint64_t)N, (uint64_t)K / 2, 32,
+                  256, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+         make_map(&tm_ws, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w_scales, (uint64_t)n_pad, (uint64_t)(K / 64),
+                  (uint64_t)n_pad * 2, 256, 1, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (ok && rank > 0)
+        ok = make_map_3d(&tm_L, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, lowrank, (uint64_t)rank, (uint64_t)M, 2,
+                         (uint64_t)rank * 2, 64, dq::BM, 1) &&
+             make_map(&tm_Lup, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L_up_t, (uint64_t)rank, (uint64_t)N,
+                      (uint64_t)rank * 2, 64, dq::BN);
+    if (!ok) return SVDQ_ERR_CUDA;
+    if (!int4_a) tm_as = tm_a;
+    if (rank == 0) {
+        tm_L = tm_a;
         tm_Lup = tm_wc;
     }
-    Int4GemmArgs a;
-    a.x_scales = reinterpret_cast<const uint16_t*>(x_scales);
-    a.w_scales = reinterpret_cast<const uint16_t*>(w_scales);
+    Dq16Args a;
     a.bias = reinterpret_cast<const __nv_bfloat16*>(bias);
     a.y = reinterpret_cast<__nv_bfloat16*>(y);
     a.M = (int)M;
     a.N = (int)N;
     a.K = (int)K;
     a.rank = rank;
-    a.rows_pad_m = (int)round_up(M, 128);
-    a.rows_pad_n = (int)round_up(N, 128);
-    const int64_t mt = (M + i4::BM - 1) / i4::BM, nt = (N + i4::BN - 1) / i4::BN;
-    if (nt > 65535 || mt > (int64_t(1) << 31) - 1) return SVDQ_ERR_UNSUPPORTED_SHAPE;
-    gemm_int4_kernel<<<dim3((unsigned)mt, (unsigned)nt, 1), i4::kThreads, i4::SMEM_BYTES, st>>>(tm_xc, tm_wc, tm_L,
-                                                                                             tm_Lup, a);
-    return launch_status("gemm_int4_kernel launch");
+    const dim3 grid((unsigned)mt, (unsigned)nt, 1);
+    if (int4_a)
+        gemm_dq16_kernel<true><<<grid, dq::kThreads, dq::SMEM_BYTES, st>>>(tm_a, tm_as, tm_wc, tm_ws, tm_L, tm_Lup, a);
+    else
+        gemm_dq16_kernel<false><<<grid, dq::kThreads, dq::SMEM_BYTES, st>>>(tm_a, tm_as, tm_wc, tm_ws, tm_L, tm_Lup, a);
+    return launch_status("gemm_dq16_kernel launch");
 }
 
 // Kernel that waits on a barrier nobody completes: exercises the bounded wait.
@@ -918,7 +931,7 @@ svdq_status svdq_gemm_w4a4(svdq_precision p, int group_size, const void* x_codes
         return gemm_nvfp4(x_codes, x_scales, x_tensor_scale, M, w_codes, w_scales, w_tensor_scale, N, K, lowrank_act,
                           L_up_t, rank, bias, y, st);
     }
-    return int4_gemm(x_codes, x_scales, M, w_codes, w_scales, N, K, lowrank_act, L_up_t, rank, bias, y, st);
+    return dq16_gemm(true, x_codes, x_scales, M, w_codes, w_scales, N, K, lowrank_act, L_up_t, rank, bias, y, st);
 }
 
 // Checks of the fused QKV + RMSNorm + RoPE arguments shared by both entry points.
@@ -1096,26 +1109,9 @@ svdq_status svdq_gemm_w4a16(const void* x, int64_t M, const void* w_codes, const
     SVDQ_TRY(check_ptr(w_scales));
     SVDQ_TRY(check_ptr(y));
     SVDQ_TRY(check_opt_ptr(bias));
-    const int64_t mt = (M + aw::BM - 1) / aw::BM, nt = (N + aw::BN - 1) / aw::BN;
-    if (mt > 0x7FFFFFFF || nt > 65535) return SVDQ_ERR_UNSUPPORTED_SHAPE;
     SVDQ_TRY(check_device());
-    CUtensorMap tm_x, tm_wc, tm_ws;
-    const int64_t n_pad = round_up(N, 128);
-    if (!make_map(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, 64, 128) ||
-        !make_map(&tm_wc, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_codes, (uint64_t)K / 2, (uint64_t)N, (uint64_t)K / 2, 32,
-                  256, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !make_map(&tm_ws, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w_scales, (uint64_t)n_pad, (uint64_t)(K / 64),
-                  (uint64_t)n_pad * 2, 256, 1, CU_TENSOR_MAP_SWIZZLE_NONE))
-        return SVDQ_ERR_CUDA;
-    W4A16Args a;
-    a.bias = reinterpret_cast<const __nv_bfloat16*>(bias);
-    a.y = reinterpret_cast<__nv_bfloat16*>(y);
-    a.M = (int)M;
-    a.N = (int)N;
-    a.K = (int)K;
-    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    gemm_w4a16_kernel<<<dim3((unsigned)mt, (unsigned)nt, 1), aw::kThreads, aw::SMEM_BYTES, st>>>(tm_x, tm_wc, tm_ws, a);
-    return launch_status("gemm_w4a16_kernel launch");
+    return dq16_gemm(false, x, nullptr, M, w_codes, w_scales, N, K, nullptr, nullptr, 0, bias, y,
+                     reinterpret_cast<cudaStream_t>(stream));
 }
 
 svdq_status svdq_svd_split_workspace_bytes(int64_t N, int64_t K, int rank, int oversample, size_t* bytes) {

@@ -193,7 +193,13 @@ svdq_status svdq_quantize_act_noalloc(svdq_precision precision, int group_size,
  *   y[m, n] = bf16( sum_g sx[m,g] sw[n,g] sum_{k in g} qx qw + sum_j L[m,j] L_up[j,n] + b[n] )  (int4)
  * Inputs are the outputs of the two calls above; bias is device bf16 [N] or
  * NULL; lowrank_act / L_up_t may be NULL when rank == 0.
- * Output: y device bf16 [M, N]. */
+ * Output: y device bf16 [M, N].
+ * Arithmetic: nvfp4 multiplies the E2M1 codes with their E4M3 group scales on
+ * the block-scaled tensor cores (fp32 accumulation); int4 expands each code
+ * times its bf16 group scale into fp16 (exact for scales in fp16's normal
+ * range) and multiplies fp16 x fp16 with fp32 accumulation.  Both add the
+ * rank-r term as bf16 MMAs of the hi and lo parts of L into the same
+ * accumulator, then the bias, and round once to bf16. */
 svdq_status svdq_gemm_w4a4(svdq_precision precision, int group_size,
                            const void* x_codes, const void* x_scales, const float* x_tensor_scale, int64_t M,
                            const void* w_codes, const void* w_scales, const float* w_tensor_scale,
