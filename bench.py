@@ -665,8 +665,10 @@ def shape_report(case, t: dict, peaks: dict, sm_mhz, world: int) -> dict:
             g["frac_at_clock"] = round(gemm_tf / fp["peak_at_clock"], 4)
         out["roofline"] = g
     else:
-        out["roofline"] = {"bound": "issue (per-group rescale on the CUDA cores)", "achieved": round(gemm_tf, 2),
-                           "unit": "TOP/s"}
+        # int4: codes times group scales expanded into fp16, fp16 x fp16 MMAs
+        out["roofline"] = {"bound": "tensor", "achieved": round(gemm_tf, 2), "peak": peaks["bf16_tflops"],
+                           "unit": "TFLOP/s", "frac": round(gemm_tf / peaks["bf16_tflops"], 4),
+                           "peak_source": f"{peaks['source']} bf16 burst (fp16 has the same nominal rate)"}
     if case.rank:
         out["lowrank_flops_not_counted"] = 2 * case.M * case.rank * (case.K + 2 * case.N)
     return out
@@ -806,7 +808,7 @@ def run_cuda(args) -> dict | None:
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": "nvfp4 (e2m1 x e2m1, ue4m3 group scales) -> fp32 accumulate -> bf16"
-                 if case.precision == "nvfp4" else "int4 x int4 (bf16 group scales) -> int32 / fp32 -> bf16",
+                 if case.precision == "nvfp4" else "int4 codes x bf16 group scales -> fp16 x fp16 -> fp32 -> bf16",
         "data": "synthetic (seeded DiT-shaped activations with 1% outlier channels; random-init weights)",
         "config": workload_config(case, args.dynamic_scale, world),
         "breakdown_us": report["breakdown_us"],
