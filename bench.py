@@ -907,6 +907,24 @@ def run_reference(args) -> dict | None:
     }
 
 
+def run_leg(args) -> dict:
+    """One extra leg on cuda:0 (one GPU), e.g. to capture its kernels with ncu."""
+    import torch
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.Stream(dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    steps = max(3, args.steps)
+    if args.leg == "qkv_norm_rope":
+        return time_qkv_fusion(dev, stream, flush, steps)
+    if args.leg == "gelu_mlp":
+        return time_gelu_mlp(dev, stream, flush, steps)
+    if args.leg == "w4a16_qkv":
+        return time_w4a16(dev, stream, flush, steps, load_peaks())
+    return time_svd_split(dev, stream, flush, steps)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -919,9 +937,14 @@ def main():
     ap.add_argument("--no-extra", action="store_true", help="skip the other DiT shapes")
     ap.add_argument("--dynamic-scale", action="store_true", help="derive S_x by the amax pre-pass every step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--leg", choices=["qkv_norm_rope", "gelu_mlp", "w4a16_qkv", "svd_split_qkv"],
+                    help="time one of the extra legs alone and print its JSON (for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    if args.leg:
+        print(json.dumps(run_leg(args)), flush=True)
+        return
     if args.impl == "reference":
         out = run_reference(args)
     else:
