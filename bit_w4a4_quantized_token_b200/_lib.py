@@ -29,6 +29,7 @@ GROUP_SIZES = {"nvfp4": 16, "int4": 64}
 # Every entry point declared in include/svdq.h.
 EXPORTS = (
     "svdq_status_string", "svdq_abi_version", "svdq_last_error", "svdq_buffer_sizes", "svdq_pack_weight",
+    "svdq_replicate_weight_scales",
     "svdq_quantize_act_workspace_bytes", "svdq_quantize_act", "svdq_quantize_act_noalloc", "svdq_gemm_w4a4",
     "svdq_gemm_w4a4_qkv_norm_rope", "svdq_qkv_norm_rope", "svdq_gelu_mlp_workspace_bytes",
     "svdq_gemm_w4a4_gelu_quant", "svdq_gelu", "svdq_gemm_w4a16", "svdq_svd_split_workspace_bytes",
@@ -50,7 +51,7 @@ class SvdqError(RuntimeError):
 
 class svdq_sizes(ctypes.Structure):
     _fields_ = [("codes_bytes", ctypes.c_size_t), ("scales_bytes", ctypes.c_size_t),
-                ("lowrank_bytes", ctypes.c_size_t)]
+                ("lowrank_bytes", ctypes.c_size_t), ("w_scales_bytes", ctypes.c_size_t)]
 
 
 def _load():
@@ -69,6 +70,8 @@ def _load():
     lib.svdq_buffer_sizes.restype = I
     lib.svdq_pack_weight.argtypes = [I, I, P, I64, I64, P, P, P, I, P, P, P, P, P, P, P]
     lib.svdq_pack_weight.restype = I
+    lib.svdq_replicate_weight_scales.argtypes = [P, I64, I64, P]
+    lib.svdq_replicate_weight_scales.restype = I
     lib.svdq_quantize_act_workspace_bytes.argtypes = [I, I64, I64, I, ctypes.POINTER(ctypes.c_size_t)]
     lib.svdq_quantize_act_workspace_bytes.restype = I
     lib.svdq_quantize_act.argtypes = [I, I, P, I64, I64, P, P, I, P, P, I, P, P, P, P, ctypes.c_size_t, P]
@@ -154,7 +157,8 @@ def svdq_buffer_sizes(precision, rows: int, K: int, rank: int) -> dict:
     out = svdq_sizes()
     _check(lib.svdq_buffer_sizes(_prec(precision), int(rows), int(K), int(rank), ctypes.byref(out)),
            "svdq_buffer_sizes")
-    return {"codes_bytes": out.codes_bytes, "scales_bytes": out.scales_bytes, "lowrank_bytes": out.lowrank_bytes}
+    return {"codes_bytes": out.codes_bytes, "scales_bytes": out.scales_bytes, "lowrank_bytes": out.lowrank_bytes,
+            "w_scales_bytes": out.w_scales_bytes}
 
 
 def svdq_pack_weight(precision, group_size, R, N, K, lam, L_down, L_up, rank, w_codes, w_scales,
@@ -163,6 +167,11 @@ def svdq_pack_weight(precision, group_size, R, N, K, lam, L_down, L_up, rank, w_
                                 _ptr(L_down), _ptr(L_up), int(rank), _ptr(w_codes), _ptr(w_scales),
                                 _ptr(w_tensor_scale), _ptr(inv_lambda), _ptr(L_down_t), _ptr(L_up_t),
                                 _stream(stream)), "svdq_pack_weight")
+
+
+def svdq_replicate_weight_scales(w_scales, N, K, stream=None) -> None:
+    _check(lib.svdq_replicate_weight_scales(_ptr(w_scales), int(N), int(K), _stream(stream)),
+           "svdq_replicate_weight_scales")
 
 
 def svdq_quantize_act_workspace_bytes(precision, M: int, K: int, rank: int) -> int:

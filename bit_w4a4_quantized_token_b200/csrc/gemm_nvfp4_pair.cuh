@@ -62,11 +62,20 @@ namespace gp {
 constexpr int BM = 256;                        // tile rows (128 per CTA)
 constexpr int BN = 256;                        // tile columns (128 weight rows loaded per CTA)
 constexpr int BK_BYTES = 128;
-constexpr int kStages = 5;
+constexpr int kStages = 4;
 constexpr int A_BYTES = 128 * BK_BYTES;        // 16 KB: this CTA's 128 activation rows
 constexpr int B_BYTES = 128 * BK_BYTES;        // 16 KB: this CTA's 128 weight rows
 constexpr int SFA_BYTES = 4 * 512;             // scale blocks of this CTA's 128 rows, 4 k-steps
-constexpr int SFB_BYTES = 8 * 512;             // scale blocks of all 256 weight rows, 4 k-steps
+// The weight scales of a stage as the GEMM-ready copy holds them: per k-step
+// the two 512-byte scale blocks of the tile's 256 weight rows, replicated for
+// the four TMEM lane quadrants (128 rows x 32 bytes, row 32 q + l holding row
+// l of both blocks, K-major without swizzle: 8-row groups 256 bytes apart,
+// the two 16-byte halves 128 bytes apart), so that one tcgen05.cp 128x256b
+// per k-step moves them into TMEM.  The copy instructions, not their bytes,
+// are what occupy the tensor pipe: the alternative, two 32x128b.warpx4
+// copies per k-step from the 1 KB of plain blocks, costs twice as many.
+constexpr int SFB_KSTEP_BYTES = 4096;
+constexpr int SFB_BYTES = 4 * SFB_KSTEP_BYTES;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
 constexpr int kEpiWarps = 8;
 constexpr int kEpiWarp0 = 4;
@@ -99,11 +108,12 @@ constexpr int kLanesPerRole = 2;               // producer lanes per role, takin
 constexpr size_t SMEM_BYTES = 1024 + (size_t)kStages * STAGE_BYTES + 256;
 static_assert(SMEM_BYTES <= 227 * 1024, "stage ring does not fit in shared memory");
 // kEpiPlain, kEpiQkv: y leaves through TMA stores of 32 x 32 boxes staged
-// per epilogue warp in two 2 KB buffers (64-byte swizzle), 1 KB aligned
+// per epilogue warp in kYBufs 2 KB buffers (64-byte swizzle), 1 KB aligned
 // after the barriers.
 constexpr int kYStageBytes = 2048;
+constexpr int kYBufs = 1;
 constexpr size_t Y_STAGE_OFF = (size_t)kStages * STAGE_BYTES + 1024;
-constexpr size_t SMEM_BYTES_PLAIN = 1024 + Y_STAGE_OFF + (size_t)kEpiWarps * 2 * kYStageBytes;
+constexpr size_t SMEM_BYTES_PLAIN = 1024 + Y_STAGE_OFF + (size_t)kEpiWarps * kYBufs * kYStageBytes;
 static_assert(SMEM_BYTES_PLAIN <= 227 * 1024, "y staging buffers do not fit in shared memory");
 // kEpiGelu: twice the epilogue warps (four per TMEM lane quadrant, 64
 // columns each: the GELU epilogue is latency-bound, and more warps hide more
@@ -119,6 +129,44 @@ static_assert(SMEM_BYTES_GELU <= 227 * 1024, "GELU epilogue buffers do not fit i
 // Epilogue variants of the pair kernel (separate instantiations, so that the
 // plain kernel keeps its registers).
 enum : int { kEpiPlain = 0, kEpiQkv = 1, kEpiGelu = 2 };
+
+// Bytes of the GEMM-ready copy of the weight scales of an N x K weight:
+// 16 KB per (256-row tile, 256 columns of K), whole tiles.
+__host__ __device__ constexpr int64_t wscales_rep_bytes(int64_t N, int64_t K) {
+    return ((N + 255) / 256) * ((K + 255) / 256) * (int64_t)gp::SFB_BYTES;
+}
+
+// Writes the GEMM-ready copy (rep) of the weight scales from their block
+// layout (blocks: 512 bytes per 128 rows x 64 columns, row l of a block at
+// 16 l; kg4 = K / 64 blocks per row block, n_rb row blocks).  Unit (t, kb) =
+// 256-row tile t, k-steps 4 kb .. 4 kb + 3, at (t * n_kb + kb) * 16 KB; in
+// it k-step k at k * 4 KB holds, for each TMEM lane quadrant q and row l,
+// row l of blocks (2 t, 4 kb + k) and (2 t + 1, 4 kb + k) at
+// (4 q + l / 8) * 256 + (l % 8) * 16 and 128 bytes further.  Blocks past the
+// weight (a missing second row block, k-steps past K) are zeros.  One
+// thread per 16 bytes of the copy.
+__global__ void __launch_bounds__(256) replicate_weight_scales_kernel(const uint8_t* __restrict__ blocks,
+                                                                      uint8_t* __restrict__ rep, int n_rb, int kg4,
+                                                                      int n_kb, int64_t chunks) {
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= chunks) return;
+    const int64_t unit = i >> 10;
+    const int c = (int)(i & 1023);
+    const int k = c >> 8, g = (c & 255) >> 4, h = (c >> 3) & 1, l8 = c & 7;
+    const int l = 8 * (g & 3) + l8;
+    const int t = (int)(unit / n_kb), kb = (int)(unit - (int64_t)t * n_kb);
+    const int rb = 2 * t + h, kk = 4 * kb + k;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (rb < n_rb && kk < kg4) v = *reinterpret_cast<const uint4*>(blocks + ((int64_t)rb * kg4 + kk) * 512 + 16 * l);
+    reinterpret_cast<uint4*>(rep)[i] = v;
+}
+
+// Descriptor of one k-step of replicated weight scales (K-major, no swizzle:
+// 8-row groups 256 bytes apart, the two 16-byte halves 128 bytes apart).
+__device__ __forceinline__ uint64_t desc_sfb_kstep(uint32_t addr) {
+    return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)(128u >> 4) << 16) | ((uint64_t)(256u >> 4) << 32) |
+           ((uint64_t)1u << 46);
+}
 // The GELU epilogue runs four warps per TMEM lane quadrant (64 columns
 // each): its chain is latency-bound, and more warps hide more of it.  The
 // plain and QKV epilogues keep two (128 columns per warp; a QKV head's
@@ -150,15 +198,14 @@ enum : uint32_t {
 template <bool WITH_SFA>
 __device__ __forceinline__ void gp_issue_stage(uint32_t acc, uint64_t da, uint64_t db, uint64_t dfa, uint64_t dfb,
                                                uint32_t ta, uint32_t tb, uint32_t idesc, uint32_t acc0) {
+    constexpr uint64_t kSfbStep = (uint64_t)(gp::SFB_KSTEP_BYTES >> 4);   // descriptor units per k-step
     if (WITH_SFA) tmem_cp_32x128b_x4_pair(ta, dfa);
-    tmem_cp_32x128b_x4_pair(tb, dfb);
-    tmem_cp_32x128b_x4_pair(tb + 4u, dfb + 128u);
+    tmem_cp_128x256b_pair(tb, dfb);
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
         if (j < 3) {
             if (WITH_SFA) tmem_cp_32x128b_x4_pair(ta + 4u * (j + 1), dfa + 32u * (j + 1));
-            tmem_cp_32x128b_x4_pair(tb + 8u * (j + 1), dfb + 32u * (j + 1));
-            tmem_cp_32x128b_x4_pair(tb + 8u * (j + 1) + 4u, dfb + 128u + 32u * (j + 1));
+            tmem_cp_128x256b_pair(tb + 8u * (j + 1), dfb + kSfbStep * (j + 1));
         }
         mma_nvfp4_pair(acc, da + 2u * j, db + 2u * j, idesc, ta + 4u * j, tb + 8u * j, j == 0 ? acc0 : 1u);
     }
@@ -351,11 +398,11 @@ __device__ __forceinline__ void gp_pack32(const uint32_t (&acc)[128], int c2, co
 // One warp's 32 rows x 32 columns of y through a 2 KB staging buffer: each
 // lane writes its row (16-byte piece j at j ^ ((lane / 2) % 4), the 64-byte
 // swizzle of the y tensor map), then lane 0 stores the box at (n, row0) with
-// TMA.  Before writing, lane 0 waits until at most one earlier store of this
-// thread still reads shared memory (the warp alternates two buffers).
+// TMA.  Before writing, lane 0 waits until at most kYBufs - 1 earlier stores
+// of this thread still read shared memory (the warp cycles kYBufs buffers).
 __device__ __forceinline__ void gp_stage_store(const uint32_t (&pk)[16], uint32_t buf, uint32_t lane,
                                                const CUtensorMap* tm_y, int n, int row0, int M) {
-    if (lane == 0) bulk_wait_group_read<1>();
+    if (lane == 0) bulk_wait_group_read<gp::kYBufs - 1>();
     __syncwarp();
 #pragma unroll
     for (int j = 0; j < 4; ++j)
@@ -494,7 +541,8 @@ __global__ void __launch_bounds__(gp_threads<kEpi>(), 1)
                             if (leader)
                                 mbar_arrive_expect_tx(&full[s], 2u * ((need_sfa ? SFA_BYTES : 0) + SFB_BYTES));
                             if (need_sfa) tma_load_3d_pair(sfa, &tm_sfa, bar, 0, 4 * kb, 2 * m_tile + (int)rank);
-                            tma_load_3d_pair(sfb, &tm_sfb, bar, 0, 4 * kb, 2 * n_tile);   // both weight row blocks
+                            // the tile's replicated weight scales for these four k-steps (16 KB)
+                            tma_load_3d_pair(sfb, &tm_sfb, bar, 0, 0, n_tile * n_kb + kb);
                         }
                     } else {
                         const int c = (kk - n_kb) >> 1, part = (kk - n_kb) & 1;
@@ -547,7 +595,7 @@ __global__ void __launch_bounds__(gp_threads<kEpi>(), 1)
                         const uint32_t sa = smem0 + (uint32_t)s * STAGE_BYTES;
                         const uint64_t da = desc_sw128(sa), db = desc_sw128(sa + A_BYTES);   // + 2 per 32-byte K-step
                         const uint64_t dfa = desc_sf_block(sa + A_BYTES + B_BYTES);         // + 32 per 512 bytes
-                        const uint64_t dfb = dfa + (uint64_t)(SFA_BYTES >> 4);
+                        const uint64_t dfb = desc_sfb_kstep(sa + A_BYTES + B_BYTES + SFA_BYTES);
                         // activation-scale columns of this stage's K-steps, weight-scale set
                         const uint32_t ta = sfa_res ? tmem + SFA_RES + 16u * (uint32_t)kk
                                                     : tmem + SF_COL + SF_SET_COLS * (uint32_t)(it & 1);
@@ -562,8 +610,7 @@ __global__ void __launch_bounds__(gp_threads<kEpi>(), 1)
                             // a last stage of fewer than four K-steps
                             for (int j = 0; j < nks_last; ++j) {
                                 if (need_sfa) tmem_cp_32x128b_x4_pair(ta + 4u * j, dfa + 32u * j);
-                                tmem_cp_32x128b_x4_pair(tb + 8u * j, dfb + 32u * j);
-                                tmem_cp_32x128b_x4_pair(tb + 8u * j + 4u, dfb + 128u + 32u * j);
+                                tmem_cp_128x256b_pair(tb + 8u * j, dfb + (uint64_t)(SFB_KSTEP_BYTES >> 4) * j);
                                 mma_nvfp4_pair(tmem + ACC_COL, da + 2u * j, db + 2u * j, idesc_fp4, ta + 4u * j,
                                                tb + 8u * j, (kk > 0 || j > 0) ? 1u : 0u);
                             }
@@ -701,7 +748,7 @@ __global__ void __launch_bounds__(gp_threads<kEpi>(), 1)
             // buffers and a TMA store (gp_stage_store); rows past M and
             // columns past N are not written
             const uint32_t stage0 =
-                smem_u32(smem + Y_STAGE_OFF) + (uint32_t)(warp - kEpiWarp0) * (2u * kYStageBytes);
+                smem_u32(smem + Y_STAGE_OFF) + (uint32_t)(warp - kEpiWarp0) * (uint32_t)(kYBufs * kYStageBytes);
             const int row0 = (int)(grow - lane);
             if (kEpi == kEpiQkv && nbase < a.qk_cols) {
                 // this warp's 128 columns are one Q or K head of a to_qkv
@@ -755,7 +802,7 @@ __global__ void __launch_bounds__(gp_threads<kEpi>(), 1)
                             pk[8 * h + p] = *reinterpret_cast<const uint32_t*>(&hv);
                         }
                     }
-                    gp_stage_store(pk, stage0 + (uint32_t)(c2 & 1) * kYStageBytes, lane, &tm_y, nbase + 32 * c2,
+                    gp_stage_store(pk, stage0 + (uint32_t)(c2 % kYBufs) * kYStageBytes, lane, &tm_y, nbase + 32 * c2,
                                    row0, a.M);
                 }
                 continue;
@@ -766,7 +813,7 @@ __global__ void __launch_bounds__(gp_threads<kEpi>(), 1)
                 if (n >= a.N) break;   // warp-uniform
                 uint32_t pk[16];
                 gp_pack32(acc, c2, a, S, n, pk);
-                gp_stage_store(pk, stage0 + (uint32_t)(c2 & 1) * kYStageBytes, lane, &tm_y, n, row0, a.M);
+                gp_stage_store(pk, stage0 + (uint32_t)(c2 % kYBufs) * kYStageBytes, lane, &tm_y, n, row0, a.M);
             }
         }
     }

@@ -167,6 +167,11 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// Cluster-scope acquire/release fence: after a wait on an mbarrier that
+// another CTA of the cluster arrived on (with release.cluster), makes that
+// CTA's earlier writes ordered before this thread's later operations.
+__device__ __forceinline__ void fence_acq_rel_cluster() { asm volatile("fence.acq_rel.cluster;" ::: "memory"); }
+
 // Tiled TMA store shared -> global of one box at (x, y) (x * element size a
 // multiple of 16 bytes, x and y >= 0; the parts outside the tensor are not
 // written), tracked in this thread's bulk async-group.
@@ -482,6 +487,13 @@ __device__ __forceinline__ void mma_bf16_pair(uint32_t d_tmem, uint64_t a_desc, 
 }
 __device__ __forceinline__ void tmem_cp_32x128b_x4_pair(uint32_t taddr, uint64_t sdesc) {
     asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+// 128 lanes x 256 bits (eight 32-bit columns per lane) from a K-major
+// no-swizzle source: row i of the source lands in lane i.  Each CTA of the
+// pair copies its own shared memory into its own TMEM.
+__device__ __forceinline__ void tmem_cp_128x256b_pair(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::2.128x256b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 
 // Two fp32 from the shared memory of a CTA of the cluster (shared::cluster address).

@@ -25,7 +25,7 @@
 namespace svdq {
 namespace {
 
-constexpr int kAbiVersion = 1;
+constexpr int kAbiVersion = 2;
 
 // ------------------------------------------------------------- validation
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -255,6 +255,16 @@ svdq_status fold_lowrank(const float* lambda, const void* L_down, const void* L_
     return launch_status("fold_lowrank_kernel");
 }
 
+// The GEMM-ready copy of nvfp4 weight scales, right after their block layout.
+svdq_status replicate_weight_scales(void* w_scales, int64_t N, int64_t K, cudaStream_t st) {
+    const int64_t rows_pad = round_up(N, 128);
+    const int64_t chunks = wscales_rep_bytes(N, K) / 16;
+    replicate_weight_scales_kernel<<<(unsigned)((chunks + 255) / 256), 256, 0, st>>>(
+        reinterpret_cast<const uint8_t*>(w_scales), reinterpret_cast<uint8_t*>(w_scales) + rows_pad * K / 16,
+        (int)(rows_pad / 128), (int)(K / 64), (int)((K + 255) / 256), chunks);
+    return launch_status("replicate_weight_scales_kernel");
+}
+
 svdq_status pack_weight_nvfp4(const void* R, int64_t N, int64_t K, void* w_codes, void* w_scales,
                               float* w_tensor_scale, cudaStream_t st) {
     SVDQ_TRY(tensor_scale_prepass(R, nullptr, N, K, w_tensor_scale, st));
@@ -263,7 +273,8 @@ svdq_status pack_weight_nvfp4(const void* R, int64_t N, int64_t K, void* w_codes
     quantize_rows_nvfp4_kernel<<<(unsigned)((work + 255) / 256), 256, 0, st>>>(
         reinterpret_cast<const __nv_bfloat16*>(R), N, rows_pad, K, w_tensor_scale,
         reinterpret_cast<uint8_t*>(w_codes), reinterpret_cast<uint8_t*>(w_scales));
-    return launch_status("quantize_rows_nvfp4_kernel");
+    SVDQ_TRY(launch_status("quantize_rows_nvfp4_kernel"));
+    return replicate_weight_scales(w_scales, N, K, st);
 }
 
 // K-split of the activation quantizer: enough CTAs for about one wave on a
@@ -566,7 +577,9 @@ svdq_status gemm_nvfp4_pair(const void* x_codes, const void* x_scales, const flo
         !make_map(&tm_wc, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_codes, (uint64_t)K / 2, (uint64_t)N, (uint64_t)K / 2,
                   gp::BK_BYTES, 128) ||
         !make_sf_map(&tm_sfa, x_scales, (uint64_t)((M + 127) / 128), (uint64_t)kg4, 1) ||
-        !make_sf_map(&tm_sfb, w_scales, (uint64_t)((N + 127) / 128), (uint64_t)kg4, 2))
+        // the GEMM-ready copy after the block layout: 32 rows of 512 bytes per 16 KB unit
+        !make_sf_map(&tm_sfb, reinterpret_cast<const uint8_t*>(w_scales) + round_up(N, 128) * K / 16,
+                     (uint64_t)(wscales_rep_bytes(N, K) / gp::SFB_BYTES), 32, 1, 32))
         return SVDQ_ERR_CUDA;
     if (rank > 0) {
         if (!make_map_3d(&tm_L, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, lowrank, (uint64_t)rank, (uint64_t)M, 2,
@@ -787,6 +800,7 @@ svdq_status svdq_buffer_sizes(svdq_precision p, int64_t rows, int64_t K, int ran
     out->codes_bytes = (size_t)(rows * K / 2);
     out->scales_bytes = p == SVDQ_NVFP4 ? (size_t)(rows_pad * K / 16) : (size_t)(2 * rows_pad * K / 64);
     out->lowrank_bytes = (size_t)(4 * rows * rank);   // hi and lo bf16 planes
+    out->w_scales_bytes = out->scales_bytes + (p == SVDQ_NVFP4 ? (size_t)wscales_rep_bytes(rows, K) : 0);
     return SVDQ_OK;
 }
 
@@ -815,6 +829,14 @@ svdq_status svdq_pack_weight(svdq_precision p, int group_size, const void* R, in
     SVDQ_TRY(fold_lowrank(lambda, L_down, L_up, N, K, rank, inv_lambda, L_down_t, L_up_t, st));
     if (p == SVDQ_NVFP4) return pack_weight_nvfp4(R, N, K, w_codes, w_scales, w_tensor_scale, st);
     return int4_quantize_rows(R, N, K, w_codes, w_scales, st);
+}
+
+svdq_status svdq_replicate_weight_scales(void* w_scales, int64_t N, int64_t K, svdq_stream_t stream) {
+    SVDQ_TRY(check_dims(N, K));
+    if (N % 16 != 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;
+    SVDQ_TRY(check_ptr(w_scales));
+    SVDQ_TRY(check_device());
+    return replicate_weight_scales(w_scales, N, K, reinterpret_cast<cudaStream_t>(stream));
 }
 
 svdq_status svdq_quantize_act_workspace_bytes(svdq_precision p, int64_t M, int64_t K, int rank, size_t* bytes) {

@@ -57,7 +57,7 @@ def pack_weight(R: torch.Tensor, lam: torch.Tensor, L_down: torch.Tensor | None,
     dev = R.device
     sz = _lib.svdq_buffer_sizes(precision, N, K, rank)
     w_codes = _empty(sz["codes_bytes"], dev)
-    w_scales = _empty(sz["scales_bytes"], dev)
+    w_scales = _empty(sz["w_scales_bytes"], dev)   # nvfp4: block layout, then the GEMM-ready copy
     w_ts = torch.empty(4, dtype=torch.float32, device=dev) if precision == "nvfp4" else None
     inv_lambda = torch.empty(K, dtype=torch.float32, device=dev)
     L_down_t = torch.empty(2, rank, K, dtype=torch.bfloat16, device=dev) if rank else None

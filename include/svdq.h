@@ -42,6 +42,15 @@
  *            multiple of 128 with zero bytes, in the tensor-core scale-factor
  *            layout: with Kg4 = K/64, the byte of (row r, group g) is at
  *              ((r/128)*Kg4 + g/4)*512 + (r%32)*16 + ((r%128)/32)*4 + g%4.
+ *  - nvfp4 weight scales (w_scales of a packed weight, w_scales_bytes): the
+ *            block layout above, then a GEMM-ready copy of the same bytes for
+ *            the tensor-memory copy unit: with Nt = ceil(N/256), Kb =
+ *            ceil(K/256), unit (t, kb) of 16 KB at (t*Kb + kb)*16384 holds
+ *            k-steps 4kb..4kb+3; in k-step k (at k*4096) the 16 bytes of row
+ *            l (0..31) of block (2t+h, 4kb+k) sit at
+ *            (4q + l/8)*256 + h*128 + (l%8)*16 for every q in 0..3 (the
+ *            four 32-lane quarters of tensor memory); blocks past the weight
+ *            are zero.  svdq_pack_weight writes both parts.
  *  - int4 scales: one bf16 per (row, group of 64), group-major:
  *            scales[g * rows_pad + r] with rows_pad = rows rounded up to 128
  *            (padding rows are zero).
@@ -89,6 +98,10 @@ typedef struct {
     size_t codes_bytes;    /* rows * K / 2 */
     size_t scales_bytes;   /* nvfp4: rows_pad * K / 16;  int4: 2 * rows_pad * K / 64 */
     size_t lowrank_bytes;  /* 4 * rows * rank (rank-r activations: hi and lo bf16 planes) */
+    size_t w_scales_bytes; /* a packed weight's w_scales: int4: scales_bytes; nvfp4: scales_bytes of
+                              the block layout, then the GEMM's tile-replicated copy of the same
+                              scales, 16 KB per 256 rows x 256 columns (rows and K rounded up to
+                              multiples of 256) */
 } svdq_sizes;
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -112,7 +125,7 @@ svdq_status svdq_buffer_sizes(svdq_precision precision, int64_t rows, int64_t K,
  *   L_down     device bf16 [K, rank] (may be NULL when rank == 0)
  *   L_up       device bf16 [rank, N] (may be NULL when rank == 0)
  * Outputs (device, caller-allocated):
- *   w_codes [N, K/2]; w_scales (scales_bytes for N rows); w_tensor_scale fp32[1]
+ *   w_codes [N, K/2]; w_scales (w_scales_bytes for N rows); w_tensor_scale fp32[1]
  *   (nvfp4: S_w = amax|R| / 2688, or 1 when R == 0; int4: may be NULL);
  *   inv_lambda fp32 [K]; L_down_t bf16 [2, rank, K]; L_up_t bf16 [N, rank].
  * group_size must be 16 for SVDQ_NVFP4 and 64 for SVDQ_INT4. */
@@ -122,6 +135,16 @@ svdq_status svdq_pack_weight(svdq_precision precision, int group_size,
                              void* w_codes, void* w_scales, float* w_tensor_scale,
                              float* inv_lambda, void* L_down_t, void* L_up_t,
                              svdq_stream_t stream);
+
+/* Writes the GEMM-ready copy of nvfp4 weight scales (the second part of a
+ * packed weight's w_scales, see "nvfp4 weight scales" above) from the block
+ * layout in its first scales_bytes bytes.  svdq_pack_weight does this itself;
+ * this call is for weight scales produced another way (for example by
+ * svdq_quantize_act on the weight) and copied into such a buffer.
+ *   w_scales   device, w_scales_bytes for N rows (svdq_buffer_sizes, nvfp4)
+ * Errors: INVALID_ARG (NULL or misaligned w_scales), UNSUPPORTED_SHAPE (as
+ * svdq_pack_weight), UNSUPPORTED_DEVICE, CUDA. */
+svdq_status svdq_replicate_weight_scales(void* w_scales, int64_t N, int64_t K, svdq_stream_t stream);
 
 /* Bytes of the workspace svdq_quantize_act needs for this shape (0 when it
  * needs none).  When K is split across several CTAs, each computes a partial

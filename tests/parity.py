@@ -35,6 +35,21 @@ def nvfp4_scale_padding_is_zero(buf: np.ndarray, rows: int, K: int) -> bool:
     return not np.asarray(buf, np.uint8).reshape(-1)[idx].any()
 
 
+def replicate_nvfp4_weight_scales(buf: np.ndarray, N: int, K: int) -> np.ndarray:
+    """The GEMM-ready copy of nvfp4 weight scales (the C header's "nvfp4 weight
+    scales" layout) built from the block layout at the start of `buf`: per
+    256-row tile t and 256 columns kb, per k-step k, each 16-byte row l of the
+    blocks (2t+h, 4kb+k) four times, at (4q + l/8)*256 + h*128 + (l%8)*16."""
+    kg4, n_rb = K // 64, (N + 127) // 128
+    n_t, n_kb = (N + 255) // 256, (K + 255) // 256
+    blocks = np.zeros((2 * n_t, 4 * n_kb, 32, 16), np.uint8)
+    blocks[:n_rb, :kg4] = np.asarray(buf, np.uint8).reshape(-1)[: n_rb * kg4 * 512].reshape(n_rb, kg4, 32, 16)
+    b = blocks.reshape(n_t, 2, n_kb, 4, 4, 8, 16)                 # t, h, kb, k, l/8, l%8, byte
+    b = b.transpose(0, 2, 3, 4, 1, 5, 6)                          # t, kb, k, l/8, h, l%8, byte
+    rep = np.broadcast_to(b[:, :, :, None], (n_t, n_kb, 4, 4, 4, 2, 8, 16))   # q before l/8
+    return np.ascontiguousarray(rep).reshape(-1)
+
+
 def unswizzle_int4_scales(buf: np.ndarray, rows: int, K: int) -> np.ndarray:
     """int4 scales are bf16, group-major: element (r, g) at g * rows_pad + r."""
     rows_pad = (rows + 127) // 128 * 128
@@ -141,6 +156,8 @@ def check_case(case: W.Case, rows=None, x_tensor_scale=None, with_bias=True, inp
         assert np.array_equal(unswizzle_nvfp4_scales(ws, N, K), ref.w_scales), "weight scales"
         assert np.array_equal(unswizzle_nvfp4_scales(xs, M, K), ref.x_scales), "activation scales"
         assert nvfp4_scale_padding_is_zero(ws, N, K) and nvfp4_scale_padding_is_zero(xs, M, K)
+        sb = (N + 127) // 128 * 128 * K // 16
+        assert np.array_equal(ws[sb:], replicate_nvfp4_weight_scales(ws, N, K)), "GEMM-ready weight scales"
         prescale = float(np.float32(ref.S_x) * np.float32(ref.S_w))
     else:
         assert np.array_equal(unswizzle_int4_scales(packed.w_scales.cpu().numpy(), N, K), ref.w_scales)

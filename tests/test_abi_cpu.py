@@ -35,7 +35,7 @@ def test_every_declared_symbol_is_exported(L):
 
 
 def test_abi_version_and_strings(L):
-    assert L.svdq_abi_version() == 1
+    assert L.svdq_abi_version() == 2
     for st in range(6):
         assert L.status_string(st)
     assert "unsupported device" in L.status_string(L.SVDQ_ERR_UNSUPPORTED_DEVICE)
@@ -43,11 +43,14 @@ def test_abi_version_and_strings(L):
 
 def test_buffer_sizes(L):
     s = L.svdq_buffer_sizes("nvfp4", 4608, 3072, 32)
-    assert s == {"codes_bytes": 4608 * 1536, "scales_bytes": 4608 * 192, "lowrank_bytes": 4608 * 128}
+    # a packed weight's scales: the block layout, then 16 KB per 256 x 256 tile of the GEMM-ready copy
+    assert s == {"codes_bytes": 4608 * 1536, "scales_bytes": 4608 * 192, "lowrank_bytes": 4608 * 128,
+                 "w_scales_bytes": 4608 * 192 + 18 * 12 * 16384}
     s = L.svdq_buffer_sizes("nvfp4", 200, 320, 16)          # rows padded to 256 for the scales
-    assert s["scales_bytes"] == 256 * 20
+    assert s["scales_bytes"] == 256 * 20 and s["w_scales_bytes"] == 256 * 20 + 1 * 2 * 16384
     s = L.svdq_buffer_sizes("int4", 200, 320, 0)
     assert s["scales_bytes"] == 2 * 256 * 5 and s["lowrank_bytes"] == 0
+    assert s["w_scales_bytes"] == s["scales_bytes"]
     for bad in [("nvfp4", 0, 64, 0), ("nvfp4", 8, 96, 0), ("nvfp4", 8, 0, 0)]:
         with pytest.raises(L.SvdqError) as e:
             L.svdq_buffer_sizes(*bad)

@@ -124,14 +124,17 @@ def test_grid_exact_unit_scales():
     inp = {"x": on_grid(M), "R": on_grid(N), "lam": torch.ones(K), "L_down": None, "L_up": None,
            "b": torch.from_numpy(rng.standard_normal(N).astype(np.float32)).to(torch.bfloat16)}
     inp["R"] = inp["R"]
-    from bit_w4a4_quantized_token_b200 import layer
+    from bit_w4a4_quantized_token_b200 import _lib, layer
 
     d = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
     packed = layer.pack_weight(d["R"], d["lam"], None, None, d["b"])
     packed.w_tensor_scale.fill_(1.0)      # static unit scales on both sides
     # re-quantize the weight with S_w = 1: quantize it as an activation with lambda = 1
     wq = layer.quantize_act(d["R"], packed, x_tensor_scale=1.0)
-    packed.w_codes, packed.w_scales = wq.x_codes, wq.x_scales
+    packed.w_codes = wq.x_codes
+    packed.w_scales.zero_()
+    packed.w_scales[: wq.x_scales.numel()].copy_(wq.x_scales.view(-1))
+    _lib.svdq_replicate_weight_scales(packed.w_scales, N, K)
     q = layer.quantize_act(d["x"], packed, x_tensor_scale=1.0)
     y = layer.gemm(q, packed)
     xv = inp["x"].double().numpy()
