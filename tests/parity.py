@@ -74,7 +74,8 @@ def bf16_half_ulp(v: np.ndarray) -> np.ndarray:
     return np.exp2(np.floor(np.log2(a)) - 8)
 
 
-def check_y(y_gpu_bits: np.ndarray, y_ref: np.ndarray, y_ref_bits: np.ndarray, what: str = "y") -> dict:
+def check_y(y_gpu_bits: np.ndarray, y_ref: np.ndarray, y_ref_bits: np.ndarray, what: str = "y",
+            min_frac1: float = 0.999) -> dict:
     """The output bar.
 
     1. max_i (|y_gpu - y_ref| - half_ulp_bf16(y_ref)) <= 1e-2 rms(y_ref): the
@@ -83,7 +84,8 @@ def check_y(y_gpu_bits: np.ndarray, y_ref: np.ndarray, y_ref_bits: np.ndarray, w
        the largest outputs is itself more than 1 % of the rms, so the bound
        cannot apply to the rounding of the bf16 store.)
     2. the bf16 output is within 1 ulp of the oracle's own bf16 rounding of
-       y_ref on >= 99.9 % of the elements.
+       y_ref on >= min_frac1 of the elements (99.9 % for a layer given the
+       same inputs as the oracle).
     """
     y_gpu = (np.asarray(y_gpu_bits, np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
     assert np.all(np.isfinite(y_gpu)), f"{what}: non-finite outputs"
@@ -95,7 +97,7 @@ def check_y(y_gpu_bits: np.ndarray, y_ref: np.ndarray, y_ref_bits: np.ndarray, w
     stats = {"rms": rms, "max_abs_err": float(err.max()), "max_excess_over_half_ulp_rel_rms": excess / rms,
              "frac_within_1ulp": frac1, "max_ulps": int(ulps.max())}
     assert excess <= 1e-2 * rms, f"{what}: {stats}"
-    assert frac1 >= 0.999, f"{what}: {stats}"
+    assert frac1 >= min_frac1, f"{what}: {stats}"
     return stats
 
 

@@ -9,8 +9,15 @@ epilogue applies GELU and performs fc2's activation step itself.  Checks:
   svdq_gelu -> svdq_quantize_act with the same static scale): identical
   nvfp4 codes and scales, bit for bit, and the rank-r activations to the
   precision of two fp32 summation orders;
-* fc2's output after the fused path against the oracle's fp64 chain, at the
-  linear layer's bf16 bar, plus its rank-r activations at the usual 1e-2;
+* fc2's output after the fused path against the oracle's fc2 applied to the
+  GPU's own h (the same input bits: its codes and scales bit for bit, the
+  output at the linear layer's bf16 bar), plus its rank-r activations at the
+  usual 1e-2;
+* the same output against the oracle's whole fp64 chain from x: fc1's bf16
+  outputs, and so h and fc2's codes, may differ from the oracle's where two
+  correct fp32 summation orders round differently (the codes agree on >= 99 %
+  of the elements), so there only the 1 %-of-rms bound holds on every element
+  and the 1-ulp agreement is asked of >= 99 % of them;
 * the workspace of partial sums is left zeroed.
 """
 import numpy as np
@@ -80,7 +87,27 @@ def _run(M, D, Hd, r1, r2, approx, rows=None, cal_rows=None):
     torch.cuda.synchronize()
     assert float(ws.abs().max()) == 0.0, "workspace not left zeroed"
     r1o, ho, r2o = O.gelu_mlp(x_bits, fc1, fc2, S1, S2, approx, rows=rows)
-    return dict(qf=qf, qu=qu, y2f=y2f, y2u=y2u, y1=y1, h=h, r1o=r1o, ho=ho, r2o=r2o, S1=S1, S2=S2, p2=p2)
+    # fc2 alone on the GPU's h (the unfused pass's bits; the fused path hands fc2 the same codes)
+    h_rows = u16(h) if rows is None else u16(h)[np.asarray(rows)]
+    r2c = O.svdq_linear("nvfp4", np.ascontiguousarray(h_rows), fc2["lam"], fc2["R"], fc2["L_down"], fc2["L_up"],
+                        fc2["b"], S_x=S2)
+    return dict(qf=qf, qu=qu, y2f=y2f, y2u=y2u, y1=y1, h=h, r1o=r1o, ho=ho, r2o=r2o, r2c=r2c, S1=S1, S2=S2, p2=p2)
+
+
+def _check_fc2(o, M, Hd, r2, rows=None):
+    """fc2 after the fused path: against the oracle on the GPU's own h (same
+    inputs, the layer's bar) and against the oracle's chain from x."""
+    qf, r2c, r2o = o["qf"], o["r2c"], o["r2o"]
+    sel = np.arange(M) if rows is None else np.asarray(rows)
+    codes = qf.x_codes[: M * Hd // 2].cpu().numpy().reshape(M, Hd // 2)[sel]
+    scales = unswizzle_nvfp4_scales(qf.x_scales.cpu().numpy(), M, Hd)[sel]
+    assert np.array_equal(codes, r2c.x_codes), "fc2 codes differ from the oracle's on the same h"
+    assert np.array_equal(scales, r2c.x_scales), "fc2 scales differ from the oracle's on the same h"
+    y = u16(o["y2f"])[sel]
+    check_y(y, r2c.y, r2c.y_bf16, "fc2 output, oracle on the same h")
+    assert np.mean(codes == r2o.x_codes) >= 0.99
+    assert np.mean(scales == r2o.x_scales) >= 0.99
+    check_y(y, r2o.y, r2o.y_bf16, "fc2 output, oracle chain from x", min_frac1=0.99)
 
 
 SMALL = [
@@ -108,15 +135,10 @@ def test_fused_mlp_small(M, D, Hd, r1, r2, approx):
         b = (qu.lowrank_act[0].double() + qu.lowrank_act[1].double())
         rel = float((a - b).norm() / b.norm().clamp_min(1e-30))
         assert rel <= 1e-5, rel
-    # against the oracle's chain
-    r2o = o["r2o"]
-    codes = qf.x_codes[:nb].cpu().numpy().reshape(M, Hd // 2)
-    scales = unswizzle_nvfp4_scales(qf.x_scales.cpu().numpy(), M, Hd)
-    assert np.mean(codes == r2o.x_codes) >= 0.99
-    assert np.mean(scales == r2o.x_scales) >= 0.99
     if r2:
-        check_lowrank(qf.lowrank_act, r2o.L, float(np.float32(o["S2"]) * np.float32(float(o["p2"].w_tensor_scale[0]))))
-    check_y(u16(o["y2f"]), r2o.y, r2o.y_bf16, "fc2 output after the fused path")
+        check_lowrank(qf.lowrank_act, o["r2c"].L,
+                      float(np.float32(o["S2"]) * np.float32(float(o["p2"].w_tensor_scale[0]))))
+    _check_fc2(o, M, Hd, r2)
 
 
 def test_gelu_pass_matches_oracle_on_every_bf16():
@@ -154,10 +176,7 @@ def test_fused_mlp_full_size_sampled_rows():
     qf, qu = o["qf"], o["qu"]
     assert torch.equal(qf.x_codes[:4608 * 6144], qu.x_codes[:4608 * 6144])
     assert torch.equal(qf.x_scales, qu.x_scales)
-    r2o = o["r2o"]
-    codes = qf.x_codes[:4608 * 6144].cpu().numpy().reshape(4608, 6144)[rows]
-    assert np.mean(codes == r2o.x_codes) >= 0.99
-    check_y(u16(o["y2f"])[rows], r2o.y, r2o.y_bf16, "fc2 output after the fused path, full size")
+    _check_fc2(o, 4608, 12288, 32, rows=rows)
 
 
 def test_fused_mlp_argument_checks():
