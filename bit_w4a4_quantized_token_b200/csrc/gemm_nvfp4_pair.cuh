@@ -7,26 +7,24 @@
 // tile belongs to a cluster of two CTAs on neighbouring SMs:
 //   * CTA r (r = 0, 1) loads rows 128 r .. 128 r + 127 of the tile's activation
 //     codes and rows 128 r .. 128 r + 127 of its weight codes, the scale block
-//     of its own 128 activation rows and the scale blocks of all 256 weight
-//     rows (the tensor core reads the weight scales of every column in both
-//     halves of the pair);
-//   * one thread of CTA 0 copies the scale blocks into both CTAs' TMEM and
-//     issues one M = 256, N = 256 MMA per 64 values of K, each copy right
-//     before the MMA ahead of the one that reads it; the accumulator rows of
-//     CTA r sit in CTA r's TMEM;
+//     of its own 128 activation rows and the GEMM-ready copy of the weight
+//     scales of all 256 columns (the tensor core reads the weight scales of
+//     every column in both halves of the pair; the copy holds them replicated
+//     for the four TMEM lane quarters, so one tcgen05.cp 128x256b per 64
+//     values of K moves them);
+//   * two warps of CTA 0 take the stages in turn; in each, one thread copies
+//     the scales into both CTAs' TMEM and issues one M = 256, N = 256 MMA per
+//     64 values of K, each copy right before the MMA ahead of the one that
+//     reads it; the accumulator rows of CTA r sit in CTA r's TMEM;
 //   * every load of either CTA completes on CTA 0's stage barrier, CTA 0's
 //     commits arrive on both CTAs' "stage free" and "accumulator full"
 //     barriers, and both CTAs' epilogue warps hand the accumulator back on
-//     CTA 0's barrier;
-//   * a fourth warp of CTA 0 waits on the stage and accumulator barriers and
-//     meets the MMA warp at named barriers, so that the thread issuing the
-//     copies never touches shared memory while they are in flight (3-5 %
-//     faster than testing the mbarriers itself).
+//     CTA 0's barrier.
 // Against 128 x 256 tiles on single CTAs this halves the weight-code bytes
-// each SM loads per FLOP and the number of scale-block copies per FLOP; with
-// the activation scales resident in TMEM (K <= 3072, below) two copies per
-// MMA remain, and those copies, not the loads, set the pace.
-//
+// each SM loads per FLOP and the number of scale copies per FLOP; with the
+// activation scales resident in TMEM (K <= 3072, below) one copy per MMA
+// remains.
+
 // All scale blocks arrive by TMA (maps over the 512-byte blocks) so that the
 // peer CTA's loads can complete on CTA 0's barrier; a box that runs past the
 // end of a scale buffer is zero-filled, which only ever feeds rows or K-steps
@@ -80,11 +78,9 @@ constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
 constexpr int kEpiWarps = 8;
 constexpr int kEpiWarp0 = 4;
 constexpr int kThreads = 32 * (kEpiWarp0 + kEpiWarps);
-constexpr uint32_t kMmaWarp = 2;
-constexpr uint32_t kWaitWarp = 3;              // waits on the mbarriers for the MMA warp
-constexpr uint32_t kBarStage0 = 2;             // named barriers 2 .. 2 + kStages - 1: stage s ready
-constexpr uint32_t kBarAcc = 7;                // named barrier: accumulator free
-static_assert(kBarStage0 + kStages <= kBarAcc, "named barriers overlap");   // 0: __syncthreads, 1: GELU epilogue
+constexpr uint32_t kMmaWarp = 2;               // MMA issuers: warps 2 and 3 (even and odd stages)
+constexpr uint32_t kMmaWarp2 = 3;
+constexpr uint32_t kBarTurn0 = 2;              // named barriers 2, 3: the turn of warp 2, 3 (0: __syncthreads, 1: GELU epilogue)
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COL = 0;
 // Scale factors in TMEM.  Stages alternate between two "scale sets"; one of
@@ -416,19 +412,6 @@ __device__ __forceinline__ void gp_stage_store(const uint32_t (&pk)[16], uint32_
     }
 }
 
-// The MMA warp and the barrier-waiting warp meet at named barrier `id` (64
-// threads); returns the OR of their flags (the waiter's "gave up").
-__device__ __forceinline__ bool gp_meet(uint32_t id, uint32_t flag) {
-    uint32_t out;
-    asm volatile(
-        "{\n\t.reg .pred q, p;\n\tsetp.ne.u32 q, %1, 0;\n\tbar.red.or.pred p, %2, 64, q;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(out)
-        : "r"(flag), "r"(id)
-        : "memory");
-    return out != 0;
-}
-
 // kEpi: kEpiPlain, kEpiQkv (the fused QKV + RMSNorm + RoPE epilogue) or
 // kEpiGelu (the fused GELU + next-layer activation epilogue).
 template <int kEpi>
@@ -466,7 +449,7 @@ __global__ void __launch_bounds__(gp_threads<kEpi>(), 1)
             mbar_init(&full[s], kFullArrivals);
             mbar_init(&empty[s], 1);
         }
-        mbar_init(acc_full, 1);
+        mbar_init(acc_full, 2);   // both MMA warps commit at the end of every tile
         mbar_init(acc_empty, 2u * (uint32_t)gp_epi_warps<kEpi>());   // both CTAs' epilogue warps
         for (int s = 0; s < kStages; ++s) s_issued[s] = 0;
         s_failed = 0;
@@ -560,120 +543,88 @@ __global__ void __launch_bounds__(gp_threads<kEpi>(), 1)
                 }
             }
         }
-    } else if (warp == kMmaWarp) {
+    } else if (warp == kMmaWarp || warp == kMmaWarp2) {
         // ------------------------------------------ copies + MMAs (CTA 0 only)
-        // The whole warp walks the stages and meets the waiting warp at a
-        // named barrier per stage; lane 0 issues the copies and MMAs.  The
-        // issuing thread never tests an mbarrier itself: a shared-memory
-        // access by a thread with scale-block copies in flight waits for
-        // them, which drained the tensor pipe at every stage.
+        // Two warps take the stages in turn (warp kMmaWarp the even ones, in
+        // the order of the whole run), each waiting on its own stage and
+        // accumulator barriers; lane 0 issues the copies and MMAs.  Issue
+        // blocks while the tensor pipe's queue is full, so a single issuer
+        // left the pipe idle for the commit, the loop and the next wait at
+        // every stage; with two, one warp's bookkeeping overlaps the other's
+        // issue.  They hand the turn over through two named barriers (the
+        // owner of stage i arrives after issuing it; the other warp syncs
+        // before stage i + 1), so the MMAs reach the pipe in stage order and
+        // the accumulation order is fixed.  Both warps commit to acc_full at
+        // the end of every tile (it counts two arrivals).
         if (rank == 0) {
+            const uint32_t me = warp - kMmaWarp;   // 0: even stages, 1: odd stages
             const uint32_t idesc_fp4 = idesc_m(idesc_nvfp4(BN), BM);
             const uint32_t idesc_lr = idesc_m(idesc_bf16_f32(BN), BM);
             const uint32_t smem0 = smem_u32(smem);
             const int nks_last = a.kg4 - 4 * (n_kb - 1);   // K-steps in the last stage (1..4)
             bool ok = true;
-            int local = 0, s = 0, it = 0;
-            uint32_t ph = 0;
+            int local = 0, it = 0;
             for (int tile = t_begin; tile < t_end && ok; ++tile, ++local) {
                 const int n_tile = tile % a.n_tiles;
                 const bool need_sfa = !sfa_res || tile == t_begin || n_tile == 0;
-                if (gp_meet(kBarAcc, 0u)) {
-                    s_failed = 1;
-                    break;
-                }
-                if (lane == 0) tc_fence_after();
-                // FP4 stages
-                for (int kk = 0; kk < n_kb; ++kk, ++it) {
-                    if (gp_meet(kBarStage0 + (uint32_t)s, 0u)) {
-                        ok = false;
-                        s_failed = 1;
-                        break;
-                    }
-                    if (lane == 0) {
+                for (int kk = 0; kk < per_tile; ++kk, ++it) {
+                    if ((uint32_t)(it & 1) != me) continue;
+                    const int s = it % kStages;
+                    const uint32_t ph = (uint32_t)(it / kStages) & 1u;
+                    bool fail = !mbar_wait(&full[s], ph, kSiteGpFull);
+                    if (!fail && kk == 0) fail = !mbar_wait(acc_empty, ((uint32_t)local & 1u) ^ 1u, kSiteGpAccEmpty);
+                    if (fail) s_failed = 1;
+                    // warp-uniform, so that the whole warp takes the same barriers
+                    fail = __any_sync(0xffffffffu, fail || *reinterpret_cast<volatile int*>(&s_failed) != 0);
+                    // everything but the issue itself before the turn comes
+                    const uint32_t sa = smem0 + (uint32_t)s * STAGE_BYTES;
+                    const uint64_t da = desc_sw128(sa), db = desc_sw128(sa + A_BYTES);   // + 2 per 32-byte K-step
+                    const uint64_t dfa = desc_sf_block(sa + A_BYTES + B_BYTES);          // + 32 per 512 bytes
+                    const uint64_t dfb = desc_sfb_kstep(sa + A_BYTES + B_BYTES + SFA_BYTES);
+                    // activation-scale columns of this stage's K-steps, weight-scale set
+                    const uint32_t ta = sfa_res ? tmem + SFA_RES + 16u * (uint32_t)kk : tmem + SF_COL + SF_SET_COLS * me;
+                    const uint32_t tb = sfa_res ? tmem + SFB_RES + 32u * me : ta + 16u;
+                    const uint32_t acc0 = kk > 0 ? 1u : 0u;
+                    if (it > 0) named_bar_sync(kBarTurn0 + me, 64);   // the other warp has issued stage it - 1
+                    if (!fail && lane == 0) {
                         tc_fence_after();
-                        const uint32_t sa = smem0 + (uint32_t)s * STAGE_BYTES;
-                        const uint64_t da = desc_sw128(sa), db = desc_sw128(sa + A_BYTES);   // + 2 per 32-byte K-step
-                        const uint64_t dfa = desc_sf_block(sa + A_BYTES + B_BYTES);         // + 32 per 512 bytes
-                        const uint64_t dfb = desc_sfb_kstep(sa + A_BYTES + B_BYTES + SFA_BYTES);
-                        // activation-scale columns of this stage's K-steps, weight-scale set
-                        const uint32_t ta = sfa_res ? tmem + SFA_RES + 16u * (uint32_t)kk
-                                                    : tmem + SF_COL + SF_SET_COLS * (uint32_t)(it & 1);
-                        const uint32_t tb = sfa_res ? tmem + SFB_RES + 32u * (uint32_t)(it & 1) : ta + 16u;
-                        const uint32_t acc0 = kk > 0 ? 1u : 0u;
-                        if (kk + 1 < n_kb || nks_last == 4) {
-                            if (need_sfa)
-                                gp_issue_stage<true>(tmem + ACC_COL, da, db, dfa, dfb, ta, tb, idesc_fp4, acc0);
-                            else
-                                gp_issue_stage<false>(tmem + ACC_COL, da, db, dfa, dfb, ta, tb, idesc_fp4, acc0);
-                        } else {
-                            // a last stage of fewer than four K-steps
-                            for (int j = 0; j < nks_last; ++j) {
-                                if (need_sfa) tmem_cp_32x128b_x4_pair(ta + 4u * j, dfa + 32u * j);
-                                tmem_cp_128x256b_pair(tb + 8u * j, dfb + (uint64_t)(SFB_KSTEP_BYTES >> 4) * j);
-                                mma_nvfp4_pair(tmem + ACC_COL, da + 2u * j, db + 2u * j, idesc_fp4, ta + 4u * j,
-                                               tb + 8u * j, (kk > 0 || j > 0) ? 1u : 0u);
+                        if (kk < n_kb) {
+                            if (kk + 1 < n_kb || nks_last == 4) {
+                                if (need_sfa)
+                                    gp_issue_stage<true>(tmem + ACC_COL, da, db, dfa, dfb, ta, tb, idesc_fp4, acc0);
+                                else
+                                    gp_issue_stage<false>(tmem + ACC_COL, da, db, dfa, dfb, ta, tb, idesc_fp4, acc0);
+                            } else {
+                                // a last stage of fewer than four K-steps
+                                for (int j = 0; j < nks_last; ++j) {
+                                    if (need_sfa) tmem_cp_32x128b_x4_pair(ta + 4u * j, dfa + 32u * j);
+                                    tmem_cp_128x256b_pair(tb + 8u * j, dfb + (uint64_t)(SFB_KSTEP_BYTES >> 4) * j);
+                                    mma_nvfp4_pair(tmem + ACC_COL, da + 2u * j, db + 2u * j, idesc_fp4, ta + 4u * j,
+                                                   tb + 8u * j, (kk > 0 || j > 0) ? 1u : 0u);
+                                }
                             }
+                        } else {
+                            // rank-r stage: bf16 MMAs of the hi or lo part into the same accumulator
+                            const int c = (kk - n_kb) >> 1;
+                            const int nks = min(4, (a.rank - 64 * c + 15) / 16);
+                            for (int j = 0; j < nks; ++j)
+                                mma_bf16_pair(tmem + ACC_COL, da + 2u * j, db + 2u * j, idesc_lr, 1u);
                         }
-                        tc_commit_pair(&empty[s], 0x3);
                     }
-                    if (++s == kStages) {
-                        s = 0;
-                        ph ^= 1u;
-                    }
-                }
-                // rank-r stages: bf16 MMAs of the hi and lo parts into the same accumulator
-                for (int kk = n_kb; kk < per_tile && ok; ++kk, ++it) {
-                    if (gp_meet(kBarStage0 + (uint32_t)s, 0u)) {
+                    __syncwarp();
+                    // the other warp may issue stage it + 1 (its MMAs are not tracked by this warp's commit)
+                    named_bar_arrive(kBarTurn0 + (me ^ 1u), 64);
+                    if (!fail && lane == 0) tc_commit_pair(&empty[s], 0x3);
+                    if (fail) {
                         ok = false;
-                        s_failed = 1;
                         break;
                     }
-                    if (lane == 0) {
-                        tc_fence_after();
-                        const uint32_t sa = smem0 + (uint32_t)s * STAGE_BYTES;
-                        const uint64_t da = desc_sw128(sa), db = desc_sw128(sa + A_BYTES);
-                        const int c = (kk - n_kb) >> 1;
-                        const int nks = min(4, (a.rank - 64 * c + 15) / 16);
-                        for (int j = 0; j < nks; ++j)
-                            mma_bf16_pair(tmem + ACC_COL, da + 2u * j, db + 2u * j, idesc_lr, 1u);
-                        tc_commit_pair(&empty[s], 0x3);
-                    }
-                    if (++s == kStages) {
-                        s = 0;
-                        ph ^= 1u;
-                    }
                 }
+                // this warp's share of the tile is issued (possibly none of it)
                 if (ok && lane == 0) tc_commit_pair(acc_full, 0x3);
             }
-        }
-    } else if (warp == kWaitWarp) {
-        // ------------------------- barrier waiter for the MMA warp (CTA 0 only)
-        // The same walk over tiles and stages: wait on the accumulator and
-        // stage barriers, then meet the MMA warp (which goes on only then).
-        if (rank == 0) {
-            bool ok = true;
-            int local = 0, s = 0, it = 0;
-            uint32_t ph = 0;
-            for (int tile = t_begin; tile < t_end && ok; ++tile, ++local) {
-                bool f = !mbar_wait(acc_empty, ((uint32_t)local & 1u) ^ 1u, kSiteGpAccEmpty);
-                if (gp_meet(kBarAcc, f ? 1u : 0u)) {
-                    s_failed = 1;
-                    break;
-                }
-                for (int kk = 0; kk < per_tile; ++kk, ++it) {
-                    f = !mbar_wait(&full[s], ph, kSiteGpFull);
-                    if (gp_meet(kBarStage0 + (uint32_t)s, f ? 1u : 0u)) {
-                        ok = false;
-                        s_failed = 1;
-                        break;
-                    }
-                    if (++s == kStages) {
-                        s = 0;
-                        ph ^= 1u;
-                    }
-                }
-            }
+            // the warp that did not issue the run's last stage takes the last turn hand-over
+            if (ok && it > 0 && (uint32_t)((it - 1) & 1) != me) named_bar_sync(kBarTurn0 + me, 64);
         }
     } else if (warp >= (uint32_t)kEpiWarp0) {
         // ------------------------------------------------------------ epilogue
