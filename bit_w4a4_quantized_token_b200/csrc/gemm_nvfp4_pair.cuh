@@ -99,9 +99,18 @@ constexpr int kResidentKSteps = 48;
 constexpr uint32_t SFA_RES = 256;
 constexpr uint32_t SFB_RES = SFA_RES + 4 * kResidentKSteps;   // 448: two sets of 32 columns
 static_assert(SFB_RES + 64 <= TMEM_COLS, "resident scale-factor columns do not fit in TMEM");
+// The fused QKV epilogue streams the activation scales (so the resident
+// layout is never used there) and keeps the rotary tables of the CTA's 128
+// rows in the columns the two streamed sets leave free: lane = row, 64
+// columns of cos, then 64 of sin (fp32).
+constexpr uint32_t QKV_TAB_COL = SF_COL + 2 * SF_SET_COLS;   // 352
+static_assert(QKV_TAB_COL + 128 <= TMEM_COLS, "rotary tables do not fit in TMEM");
 constexpr uint32_t kFullArrivals = 3;          // CTA 0's three producer roles, for both CTAs' bytes
 constexpr int kLanesPerRole = 2;               // producer lanes per role, taking alternate stages
 constexpr size_t SMEM_BYTES = 1024 + (size_t)kStages * STAGE_BYTES + 256;
+// the mbarriers (full and empty per stage; acc_full, acc_empty; tab_free and
+// tab_ready per lane quarter) and the TMEM address
+static_assert((2 * kStages + 2 + 8) * 8 + 4 <= 256, "barriers do not fit their 256 bytes");
 static_assert(SMEM_BYTES <= 227 * 1024, "stage ring does not fit in shared memory");
 // kEpiPlain, kEpiQkv: y leaves through TMA stores of 32 x 32 boxes staged
 // per epilogue warp in kYBufs 2 KB buffers (64-byte swizzle), 1 KB aligned
@@ -182,7 +191,8 @@ enum : uint32_t {
     kSiteGpFull = 25,
     kSiteGpAcc = 26,
     kSiteGpDrain = 27,
-    kSiteGpAccEmpty = 28
+    kSiteGpAccEmpty = 28,
+    kSiteGpTab = 29
 };
 
 // One stage of four K-steps, issued by the MMA thread: the scale-block copies
@@ -368,26 +378,20 @@ __device__ __forceinline__ void gp_gelu_epilogue(const uint32_t (&acc)[NC], cons
         }
 }
 
-// bf16(S acc + b) of one thread's row for the 32 columns n .. n + 31
-// (chunk c2 of its 128 accumulators), as 16 packed words.
-__device__ __forceinline__ void gp_pack32(const uint32_t (&acc)[128], int c2, const GemmArgs& a, float S, int n,
+// bf16(S acc + b) of one thread's row for the 32 columns of chunk c2 of its
+// 128 accumulators, as 16 packed words.  The bias pair of the warp's columns
+// 2j, 2j + 1 (word j of its bias) sits in lane j % 32, entry j / 32 of qb
+// (zero past N), fetched before the accumulator was ready.
+__device__ __forceinline__ void gp_pack32(const uint32_t (&acc)[128], int c2, const uint32_t (&qb)[2], float S,
                                           uint32_t (&pk)[16]) {
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        uint32_t bw[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-        if (a.bias && n + 16 * h < a.N) {   // N % 16 == 0
-            const uint4 w0 = __ldg(reinterpret_cast<const uint4*>(a.bias + n + 16 * h));
-            const uint4 w1 = __ldg(reinterpret_cast<const uint4*>(a.bias + n + 16 * h) + 1);
-            bw[0] = w0.x, bw[1] = w0.y, bw[2] = w0.z, bw[3] = w0.w;
-            bw[4] = w1.x, bw[5] = w1.y, bw[6] = w1.z, bw[7] = w1.w;
-        }
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const float o0 = fmaf(__uint_as_float(acc[32 * c2 + 16 * h + 2 * i]), S, bf16lo_to_f32(bw[i]));
-            const float o1 = fmaf(__uint_as_float(acc[32 * c2 + 16 * h + 2 * i + 1]), S, bf16hi_to_f32(bw[i]));
-            const __nv_bfloat162 hv = __floats2bfloat162_rn(o0, o1);
-            pk[8 * h + i] = *reinterpret_cast<const uint32_t*>(&hv);
-        }
+    for (int i = 0; i < 16; ++i) {
+        const int j = 16 * c2 + i;
+        const uint32_t bw = __shfl_sync(0xffffffffu, qb[j / 32], j % 32);
+        const float o0 = fmaf(__uint_as_float(acc[2 * j]), S, bf16lo_to_f32(bw));
+        const float o1 = fmaf(__uint_as_float(acc[2 * j + 1]), S, bf16hi_to_f32(bw));
+        const __nv_bfloat162 hv = __floats2bfloat162_rn(o0, o1);
+        pk[i] = *reinterpret_cast<const uint32_t*>(&hv);
     }
 }
 
@@ -427,7 +431,9 @@ __global__ void __launch_bounds__(gp_threads<kEpi>(), 1)
     uint64_t* empty = full + kStages;
     uint64_t* acc_full = empty + kStages;
     uint64_t* acc_empty = acc_full + 1;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
+    uint64_t* tab_free = acc_empty + 1;    // [4] fused QKV: both warps of a lane quarter are done with its table
+    uint64_t* tab_ready = tab_free + 4;    // [4] fused QKV: both halves of a lane quarter's new table are in TMEM
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tab_ready + 4);
     __shared__ int s_failed;
     __shared__ int s_issued[gp::kStages];   // phases this CTA's A producers started in each stage
 
@@ -442,7 +448,7 @@ __global__ void __launch_bounds__(gp_threads<kEpi>(), 1)
     // the same 256 activation rows for several tiles in a row.
     const int t_begin = (int)(((int64_t)total_tiles * cluster) / n_clusters);
     const int t_end = (int)(((int64_t)total_tiles * (cluster + 1)) / n_clusters);
-    const bool sfa_res = a.kg4 <= kResidentKSteps;
+    const bool sfa_res = kEpi != kEpiQkv && a.kg4 <= kResidentKSteps;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -451,6 +457,10 @@ __global__ void __launch_bounds__(gp_threads<kEpi>(), 1)
         }
         mbar_init(acc_full, 2);   // both MMA warps commit at the end of every tile
         mbar_init(acc_empty, 2u * (uint32_t)gp_epi_warps<kEpi>());   // both CTAs' epilogue warps
+        for (int i = 0; i < 4; ++i) {
+            mbar_init(&tab_free[i], 2);
+            mbar_init(&tab_ready[i], 2);
+        }
         for (int s = 0; s < kStages; ++s) s_issued[s] = 0;
         s_failed = 0;
         fence_barrier_init();
@@ -653,10 +663,73 @@ __global__ void __launch_bounds__(gp_threads<kEpi>(), 1)
             named_bar_sync(1, 32 * kEpiWarpsGelu);
         }
         int local = 0;
+        int epoch = -1, prev_m = -1;   // fused QKV: rotary tables loaded so far, and for which row block
         for (int tile = t_begin; tile < t_end; ++tile, ++local) {
             const int m_tile = tile / a.n_tiles, n_tile = tile - m_tile * a.n_tiles;
             const int64_t grow = (int64_t)m_tile * BM + 128 * (int64_t)rank + row;
             const int nbase = n_tile * BN + 128 * half;
+            // Before the accumulator is ready: this warp's 128 columns of bias,
+            // pairs l and 32 + l in lane l (uniform loads inside the epilogue
+            // each waited a full L2 round trip under the main loop's traffic);
+            // fused QKV: on a new row block the two warps of this lane quarter
+            // put the rows' rotary tables into TMEM (this warp one of cos /
+            // sin), and a Q or K head's RMSNorm weights go with the bias
+            uint32_t qbias[2] = {0u, 0u}, qgam[2] = {0u, 0u};
+            const bool qk_head = kEpi == kEpiQkv && nbase < a.qk_cols;
+            if (kEpi != kEpiGelu && a.bias) {
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    const int col = nbase + 2 * (32 * i + (int)lane);
+                    if (col < a.N) qbias[i] = __ldg(reinterpret_cast<const uint32_t*>(a.bias + col));
+                }
+            }
+            if (kEpi == kEpiQkv) {
+                if (m_tile != prev_m) {
+                    ++epoch;
+                    prev_m = m_tile;
+                    if (epoch > 0) {   // the old table: this warp is done with it; wait for the other
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&tab_free[q]);
+                        if (!mbar_wait(&tab_free[q], (uint32_t)(epoch - 1) & 1u, kSiteGpTab)) {
+                            s_failed = 1;
+                            break;
+                        }
+                        tc_fence_after();
+                    }
+                    // rows past M take the last row's table (their results are not stored)
+                    const int64_t trow = grow < a.M ? grow : (int64_t)a.M - 1;
+                    const float4* src = reinterpret_cast<const float4*>((half == 0 ? a.rope_cos : a.rope_sin) + trow * 64);
+#pragma unroll
+                    for (int p2 = 0; p2 < 2; ++p2) {
+                        uint32_t t32[32];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const float4 v = __ldg(src + 8 * p2 + i);
+                            t32[4 * i] = __float_as_uint(v.x);
+                            t32[4 * i + 1] = __float_as_uint(v.y);
+                            t32[4 * i + 2] = __float_as_uint(v.z);
+                            t32[4 * i + 3] = __float_as_uint(v.w);
+                        }
+                        tmem_st_32x32b_x32(tmem + ((32u * q) << 16) + QKV_TAB_COL + 64u * (uint32_t)half + 32u * p2,
+                                           t32);
+                    }
+                    tmem_st_wait();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&tab_ready[q]);
+                    if (!mbar_wait(&tab_ready[q], (uint32_t)epoch & 1u, kSiteGpTab)) {
+                        s_failed = 1;
+                        break;
+                    }
+                    tc_fence_after();
+                }
+                if (qk_head) {
+                    const __nv_bfloat16* gw = nbase < a.q_cols ? a.norm_q : a.norm_k;
+#pragma unroll
+                    for (int i = 0; i < 2; ++i) qgam[i] = __ldg(reinterpret_cast<const uint32_t*>(gw) + 32 * i + lane);
+                }
+            }
             if (!mbar_wait(acc_full, (uint32_t)local & 1u, kSiteGpAcc)) {
                 s_failed = 1;
                 break;
@@ -701,57 +774,39 @@ __global__ void __launch_bounds__(gp_threads<kEpi>(), 1)
             const uint32_t stage0 =
                 smem_u32(smem + Y_STAGE_OFF) + (uint32_t)(warp - kEpiWarp0) * (uint32_t)(kYBufs * kYStageBytes);
             const int row0 = (int)(grow - lane);
-            if (kEpi == kEpiQkv && nbase < a.qk_cols) {
+            if (qk_head) {
                 // this warp's 128 columns are one Q or K head of a to_qkv
                 // projection (qkv_norm_rope.cuh): RMSNorm over them, then the
                 // rotary pairs, on the fp32 values before the single bf16 rounding
                 float ss = 0.0f;
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const int n = nbase + 16 * c;
-                    uint4 w0 = make_uint4(0u, 0u, 0u, 0u), w1 = w0;
-                    if (a.bias) {
-                        w0 = __ldg(reinterpret_cast<const uint4*>(a.bias + n));
-                        w1 = __ldg(reinterpret_cast<const uint4*>(a.bias + n) + 1);
-                    }
-                    const uint32_t ws[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-#pragma unroll
-                    for (int p = 0; p < 8; ++p) {
-                        const float o0 = fmaf(__uint_as_float(acc[16 * c + 2 * p]), S, bf16lo_to_f32(ws[p]));
-                        const float o1 = fmaf(__uint_as_float(acc[16 * c + 2 * p + 1]), S, bf16hi_to_f32(ws[p]));
-                        acc[16 * c + 2 * p] = __float_as_uint(o0);
-                        acc[16 * c + 2 * p + 1] = __float_as_uint(o1);
-                        ss = fmaf(o0, o0, ss);
-                        ss = fmaf(o1, o1, ss);
-                    }
+                for (int j = 0; j < 64; ++j) {   // pair j: columns nbase + 2j, + 1; its bias in lane j % 32
+                    const uint32_t bw = __shfl_sync(0xffffffffu, qbias[j / 32], j % 32);
+                    const float o0 = fmaf(__uint_as_float(acc[2 * j]), S, bf16lo_to_f32(bw));
+                    const float o1 = fmaf(__uint_as_float(acc[2 * j + 1]), S, bf16hi_to_f32(bw));
+                    acc[2 * j] = __float_as_uint(o0);
+                    acc[2 * j + 1] = __float_as_uint(o1);
+                    ss = fmaf(o0, o0, ss);
+                    ss = fmaf(o1, o1, ss);
                 }
                 const float r = rsqrtf(ss * (1.0f / 128.0f) + a.eps);
-                const __nv_bfloat16* w = nbase < a.q_cols ? a.norm_q : a.norm_k;
-                // rows past M read the last row's rotary table (their results are not stored)
-                const int64_t trow = grow < a.M ? grow : (int64_t)a.M - 1;
-                const float4* cs4 = reinterpret_cast<const float4*>(a.rope_cos + trow * 64);
-                const float4* sn4 = reinterpret_cast<const float4*>(a.rope_sin + trow * 64);
 #pragma unroll
                 for (int c2 = 0; c2 < 4; ++c2) {
+                    // the rotary table of pairs 16 c2 .. 16 c2 + 15 of this row, from TMEM
+                    uint32_t cc[16], sc[16];
+                    tmem_ld_32x32b_x16(tmem + ((32u * q) << 16) + QKV_TAB_COL + 16u * c2, cc);
+                    tmem_ld_32x32b_x16(tmem + ((32u * q) << 16) + QKV_TAB_COL + 64u + 16u * c2, sc);
+                    tmem_ld_wait();
                     uint32_t pk[16];
 #pragma unroll
-                    for (int h = 0; h < 2; ++h) {   // 16 columns = 8 rotary pairs
-                        const int c = 2 * c2 + h;
-                        const uint4 g0 = __ldg(reinterpret_cast<const uint4*>(w + 16 * c));
-                        const uint4 g1 = __ldg(reinterpret_cast<const uint4*>(w + 16 * c) + 1);
-                        const uint32_t gs[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-                        const float4 c0 = __ldg(cs4 + 2 * c), c1 = __ldg(cs4 + 2 * c + 1);
-                        const float4 s0 = __ldg(sn4 + 2 * c), s1 = __ldg(sn4 + 2 * c + 1);
-                        const float cc[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-                        const float sc[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-#pragma unroll
-                        for (int p = 0; p < 8; ++p) {
-                            const float v0 = __uint_as_float(acc[16 * c + 2 * p]) * r * bf16lo_to_f32(gs[p]);
-                            const float v1 = __uint_as_float(acc[16 * c + 2 * p + 1]) * r * bf16hi_to_f32(gs[p]);
-                            const __nv_bfloat162 hv =
-                                __floats2bfloat162_rn(v0 * cc[p] - v1 * sc[p], v1 * cc[p] + v0 * sc[p]);
-                            pk[8 * h + p] = *reinterpret_cast<const uint32_t*>(&hv);
-                        }
+                    for (int p = 0; p < 16; ++p) {
+                        const int j = 16 * c2 + p;
+                        const uint32_t gw = __shfl_sync(0xffffffffu, qgam[j / 32], j % 32);
+                        const float v0 = __uint_as_float(acc[2 * j]) * r * bf16lo_to_f32(gw);
+                        const float v1 = __uint_as_float(acc[2 * j + 1]) * r * bf16hi_to_f32(gw);
+                        const float cj = __uint_as_float(cc[p]), sj = __uint_as_float(sc[p]);
+                        const __nv_bfloat162 hv = __floats2bfloat162_rn(v0 * cj - v1 * sj, v1 * cj + v0 * sj);
+                        pk[p] = *reinterpret_cast<const uint32_t*>(&hv);
                     }
                     gp_stage_store(pk, stage0 + (uint32_t)(c2 % kYBufs) * kYStageBytes, lane, &tm_y, nbase + 32 * c2,
                                    row0, a.M);
@@ -763,7 +818,7 @@ __global__ void __launch_bounds__(gp_threads<kEpi>(), 1)
                 const int n = nbase + 32 * c2;
                 if (n >= a.N) break;   // warp-uniform
                 uint32_t pk[16];
-                gp_pack32(acc, c2, a, S, n, pk);
+                gp_pack32(acc, c2, qbias, S, pk);
                 gp_stage_store(pk, stage0 + (uint32_t)(c2 % kYBufs) * kYStageBytes, lane, &tm_y, n, row0, a.M);
             }
         }
