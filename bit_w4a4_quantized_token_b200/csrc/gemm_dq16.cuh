@@ -21,10 +21,12 @@
 //
 // One CTA per 128 x 256 output tile.  Warp 0 loads, per 64 columns of K, the
 // activation tile (bf16 x, or int4 codes and their group scales), the packed
-// weight tile (256 rows x 32 bytes) and its 256 group scales; warps 4..11
+// weight tile (256 rows x 32 bytes) and its 256 group scales; warps 4..19
 // expand both into fp16 tiles in the MMA's swizzled layout (x converted in
 // place); warp 1 issues four M = 128, N = 256, K = 16 MMAs per stage into
-// TMEM; warps 12..19 add the bias and store bf16.
+// TMEM; after the last stage warps 12..19 add the bias and store bf16.  The
+// expansion sets the pace, so every warp that would otherwise wait for the
+// accumulator takes part in it.
 #pragma once
 #include "sm100_ptx.cuh"
 
@@ -45,7 +47,7 @@ constexpr int OFF_AP = OFF_WP + WP_BYTES;
 constexpr int OFF_WS = OFF_AP + AP_BYTES;
 constexpr int OFF_AS = OFF_WS + WS_BYTES;
 constexpr int STAGE_BYTES = ((OFF_AS + AS_BYTES + 1023) / 1024) * 1024;
-constexpr int kConvWarp0 = 4, kConvWarps = 8;
+constexpr int kConvWarp0 = 4, kConvWarps = 16;   // the epilogue warps convert too
 constexpr int kEpiWarp0 = 12, kEpiWarps = 8;
 constexpr int kThreads = 32 * (kEpiWarp0 + kEpiWarps);
 constexpr size_t SMEM_BYTES = 1024 + (size_t)kStages * STAGE_BYTES + 256;
@@ -211,9 +213,9 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
             }
             if (ok) tc_commit(acc_full);
         }
-    } else if (warp >= (uint32_t)kConvWarp0 && warp < (uint32_t)kConvWarp0 + kConvWarps) {
+    } else if (warp >= (uint32_t)kConvWarp0) {
         // ----------------------------------- activations and weights -> fp16
-        const int t = (int)threadIdx.x - 32 * kConvWarp0;   // 0..255: weight row t
+        const int t = (int)threadIdx.x - 32 * kConvWarp0;   // 0..511: half of weight row t / 2
         for (int it = 0; it < n_st; ++it) {
             const int s = it % kStages;
             if (!mbar_wait(&full[s], (uint32_t)(it / kStages) & 1u, kSiteDqFull)) {
@@ -223,24 +225,24 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
             uint8_t* st = smem + (size_t)s * STAGE_BYTES;
             if (it < n_kc) {
                 if (kInt4A) {
-                    // activation row t / 2, values 32 (t % 2) .. + 31: codes -> fp16 (q s_x)
-                    const int r = t >> 1, h = t & 1;
+                    // activation row t / 4, values 16 (t % 4) .. + 15: codes -> fp16 (q s_x)
+                    const int r = t >> 2, h = t & 3;
                     const __half2 s2 = bf16_scale_to_h2(*reinterpret_cast<const uint16_t*>(st + OFF_AS + 2 * r));
-                    const uint4 c4 = *reinterpret_cast<const uint4*>(st + OFF_AP + 32 * r + 16 * h);
-                    const uint32_t cw[4] = {c4.x, c4.y, c4.z, c4.w};
+                    const uint2 c2 = *reinterpret_cast<const uint2*>(st + OFF_AP + 32 * r + 8 * h);
+                    const uint32_t cw[2] = {c2.x, c2.y};
                     uint8_t* arow = st + r * 128;
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {   // 16-byte chunk 4h + c: values 8 (4h + c) .. + 7
+                    for (int c = 0; c < 2; ++c) {   // 16-byte chunk 2h + c: values 8 (2h + c) .. + 7
                         uint32_t o[4];
                         int4x8_to_f16(cw[c], s2, o);
-                        *reinterpret_cast<uint4*>(arow + (((4 * h + c) ^ (r & 7)) << 4)) =
+                        *reinterpret_cast<uint4*>(arow + (((2 * h + c) ^ (r & 7)) << 4)) =
                             make_uint4(o[0], o[1], o[2], o[3]);
                     }
                 } else {
-                    // x: 16 KB of bf16 in place, 64 bytes per thread (position-preserving)
+                    // x: 16 KB of bf16 in place, 32 bytes per thread (position-preserving)
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        uint4* p = reinterpret_cast<uint4*>(st + 16 * (t + 256 * i));
+                    for (int i = 0; i < 2; ++i) {
+                        uint4* p = reinterpret_cast<uint4*>(st + 16 * (t + 512 * i));
                         const uint4 v = *p;
                         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
                         uint32_t o[4];
@@ -252,24 +254,27 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
                         *p = make_uint4(o[0], o[1], o[2], o[3]);
                     }
                 }
-                // weight row t: 64 codes -> 64 fp16 (q s_w) in the swizzled 128-byte row
-                const uint8_t* wp = st + OFF_WP + 32 * t;
-                const __half2 s2 = bf16_scale_to_h2(*reinterpret_cast<const uint16_t*>(st + OFF_WS + 2 * t));
-                const uint4 c0 = *reinterpret_cast<const uint4*>(wp), c1 = *reinterpret_cast<const uint4*>(wp + 16);
-                const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-                uint8_t* wrow = st + OFF_WF + t * 128;
+                // weight row t / 2, codes 32 (t % 2) .. + 31 -> fp16 (q s_w) in the swizzled 128-byte row
+                const int wr = t >> 1, wh = t & 1;
+                const uint8_t* wp = st + OFF_WP + 32 * wr + 16 * wh;
+                const __half2 s2 = bf16_scale_to_h2(*reinterpret_cast<const uint16_t*>(st + OFF_WS + 2 * wr));
+                const uint4 c0 = *reinterpret_cast<const uint4*>(wp);
+                const uint32_t cw[4] = {c0.x, c0.y, c0.z, c0.w};
+                uint8_t* wrow = st + OFF_WF + wr * 128;
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {   // 16-byte chunk c: K values 8c .. 8c + 7
+                for (int c = 0; c < 4; ++c) {   // 16-byte chunk 4 wh + c: K values 8 (4 wh + c) .. + 7
                     uint32_t o[4];
                     int4x8_to_f16(cw[c], s2, o);
-                    *reinterpret_cast<uint4*>(wrow + ((c ^ (t & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+                    *reinterpret_cast<uint4*>(wrow + (((4 * wh + c) ^ (wr & 7)) << 4)) =
+                        make_uint4(o[0], o[1], o[2], o[3]);
                 }
                 fence_proxy_async_smem();   // both tiles are read by the tensor core
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&conv[s]);
         }
-    } else if (warp >= (uint32_t)kEpiWarp0) {
+    }
+    if (warp >= (uint32_t)kEpiWarp0) {
         // ------------------------------------------------------------ epilogue
         const uint32_t q = warp & 3u;
         const int half = (int)(warp - kEpiWarp0) >> 2;
