@@ -110,6 +110,27 @@ def test_argument_validation_before_device(L):
                         w_tensor_scale=None) in (0, L.SVDQ_ERR_UNSUPPORTED_DEVICE)
 
 
+def test_replicate_weight_scales_argument_checks(L):
+    """The GEMM-ready weight-scale copy: argument errors come before any device check."""
+    fake = 1 << 20
+
+    def status(**kw):
+        args = dict(w_scales=fake, N=256, K=256, stream=0)
+        args.update(kw)
+        try:
+            L.svdq_replicate_weight_scales(**args)
+            return 0
+        except L.SvdqError as e:
+            return e.status
+
+    assert status(w_scales=None) == L.SVDQ_ERR_INVALID_ARG
+    assert status(w_scales=fake + 8) == L.SVDQ_ERR_INVALID_ARG      # misaligned
+    assert status(N=8) == L.SVDQ_ERR_UNSUPPORTED_SHAPE              # N % 16 != 0
+    assert status(K=96) == L.SVDQ_ERR_UNSUPPORTED_SHAPE             # K % 64 != 0
+    assert status(N=0) == L.SVDQ_ERR_UNSUPPORTED_SHAPE
+    assert status() in (0, L.SVDQ_ERR_UNSUPPORTED_DEVICE)
+
+
 def test_capability_check_rejects_other_devices(L):
     """With any capability other than 10.0 (or no GPU) nothing is launched."""
     L.svdq_debug_override_capability(12, 0)        # an sm_120 consumer Blackwell part
