@@ -364,17 +364,17 @@ class Shape:
         self._lib = _lib
         torch.cuda.synchronize(dev)
 
-    def quant(self):
+    def quant(self, x=None):
         c, p, q = self.case, self.packed, self.q
-        self._lib.svdq_quantize_act(c.precision, c.group_size, self.x, c.M, c.K, p.inv_lambda, q.x_tensor_scale,
-                                    self.compute_scale, p.w_tensor_scale, p.L_down_t, c.rank, q.x_codes, q.x_scales,
-                                    q.lowrank_act, q.workspace, stream=self.stream)
+        self._lib.svdq_quantize_act(c.precision, c.group_size, self.x if x is None else x, c.M, c.K, p.inv_lambda,
+                                    q.x_tensor_scale, self.compute_scale, p.w_tensor_scale, p.L_down_t, c.rank,
+                                    q.x_codes, q.x_scales, q.lowrank_act, q.workspace, stream=self.stream)
 
-    def gemm(self):
+    def gemm(self, y=None):
         c, p, q = self.case, self.packed, self.q
         self._lib.svdq_gemm_w4a4(c.precision, c.group_size, q.x_codes, q.x_scales, q.x_tensor_scale, c.M, p.w_codes,
-                                 p.w_scales, p.w_tensor_scale, c.N, c.K, q.lowrank_act, p.L_up_t, c.rank, p.bias, self.y,
-                                 stream=self.stream)
+                                 p.w_scales, p.w_tensor_scale, c.N, c.K, q.lowrank_act, p.L_up_t, c.rank, p.bias,
+                                 self.y if y is None else y, stream=self.stream)
 
     def graphs(self):
         """CUDA graphs of the step and of each kernel (captured after warm-up)."""
@@ -724,23 +724,53 @@ def run_cuda(args) -> dict | None:
         raise RuntimeError(f"device status {st} at site {site} in the timed region")
     t = {k: max_over_ranks(v, world, dev) for k, v in t.items()}
 
-    # end to end through the public API: pinned host x -> device, forward, y -> pinned host
+    # end to end through the public API: every step copies its x from pinned
+    # host memory to the device, runs the quantizer and the GEMM, and copies
+    # y back to pinned host memory.  Steps are pipelined over three streams
+    # (input copies, compute, output copies) with two device buffers of x and
+    # of y, so that step i's copies overlap the neighbouring steps' work, as a
+    # serving loop would run them; the copy engines of both directions work
+    # at once.
     x_host = sh.x_host.pin_memory()
-    y_host = torch.empty(case.M, case.N, dtype=torch.bfloat16).pin_memory()
-    e2e_steps = max(1, min(args.steps, 20))
-    with torch.cuda.stream(stream):
-        for i in range(2 + e2e_steps):
-            if i == 2:
-                torch.cuda.synchronize(dev)
-                if world > 1:
-                    dist.barrier()
-                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                e0.record(stream)
-            sh.x.copy_(x_host, non_blocking=True)
-            sh.quant()
-            sh.gemm()
-            y_host.copy_(sh.y, non_blocking=True)
-        e1.record(stream)
+    y_host = [torch.empty(case.M, case.N, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    xd = [sh.x, torch.empty_like(sh.x)]
+    yd = [sh.y, torch.empty_like(sh.y)]
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    x_ready, x_free, y_ready, y_free = ([torch.cuda.Event() for _ in range(2)] for _ in range(4))
+
+    def e2e_step(i):
+        b = i % 2
+        if i >= 2:
+            s_in.wait_event(x_free[b])
+        with torch.cuda.stream(s_in):
+            xd[b].copy_(x_host, non_blocking=True)
+            x_ready[b].record(s_in)
+        stream.wait_event(x_ready[b])
+        with torch.cuda.stream(stream):
+            sh.quant(x=xd[b])
+            x_free[b].record(stream)
+            if i >= 2:
+                stream.wait_event(y_free[b])
+            sh.gemm(y=yd[b])
+            y_ready[b].record(stream)
+        s_out.wait_event(y_ready[b])
+        with torch.cuda.stream(s_out):
+            y_host[b].copy_(yd[b], non_blocking=True)
+            y_free[b].record(s_out)
+
+    e2e_steps = max(2, min(args.steps, 20))
+    for i in range(2):
+        e2e_step(i)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s_in)
+    for i in range(2, 2 + e2e_steps):
+        e2e_step(i)
+    s_out.wait_stream(s_in)
+    s_out.wait_stream(stream)
+    e1.record(s_out)
     torch.cuda.synchronize(dev)
     t_e2e = max_over_ranks(e0.elapsed_time(e1) / e2e_steps / 1e3, world, dev)
     del gs
