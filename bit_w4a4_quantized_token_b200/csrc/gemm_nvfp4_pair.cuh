@@ -83,15 +83,15 @@ constexpr uint32_t kMmaWarp2 = 3;
 constexpr uint32_t kBarTurn0 = 2;              // named barriers 2, 3: the turn of warp 2, 3 (0: __syncthreads, 1: GELU epilogue)
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COL = 0;
-// Scale factors in TMEM.  Stages alternate between two "scale sets"; one of
-// two layouts:
+// Scale factors in TMEM.  Stages alternate between two "scale sets" (one per
+// MMA-issuing warp); one of two layouts:
 //  * streamed (any K): set b at SF_COL + 48 b: 4 k-steps x 4 columns of
 //    activation scales, then 4 k-steps x 8 columns of weight scales;
 //  * resident activation scales (K <= 64 * kResidentKSteps): the activation
 //    scales of the whole K for the current 256-row tile stay at SFA_RES +
 //    4 k, copied once per run of tiles that share those rows, and set b holds
 //    only weight scales, at SFB_RES + 32 b.  This takes the activation-scale
-//    copies (a third of all copies) off the tensor pipe.
+//    copies off the tensor pipe.
 constexpr uint32_t SF_COL = 256;
 constexpr uint32_t SF_SET_COLS = 48;
 static_assert(SF_COL + 2 * SF_SET_COLS <= TMEM_COLS, "scale-factor columns do not fit in TMEM");
@@ -195,12 +195,12 @@ enum : uint32_t {
     kSiteGpTab = 29
 };
 
-// One stage of four K-steps, issued by the MMA thread: the scale-block copies
-// of K-step j + 1 go in right before the MMA of step j.  The tensor pipe keeps
-// only a few instructions queued, so this sequence is written to have nothing
-// between its tcgen05 instructions but address arithmetic on registers: every
-// cycle the issuing thread spends elsewhere (branches, loads, waits) is a cycle
-// the pipe may sit idle.  WITH_SFA: also copy the activation scales.
+// One stage of four K-steps, issued by an MMA thread: the scale copies of
+// K-step j + 1 go in right before the MMA of step j (one 128x256b copy of
+// the replicated weight scales; WITH_SFA: also a 32x128b.warpx4 copy of the
+// activation scales).  The tensor pipe keeps only a few instructions queued,
+// so this sequence has nothing between its tcgen05 instructions but address
+// arithmetic on registers.
 template <bool WITH_SFA>
 __device__ __forceinline__ void gp_issue_stage(uint32_t acc, uint64_t da, uint64_t db, uint64_t dfa, uint64_t dfb,
                                                uint32_t ta, uint32_t tb, uint32_t idesc, uint32_t acc0) {
