@@ -82,23 +82,44 @@ __device__ __forceinline__ uint32_t quant_group64_int4(const float (&v)[64], uin
 __global__ void __launch_bounds__(256) amax_kernel(const __nv_bfloat16* __restrict__ x,
                                                    const float* __restrict__ inv_lambda, int64_t rows, int64_t K,
                                                    unsigned int* out) {
-    const int64_t nvec = rows * K / 8;
+    const int64_t nvec = rows * K / 8;   // 16-byte vectors of 8 values, grid-stride
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    const int64_t kv = K / 8;            // vectors per row (K % 64 == 0)
+    const int64_t dk = stride % kv;      // how far the column advances per stride
+    int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    int64_t col = v % kv;                // the vector's column position, kept without a division per step
     float m = 0.0f;
-    for (int64_t v = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; v < nvec;
-         v += (int64_t)gridDim.x * blockDim.x) {
-        const uint4 w = __ldg(reinterpret_cast<const uint4*>(x) + v);
-        const int64_t k0 = (v * 8) % K;
+    // |v_i| of 8 values starting at column 8 c, with v = x / lambda when given
+    auto fold = [&](const uint4 w, int64_t c) {
         const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+        float4 l0 = make_float4(1.0f, 1.0f, 1.0f, 1.0f), l1 = l0;
+        if (inv_lambda) {
+            l0 = __ldg(reinterpret_cast<const float4*>(inv_lambda) + 2 * c);
+            l1 = __ldg(reinterpret_cast<const float4*>(inv_lambda) + 2 * c + 1);
+        }
+        const float il[8] = {l0.x, l0.y, l0.z, l0.w, l1.x, l1.y, l1.z, l1.w};
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
             float a0 = bf16lo_to_f32(ws[q]), a1 = bf16hi_to_f32(ws[q]);
             if (inv_lambda) {
-                a0 = __fmul_rn(a0, __ldg(inv_lambda + k0 + 2 * q));
-                a1 = __fmul_rn(a1, __ldg(inv_lambda + k0 + 2 * q + 1));
+                a0 = __fmul_rn(a0, il[2 * q]);
+                a1 = __fmul_rn(a1, il[2 * q + 1]);
             }
             m = fmaxf(m, fmaxf(fabsf(a0), fabsf(a1)));
         }
+    };
+    // two vectors in flight per thread
+    for (; v + stride < nvec; v += 2 * stride) {
+        int64_t col2 = col + dk;
+        if (col2 >= kv) col2 -= kv;
+        const uint4 w0 = __ldg(reinterpret_cast<const uint4*>(x) + v);
+        const uint4 w1 = __ldg(reinterpret_cast<const uint4*>(x) + v + stride);
+        fold(w0, col);
+        fold(w1, col2);
+        col = col2 + dk;
+        if (col >= kv) col -= kv;
     }
+    if (v < nvec) fold(__ldg(reinterpret_cast<const uint4*>(x) + v), col);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
     __shared__ float red[8];
