@@ -344,17 +344,19 @@ __global__ void __launch_bounds__(qa::kThreads, 1)
         float* part = reinterpret_cast<float*>(smem);          // [128][rank + 4] fp32
         const float inv_ss =
             (PREC == kPrecNvfp4) ? __frcp_rn(__fmul_rn(*a.x_scale, *a.w_scale)) : 1.0f;
-        if (warp >= (uint32_t)qa::kWorker0 && warp < (uint32_t)qa::kWorker0 + 4) {
-            // four warps cover the four TMEM lane quadrants: one thread per row,
-            // 16 columns at a time
+        if (warp >= (uint32_t)qa::kWorker0) {
+            // the sixteen quantizer warps drain the accumulator: warp w reads
+            // TMEM lane quadrant w % 4 (one thread per row) and every fourth
+            // 16-column block from block (w - 4) / 4 on
             const uint32_t q = warp & 3u;
             const int row = (int)(32u * q + lane);
+            const int first = 16 * (int)((warp - (uint32_t)qa::kWorker0) >> 2);
             const bool ok = mbar_wait(accb, 0, kSiteQaAcc);
             if (!ok) s_failed = 1;
             tc_fence_after();
             float* mine = workspace_mode ? a.partials + (((int64_t)rb * a.splits + split) * qa::kRows + row) * a.rank
                                          : part + row * pstride;
-            for (int c0 = 0; c0 < a.rank; c0 += 16) {
+            for (int c0 = first; c0 < a.rank; c0 += 64) {
                 uint32_t r16[16], s16[16];
                 tmem_ld_32x32b_x16(tmem + ((32u * q) << 16) + (uint32_t)c0, r16);              // x . hi
                 tmem_ld_32x32b_x16(tmem + ((32u * q) << 16) + (uint32_t)(a.rank + c0), s16);   // x . lo
@@ -369,41 +371,57 @@ __global__ void __launch_bounds__(qa::kThreads, 1)
             }
             if (workspace_mode) {
                 __threadfence();
-                named_bar_sync(2, 128);
+                named_bar_sync(2, qa::kWorkers);
                 if (threadIdx.x == 32 * qa::kWorker0) {
                     const unsigned int prev = atomicAdd(a.counters + rb, 1u);
                     s_last = (prev == (unsigned int)(a.splits - 1)) ? 1 : 0;
                 }
-                named_bar_sync(2, 128);
+                named_bar_sync(2, qa::kWorkers);
                 if (s_last) {
-                    // the last CTA of this row block adds the partials in split order
+                    // the last CTA of this row block adds the partials in split
+                    // order, one row and 4 columns per item, consecutive threads
+                    // on consecutive columns; the loads of up to four splits are
+                    // issued before the first add
                     __threadfence();
-                    const int64_t grow = (int64_t)m0 + row;
+                    const int t = (int)threadIdx.x - 32 * qa::kWorker0;
+                    const int q4 = a.rank / 4;
                     const int64_t plane = (int64_t)a.M * a.rank;
-                    for (int c0 = 0; c0 < a.rank; c0 += 4) {
+                    const float* base = a.partials + (int64_t)rb * a.splits * qa::kRows * a.rank;
+                    const int64_t pstep = (int64_t)qa::kRows * a.rank;
+                    for (int i = t; i < qa::kRows * q4; i += qa::kWorkers) {
+                        const int rl = i / q4, c0 = 4 * (i - rl * q4);
+                        const float* src = base + (int64_t)rl * a.rank + c0;
                         float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-                        for (int p = 0; p < a.splits; ++p) {
-                            const float4 f = __ldcg(reinterpret_cast<const float4*>(
-                                a.partials + (((int64_t)rb * a.splits + p) * qa::kRows + row) * a.rank + c0));
-                            acc.x += f.x;
-                            acc.y += f.y;
-                            acc.z += f.z;
-                            acc.w += f.w;
+                        for (int p0 = 0; p0 < a.splits; p0 += 4) {
+                            float4 f[4];
+#pragma unroll
+                            for (int j = 0; j < 4; ++j)
+                                if (p0 + j < a.splits) f[j] = __ldcg(reinterpret_cast<const float4*>(src + (p0 + j) * pstep));
+#pragma unroll
+                            for (int j = 0; j < 4; ++j)
+                                if (p0 + j < a.splits) {
+                                    acc.x += f[j].x;
+                                    acc.y += f[j].y;
+                                    acc.z += f[j].z;
+                                    acc.w += f[j].w;
+                                }
                         }
+                        const int64_t grow = (int64_t)m0 + rl;
                         if (grow < a.M) {
                             __nv_bfloat16* hi = a.lowrank + grow * a.rank + c0;
                             store_lowrank_pair(hi, hi + plane, acc.x, acc.y, inv_ss);
                             store_lowrank_pair(hi + 2, hi + 2 + plane, acc.z, acc.w, inv_ss);
                         }
                     }
-                    if (threadIdx.x == 32 * qa::kWorker0) a.counters[rb] = 0u;   // ready for the next call
+                    if (t == 0) a.counters[rb] = 0u;   // ready for the next call
                 }
             }
         }
         if (!workspace_mode) {
             // Add the partials of the cluster (or take this CTA's own) in split
             // order; this CTA stores rows [r_lo, r_hi) of the row block with
-            // consecutive threads on consecutive column pairs (coalesced).
+            // consecutive threads on consecutive column pairs (coalesced).  The
+            // loads from the peers' shared memory are issued before the adds.
             if (cluster_mode)
                 cluster_sync_all();
             else
@@ -421,13 +439,20 @@ __global__ void __launch_bounds__(qa::kThreads, 1)
                     const uint32_t off = (uint32_t)(rl * pstride + 2 * j) * 4u;
                     float2 acc = make_float2(0.0f, 0.0f);
                     if (cluster_mode) {
-                        for (int p = 0; p < C; ++p) {
-                            uint32_t remote;
-                            asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(part_u32 + off), "r"(p));
-                            const float2 f = ld_cluster_f32x2(remote);
-                            acc.x += f.x;
-                            acc.y += f.y;
-                        }
+                        float2 f[qa::kMaxCluster];
+#pragma unroll
+                        for (int p = 0; p < qa::kMaxCluster; ++p)
+                            if (p < C) {
+                                uint32_t remote;
+                                asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(part_u32 + off), "r"(p));
+                                f[p] = ld_cluster_f32x2(remote);
+                            }
+#pragma unroll
+                        for (int p = 0; p < qa::kMaxCluster; ++p)
+                            if (p < C) {
+                                acc.x += f[p].x;
+                                acc.y += f[p].y;
+                            }
                     } else {
                         acc = *reinterpret_cast<const float2*>(part + rl * pstride + 2 * j);
                     }

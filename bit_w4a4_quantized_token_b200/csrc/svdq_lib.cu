@@ -329,8 +329,13 @@ int quant_max_clusters(int c) {
 }
 
 // How the K range is split: `splits` CTAs per 128-row block; cluster mode
-// (cluster == splits) when those CTAs can form one cluster and every row
-// block's cluster is resident at once, else the workspace (cluster == 1).
+// (cluster == splits) when those CTAs form one cluster and every row block's
+// cluster is resident at once, else the workspace (cluster == 1).  The split
+// is never narrowed to fit a cluster: the quantizer warps bound the rate at
+// which a CTA streams its chunks, so fewer CTAs cost more than the
+// workspace's round trip (B200, M = 4608: three-CTA clusters on 108 SMs
+// against the workspace on 144 take 22.5 / 22.6 us at K = 3072 and 49.2 /
+// 43.0 us at K = 12288).
 struct QuantPlan {
     int splits, cluster;
 };
@@ -341,8 +346,7 @@ QuantPlan quant_plan(int64_t M, int64_t K, int rank) {
     if (mode == 1) return {sp, 1};
     if (mode == 2) return {std::min(sp, qa::kMaxCluster), std::min(sp, qa::kMaxCluster)};
     const int64_t row_blocks = (M + qa::kRows - 1) / qa::kRows;
-    for (int c = std::min(sp, qa::kMaxCluster); c >= 2; --c)
-        if (quant_max_clusters(c) >= row_blocks) return {c, c};
+    if (sp <= qa::kMaxCluster && quant_max_clusters(sp) >= row_blocks) return {sp, sp};
     return {sp, 1};
 }
 

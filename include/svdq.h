@@ -148,10 +148,11 @@ svdq_status svdq_replicate_weight_scales(void* w_scales, int64_t N, int64_t K, s
 
 /* Bytes of the workspace svdq_quantize_act needs for this shape (0 when it
  * needs none).  When K is split across several CTAs, each computes a partial
- * rank-r product.  The CTAs of a 128-row block normally form one thread-block
- * cluster and add their partials through distributed shared memory; when such
- * clusters cannot all be resident at once (fewer SMs available than the split
- * needs), they add them through this workspace instead: fp32 partial sums
+ * rank-r product.  The CTAs of a 128-row block form one thread-block cluster
+ * and add their partials through distributed shared memory when the split
+ * fits one cluster (at most 8 CTAs) and all row blocks' clusters can be
+ * resident at once; otherwise (on a B200, the M = 4608 layers of a 3072-wide
+ * DiT among them) they add them through this workspace: fp32 partial sums
  * plus one counter per 128-row block.  The size returned covers that case;
  * a call that runs in cluster mode leaves the workspace untouched.
  * Pure host function; errors as svdq_buffer_sizes. */

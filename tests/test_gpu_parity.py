@@ -36,6 +36,7 @@ SMALL = [
     W.scaled(W.QKV, M=129, K=512, N=384, rank=0, name="rank0"),
     W.scaled(W.QKV, M=256, K=768, N=256, rank=128, name="r128"),
     W.scaled(W.FC2, M=130, K=2048, N=512, rank=32, name="fc2_small"),
+    W.scaled(W.FC2, M=260, K=3136, N=272, rank=32, name="streamed_scales_ragged"),   # K > 3072, 49 k-steps
     W.scaled(W.QKV, M=1, K=64, N=16, rank=16, name="minimal"),
 ]
 
