@@ -475,6 +475,17 @@ __global__ void __launch_bounds__(gp_threads<kEpi>(), 1)
             prefetch_tensormap(&tm_Lup);
         }
     }
+    if (warp == 1 && lane == 0 && t_begin < t_end) {
+        // the first stages' weight codes and replicated weight scales are
+        // packed long before this call: start pulling them into the L2 while
+        // the previous kernel finishes
+        const int n_tile = t_begin % a.n_tiles;
+        const int n0 = n_tile * BN + 128 * (int)rank;
+        for (int kb = 0; kb < kStages && kb < n_kb; ++kb) {
+            tma_prefetch_l2_2d(&tm_wc, kb * BK_BYTES, n0);
+            tma_prefetch_l2_3d(&tm_sfb, 0, 0, n_tile * n_kb + kb);
+        }
+    }
     if (warp == kMmaWarp) {   // the same warp in both CTAs, the same slot offset
         tmem_alloc_pair(tmem_slot, TMEM_COLS);
         tmem_relinquish_pair();
