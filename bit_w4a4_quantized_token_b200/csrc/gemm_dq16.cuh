@@ -70,19 +70,24 @@ __host__ __device__ constexpr uint32_t idesc_f16_f32(uint32_t n) {
 }
 
 // 8 int4 codes (two's complement, element i in bits 4i+3..4i) times the fp16
-// scale pair s2 -> 8 fp16 values in element order (four fp16x2 words).  The
-// nibble n is q + 8 after flipping its top bit, and the fp16 with bits
-// 0x6400 | (q + 8) is 1024 + q + 8; subtracting 1032 leaves q exactly.
+// scale pair s2 -> 8 fp16 values in element order (four fp16x2 words).  After
+// flipping the top bit of every nibble, nibble n = q + 8.  For the byte b
+// holding elements 2p and 2p+1, one byte permute puts b in both halves of a
+// word and one mask-and-or makes the fp16 pair (1024 + n_lo, 1024 + 16 n_hi);
+// one fp16 fma with (1, 1/16) and (-1032, -72) leaves (q_lo, q_hi) exactly
+// (every step is exact: integers and power-of-two scalings well inside fp16's
+// range), and the multiply by the scale rounds once, as q s is exact anyway.
 __device__ __forceinline__ void int4x8_to_f16(uint32_t w, __half2 s2, uint32_t (&out)[4]) {
     const uint32_t u = w ^ 0x88888888u;
-    const __half2 bias2 = __halves2half2(__ushort_as_half(0x6408), __ushort_as_half(0x6408));   // 1032
+    const __half2 mul2 = __halves2half2(__ushort_as_half(0x3C00), __ushort_as_half(0x2C00));   // 1, 1/16
+    const __half2 add2 = __halves2half2(__ushort_as_half(0xE408), __ushort_as_half(0xD480));   // -1032, -72
 #pragma unroll
     for (int p = 0; p < 4; ++p) {
-        // elements 2p (bits 8p..8p+3) and 2p+1 (bits 8p+4..8p+7)
-        const uint32_t lo = (u >> (8 * p)) & 0xFu, hi = (u >> (8 * p + 4)) & 0xFu;
-        const uint32_t bits = (0x6400u | lo) | ((0x6400u | hi) << 16);
+        // bytes (b_p, 0, b_p, 0): selector nibbles p, 4 (a zero byte), p, 4
+        const uint32_t x = __byte_perm(u, 0u, (uint32_t)(0x4040 | (p << 8) | p));
+        const uint32_t bits = (x & 0x00F0000Fu) | 0x64006400u;
         __half2 v = *reinterpret_cast<const __half2*>(&bits);
-        v = __hmul2(__hsub2(v, bias2), s2);
+        v = __hmul2(__hfma2(v, mul2, add2), s2);
         out[p] = *reinterpret_cast<const uint32_t*>(&v);
     }
 }
