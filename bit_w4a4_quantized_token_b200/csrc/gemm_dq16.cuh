@@ -19,34 +19,47 @@
 // rescale is left for the CUDA cores.  The rank-r term runs as bf16 MMAs
 // (the hi and lo parts of L against L_up) into the same accumulator.
 //
-// One CTA per 128 x 256 output tile.  Warp 0 loads, per 64 columns of K, the
-// activation tile (bf16 x, or int4 codes and their group scales), the packed
-// weight tile (256 rows x 32 bytes) and its 256 group scales; warps 4..19
-// expand both into fp16 tiles in the MMA's swizzled layout (x converted in
-// place); warp 1 issues four M = 128, N = 256, K = 16 MMAs per stage into
-// TMEM; after the last stage warps 12..19 add the bias and store bf16.  The
-// expansion sets the pace, so every warp that would otherwise wait for the
-// accumulator takes part in it.
+// One CTA per 128 x 256 output tile, computed transposed: the tensor core
+// takes the weights as its A operand from TMEM and the activations as B from
+// shared memory, two M = 128 (weight rows), N = 128 (activation rows), K = 16
+// MMAs per 16 values of K into two TMEM accumulators.  Warp 0 loads, per 64
+// columns of K, the activation tile (bf16 x, or int4 codes and their group
+// scales), the packed weight tile (256 rows x 32 bytes) and its 256 group
+// scales; warps 4..19 expand the activations into an fp16 tile in the MMA's
+// swizzled layout in shared memory and the weights into fp16 rows of TMEM
+// (tcgen05.st: lane = weight row, two values per column); warp 1 issues the
+// MMAs; after the last stage warps 12..19 add the bias and store bf16,
+// transposing through shared memory.  Expanding the weights into TMEM instead
+// of shared memory takes their 32 KB per stage of stores and tensor-core reads
+// off the shared-memory pipe, which the expansion and the MMAs otherwise
+// saturate.  The rank-r chunks (already bf16) are multiplied from shared
+// memory (L_up as A, L as B).
 #pragma once
 #include "sm100_ptx.cuh"
 
 namespace svdq {
 namespace dq {
-constexpr int BM = 128;
-constexpr int BN = 256;
-constexpr int kStages = 3;
-constexpr int A_BYTES = 128 * 128;            // fp16 A: 128 rows x 64 values (x arrives here as bf16)
-constexpr int WF_BYTES = 256 * 128;           // fp16 weights: 256 rows x 64 values
-constexpr int WP_BYTES = 256 * 32;            // packed int4 weights: 256 rows x 64 codes
+constexpr int BM = 128;                       // activation rows per tile
+constexpr int BN = 256;                       // weight rows per tile
+constexpr int kStages = 4;
+constexpr int XF_BYTES = 128 * 128;           // fp16 activations: 128 rows x 64 values (x arrives here as bf16;
+                                              // a rank-r chunk's bf16 L tile)
 constexpr int AP_BYTES = 128 * 32;            // packed int4 activations: 128 rows x 64 codes
+constexpr int WP_BYTES = 256 * 32;            // packed int4 weights: 256 rows x 64 codes
 constexpr int WS_BYTES = 256 * 2;             // bf16 group scales of the 256 weight rows
 constexpr int AS_BYTES = 128 * 2;             // bf16 group scales of the 128 activation rows
-constexpr int OFF_WF = A_BYTES;
-constexpr int OFF_WP = OFF_WF + WF_BYTES;
-constexpr int OFF_AP = OFF_WP + WP_BYTES;
-constexpr int OFF_WS = OFF_AP + AP_BYTES;
+constexpr int OFF_AP = XF_BYTES;
+constexpr int OFF_WP = OFF_AP + AP_BYTES;
+constexpr int OFF_WS = OFF_WP + WP_BYTES;
 constexpr int OFF_AS = OFF_WS + WS_BYTES;
-constexpr int STAGE_BYTES = ((OFF_AS + AS_BYTES + 1023) / 1024) * 1024;
+constexpr int OFF_LUP = XF_BYTES;             // a rank-r chunk's L_up tile: 256 rows x 64 bf16 (two 16 KB halves)
+constexpr int LUP_BYTES = 256 * 128;
+constexpr int STAGE_BYTES = XF_BYTES + LUP_BYTES;   // a rank-r chunk is the largest stage
+static_assert(OFF_AS + AS_BYTES <= STAGE_BYTES, "packed tiles do not fit in a stage");
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t D_COL = 0;                 // weight rows 0-127 at column 0, rows 128-255 at 128 (fp32)
+constexpr uint32_t WT_COL = 256;              // stage s: fp16 weight rows 0-127 at 256 + 64 s, rows 128-255 at + 32
+static_assert(WT_COL + 64 * kStages <= TMEM_COLS, "weight tiles do not fit in TMEM");
 constexpr int kConvWarp0 = 4, kConvWarps = 16;   // the epilogue warps convert too
 constexpr int kEpiWarp0 = 12, kEpiWarps = 8;
 constexpr int kThreads = 32 * (kEpiWarp0 + kEpiWarps);
@@ -67,6 +80,19 @@ __host__ __device__ constexpr uint32_t idesc_f16_f32(uint32_t n) {
     return (1u << 4)            // D format f32; A and B format f16 (0)
            | ((n >> 3) << 17)   // N / 8
            | ((128u >> 4) << 24);  // M / 16
+}
+
+// D[tmem] (+)= A[tmem] * B[smem]^T, fp16 inputs, fp32 accumulate.  A sits in
+// TMEM with lane = row and two consecutive K values per 32-bit column (low
+// half first), so one K = 16 instruction reads 8 columns.
+__device__ __forceinline__ void mma_f16_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                               uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
 }
 
 // 8 int4 codes (two's complement, element i in bits 4i+3..4i) times the fp16
@@ -147,7 +173,7 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
         }
     }
     if (warp == 1) {
-        tmem_alloc(tmem_slot, 256);
+        tmem_alloc(tmem_slot, TMEM_COLS);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -173,7 +199,7 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
                         tma_load_2d(st + OFF_AP, &tm_a, &full[s], kc * 32, m0);
                         tma_load_2d(st + OFF_AS, &tm_as, &full[s], m0, kc);
                     } else {
-                        mbar_arrive_expect_tx(&full[s], A_BYTES + WP_BYTES + WS_BYTES);
+                        mbar_arrive_expect_tx(&full[s], XF_BYTES + WP_BYTES + WS_BYTES);
                         tma_load_2d(st, &tm_a, &full[s], kc * 64, m0);
                     }
                     tma_load_2d(st + OFF_WP, &tm_wc, &full[s], kc * 32, n0);
@@ -181,9 +207,9 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
                 } else {
                     // rank-r chunk: an L tile (hi or lo plane) and an L_up tile, already bf16
                     const int c = (it - n_kc) >> 1, part = (it - n_kc) & 1;
-                    mbar_arrive_expect_tx(&full[s], A_BYTES + WF_BYTES);
+                    mbar_arrive_expect_tx(&full[s], XF_BYTES + LUP_BYTES);
                     tma_load_3d(st, &tm_L, &full[s], c * 64, m0, part);
-                    tma_load_2d(st + OFF_WF, &tm_Lup, &full[s], c * 64, n0);
+                    tma_load_2d(st + OFF_LUP, &tm_Lup, &full[s], c * 64, n0);
                 }
                 reinterpret_cast<volatile int*>(s_issued)[s] += 1;
             }
@@ -191,8 +217,8 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
     } else if (warp == 1) {
         // ---------------------------------------------------------- MMA issuer
         if (lane == 0) {
-            const uint32_t idesc = idesc_m(idesc_f16_f32(BN), BM);
-            const uint32_t idesc_lr = idesc_m(idesc_bf16_f32(BN), BM);
+            const uint32_t idesc = idesc_f16_f32(128);     // M = 128 weight rows, N = 128 activation rows
+            const uint32_t idesc_lr = idesc_bf16_f32(128);
             bool ok = true;
             for (int it = 0; it < n_st; ++it) {
                 const int s = it % kStages;
@@ -202,17 +228,24 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
                     break;
                 }
                 tc_fence_after();
-                const uint32_t sx = smem_u32(smem + (size_t)s * STAGE_BYTES), sw = sx + OFF_WF;
+                const uint32_t sx = smem_u32(smem + (size_t)s * STAGE_BYTES);
                 if (it < n_kc) {
+                    const uint32_t wt = tmem + WT_COL + 64u * (uint32_t)s;
 #pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        mma_bf16(tmem, desc_sw128(sx + 32u * j), desc_sw128(sw + 32u * j), idesc,
-                                 (it > 0 || j > 0) ? 1u : 0u);
+                    for (int j = 0; j < 4; ++j) {
+                        const uint64_t bd = desc_sw128(sx + 32u * j);
+                        const uint32_t acc = (it > 0 || j > 0) ? 1u : 0u;
+                        mma_f16_tmem_a(tmem + D_COL, wt + 8u * j, bd, idesc, acc);
+                        mma_f16_tmem_a(tmem + D_COL + 128u, wt + 32u + 8u * j, bd, idesc, acc);
+                    }
                 } else {
                     const int c = (it - n_kc) >> 1;
                     const int nks = min(4, (a.rank - 64 * c + 15) / 16);
-                    for (int j = 0; j < nks; ++j)
-                        mma_bf16(tmem, desc_sw128(sx + 32u * j), desc_sw128(sw + 32u * j), idesc_lr, 1u);
+                    for (int j = 0; j < nks; ++j) {
+                        const uint64_t bd = desc_sw128(sx + 32u * j);
+                        mma_bf16(tmem + D_COL, desc_sw128(sx + OFF_LUP + 32u * j), bd, idesc_lr, 1u);
+                        mma_bf16(tmem + D_COL + 128u, desc_sw128(sx + OFF_LUP + 16384u + 32u * j), bd, idesc_lr, 1u);
+                    }
                 }
                 tc_commit(&empty[s]);
             }
@@ -220,7 +253,11 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
         }
     } else if (warp >= (uint32_t)kConvWarp0) {
         // ----------------------------------- activations and weights -> fp16
-        const int t = (int)threadIdx.x - 32 * kConvWarp0;   // 0..511: half of weight row t / 2
+        const int t = (int)threadIdx.x - 32 * kConvWarp0;        // 0..511
+        const uint32_t q = warp & 3u;                            // this warp's TMEM lane quadrant
+        const int j = (int)(warp - (uint32_t)kConvWarp0) >> 2;   // 0..3: weight half j / 2, K half j % 2
+        const int wr = 128 * (j >> 1) + 32 * (int)q + (int)lane; // weight row of this thread
+        const int kh = j & 1;
         for (int it = 0; it < n_st; ++it) {
             const int s = it % kStages;
             if (!mbar_wait(&full[s], (uint32_t)(it / kStages) & 1u, kSiteDqFull)) {
@@ -259,21 +296,20 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
                         *p = make_uint4(o[0], o[1], o[2], o[3]);
                     }
                 }
-                // weight row t / 2, codes 32 (t % 2) .. + 31 -> fp16 (q s_w) in the swizzled 128-byte row
-                const int wr = t >> 1, wh = t & 1;
-                const uint8_t* wp = st + OFF_WP + 32 * wr + 16 * wh;
+                // weight row wr, K values 32 kh .. + 31 -> fp16 (q s_w) in TMEM columns
+                // 16 kh .. + 15 of its half's tile (lane = row)
                 const __half2 s2 = bf16_scale_to_h2(*reinterpret_cast<const uint16_t*>(st + OFF_WS + 2 * wr));
-                const uint4 c0 = *reinterpret_cast<const uint4*>(wp);
+                const uint4 c0 = *reinterpret_cast<const uint4*>(st + OFF_WP + 32 * wr + 16 * kh);
                 const uint32_t cw[4] = {c0.x, c0.y, c0.z, c0.w};
-                uint8_t* wrow = st + OFF_WF + wr * 128;
+                uint32_t o[16];
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {   // 16-byte chunk 4 wh + c: K values 8 (4 wh + c) .. + 7
-                    uint32_t o[4];
-                    int4x8_to_f16(cw[c], s2, o);
-                    *reinterpret_cast<uint4*>(wrow + (((4 * wh + c) ^ (wr & 7)) << 4)) =
-                        make_uint4(o[0], o[1], o[2], o[3]);
-                }
-                fence_proxy_async_smem();   // both tiles are read by the tensor core
+                for (int c = 0; c < 4; ++c) int4x8_to_f16(cw[c], s2, *reinterpret_cast<uint32_t(*)[4]>(o + 4 * c));
+                tmem_st_32x32b_x16(tmem + ((32u * q) << 16) + WT_COL + 64u * (uint32_t)s + 32u * (uint32_t)(j >> 1) +
+                                       16u * (uint32_t)kh,
+                                   o);
+                tmem_st_wait();
+                fence_proxy_async_smem();   // the activation tile is read by the tensor core
+                tc_fence_before();
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&conv[s]);
@@ -281,36 +317,40 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
     }
     if (warp >= (uint32_t)kEpiWarp0) {
         // ------------------------------------------------------------ epilogue
+        // lane = weight row n, TMEM columns = activation rows; each 32 x 32
+        // block goes out through this warp's 2 KB of the (now idle) ring as
+        // 32 rows of 64 bytes
         const uint32_t q = warp & 3u;
         const int half = (int)(warp - kEpiWarp0) >> 2;
-        const int64_t grow = (int64_t)m0 + 32 * q + lane;
+        const int nl = 128 * half + 32 * (int)q;               // first weight row of this warp
+        const int n = n0 + nl + (int)lane;
         const bool ok = mbar_wait(acc_full, 0, kSiteDqAcc);
         if (!ok) s_failed = 1;
         tc_fence_after();
         if (ok) {
-            __nv_bfloat16* yrow = a.y + grow * (int64_t)a.N;
+            float bv = 0.0f;
+            if (a.bias != nullptr && n < a.N) bv = __bfloat162float(a.bias[n]);
+            uint16_t* stg = reinterpret_cast<uint16_t*>(smem + (size_t)(warp - kEpiWarp0) * 2048);
 #pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
+            for (int c0 = 0; c0 < BM; c0 += 32) {
                 uint32_t acc[32];
-                tmem_ld_32x32b_x32(tmem + ((32u * q) << 16) + 128u * half + 32u * c, acc);
+                tmem_ld_32x32b_x32(tmem + ((32u * q) << 16) + D_COL + 128u * (uint32_t)half + (uint32_t)c0, acc);
                 tmem_ld_wait();
-                const int n = n0 + 128 * half + 32 * c;
 #pragma unroll
-                for (int p = 0; p < 4; ++p) {
-                    if (n + 8 * p >= a.N) break;   // N % 16 == 0
-                    uint4 bw = make_uint4(0u, 0u, 0u, 0u);
-                    if (a.bias) bw = __ldg(reinterpret_cast<const uint4*>(a.bias + n + 8 * p));
-                    const uint32_t ws[4] = {bw.x, bw.y, bw.z, bw.w};
-                    uint32_t pk[4];
+                for (int i = 0; i < 32; ++i)
+                    stg[i * 32 + (int)lane] =
+                        __bfloat16_as_ushort(__float2bfloat16_rn(__fadd_rn(__uint_as_float(acc[i]), bv)));
+                __syncwarp();
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const float o0 = __fadd_rn(__uint_as_float(acc[8 * p + 2 * i]), bf16lo_to_f32(ws[i]));
-                        const float o1 = __fadd_rn(__uint_as_float(acc[8 * p + 2 * i + 1]), bf16hi_to_f32(ws[i]));
-                        const __nv_bfloat162 h2 = __floats2bfloat162_rn(o0, o1);
-                        pk[i] = *reinterpret_cast<const uint32_t*>(&h2);
-                    }
-                    if (grow < a.M) *reinterpret_cast<uint4*>(yrow + n + 8 * p) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                for (int k = 0; k < 4; ++k) {
+                    const int i = (int)(lane >> 2) + 8 * k, ch = (int)(lane & 3u);
+                    const int64_t m = (int64_t)m0 + c0 + i;
+                    const int ncol = n0 + nl + 8 * ch;
+                    if (m < a.M && ncol < a.N)
+                        *reinterpret_cast<uint4*>(a.y + m * (int64_t)a.N + ncol) =
+                            *reinterpret_cast<const uint4*>(stg + i * 32 + 8 * ch);
                 }
+                __syncwarp();
             }
         }
     }
@@ -326,7 +366,7 @@ __global__ void __launch_bounds__(dq::kThreads, 1)
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, 256);
+        tmem_dealloc(tmem, TMEM_COLS);
     }
 }
 
