@@ -51,19 +51,45 @@ struct QuantActArgs {
     uint8_t* x_scales;         // nvfp4: scale-factor layout; int4: bf16 [K/64, rows_pad]
     __nv_bfloat16* lowrank;    // [2, M, rank]: hi and lo bf16 planes
     float* partials;           // workspace mode: [row_blocks, splits, 128, rank] fp32
-    unsigned int* counters;    // workspace mode: [row_blocks]; zero between calls
+    unsigned int* counters;    // workspace mode: [row_blocks][2] (partials written, slices added); zero between calls
     int M, K, rank;
     int rows_pad;              // M rounded up to 128
     int chunks;                // K / 64
     int splits;                // CTAs sharing one 128-row block (blockIdx.x)
     int cluster;               // == splits in cluster mode, else 1
+    int coop;                  // workspace mode, whole grid resident at once: every split adds a slice of rows
     int stages;
     uint32_t stage_bytes;      // x tile + hi/lo L_down_t tiles + 1/lambda chunk, rounded to 1 KB
     uint32_t invl_off;         // offset of the 1/lambda chunk in a stage
     uint32_t tmem_cols;
 };
 
-enum : uint32_t { kSiteQaEmpty = 1, kSiteQaFullMma = 2, kSiteQaFullWork = 3, kSiteQaAcc = 4, kSiteQaDrain = 5 };
+enum : uint32_t {
+    kSiteQaEmpty = 1,
+    kSiteQaFullMma = 2,
+    kSiteQaFullWork = 3,
+    kSiteQaAcc = 4,
+    kSiteQaDrain = 5,
+    kSiteQaSplits = 6
+};
+
+// Bounded wait until the global counter reaches `target` (acquire): the other
+// CTAs of a K split writing their partials.  False (and the timeout recorded)
+// after the wait limit.
+__device__ __noinline__ bool qa_wait_count(const unsigned int* p, unsigned int target, uint32_t site) {
+    const uint64_t t0 = globaltimer_ns();
+    const uint64_t limit = g_wait_limit_ns;
+    while (true) {
+        unsigned int v;
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+        if (v >= target) return true;
+        if (globaltimer_ns() - t0 > limit) {
+            record_timeout(site);
+            return false;
+        }
+        __nanosleep(64);
+    }
+}
 
 // L' = v * inv_ss as a bf16 hi/lo pair for two adjacent columns.
 __device__ __forceinline__ void store_lowrank_pair(__nv_bfloat16* hi_dst, __nv_bfloat16* lo_dst, float v0, float v1,
@@ -370,26 +396,38 @@ __global__ void __launch_bounds__(qa::kThreads, 1)
                     *reinterpret_cast<float4*>(mine + c0 + i) = make_float4(v16[i], v16[i + 1], v16[i + 2], v16[i + 3]);
             }
             if (workspace_mode) {
+                // the partials are added in split order, one row and 4 columns
+                // per item, consecutive threads on consecutive columns, the
+                // loads of up to four splits issued before the first add:
+                //  * coop (the whole grid resident at once): once every split
+                //    has written its partial, split s adds rows
+                //    [128 s / splits, 128 (s + 1) / splits); the last to finish
+                //    zeroes the two counters;
+                //  * otherwise the last CTA to write its partial adds all rows.
+                unsigned int* cnt = a.counters + 2 * rb;   // [0]: partials written, [1]: slices added
                 __threadfence();
                 named_bar_sync(2, qa::kWorkers);
                 if (threadIdx.x == 32 * qa::kWorker0) {
-                    const unsigned int prev = atomicAdd(a.counters + rb, 1u);
-                    s_last = (prev == (unsigned int)(a.splits - 1)) ? 1 : 0;
+                    const unsigned int prev = atomicAdd(cnt, 1u);
+                    if (a.coop) {
+                        s_last = qa_wait_count(cnt, (unsigned int)a.splits, kSiteQaSplits) ? 1 : 0;
+                        if (!s_last) s_failed = 1;
+                    } else {
+                        s_last = (prev == (unsigned int)(a.splits - 1)) ? 1 : 0;
+                    }
+                    __threadfence();
                 }
                 named_bar_sync(2, qa::kWorkers);
                 if (s_last) {
-                    // the last CTA of this row block adds the partials in split
-                    // order, one row and 4 columns per item, consecutive threads
-                    // on consecutive columns; the loads of up to four splits are
-                    // issued before the first add
-                    __threadfence();
                     const int t = (int)threadIdx.x - 32 * qa::kWorker0;
                     const int q4 = a.rank / 4;
+                    const int r_lo = a.coop ? qa::kRows * split / a.splits : 0;
+                    const int r_hi = a.coop ? qa::kRows * (split + 1) / a.splits : qa::kRows;
                     const int64_t plane = (int64_t)a.M * a.rank;
                     const float* base = a.partials + (int64_t)rb * a.splits * qa::kRows * a.rank;
                     const int64_t pstep = (int64_t)qa::kRows * a.rank;
-                    for (int i = t; i < qa::kRows * q4; i += qa::kWorkers) {
-                        const int rl = i / q4, c0 = 4 * (i - rl * q4);
+                    for (int i = t; i < (r_hi - r_lo) * q4; i += qa::kWorkers) {
+                        const int rl = r_lo + i / q4, c0 = 4 * (i % q4);
                         const float* src = base + (int64_t)rl * a.rank + c0;
                         float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
                         for (int p0 = 0; p0 < a.splits; p0 += 4) {
@@ -413,7 +451,15 @@ __global__ void __launch_bounds__(qa::kThreads, 1)
                             store_lowrank_pair(hi + 2, hi + 2 + plane, acc.z, acc.w, inv_ss);
                         }
                     }
-                    if (t == 0) a.counters[rb] = 0u;   // ready for the next call
+                    if (t == 0) {
+                        if (!a.coop) {
+                            cnt[0] = 0u;   // ready for the next call
+                        } else if (atomicAdd(cnt + 1, 1u) == (unsigned int)(a.splits - 1)) {
+                            // every split has passed its wait: ready for the next call
+                            cnt[0] = 0u;
+                            cnt[1] = 0u;
+                        }
+                    }
                 }
             }
         }

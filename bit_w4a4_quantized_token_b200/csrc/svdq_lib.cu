@@ -286,6 +286,9 @@ int quant_splits(int64_t M, int64_t K) {
     return (int)std::max<int64_t>(sp, 1);
 }
 
+// The workspace plan's two counters per 128-row block, ahead of the partials.
+size_t quant_counter_bytes(int64_t row_blocks) { return (size_t)round_up(row_blocks * 8, 256); }
+
 // Workspace of the K-split when its CTAs add their rank-r partials through
 // global memory (the upper bound: a launch that runs in cluster mode leaves
 // the workspace untouched).
@@ -293,7 +296,7 @@ size_t quant_workspace_bytes(int64_t M, int64_t K, int rank) {
     const int sp = quant_splits(M, K);
     if (rank == 0 || sp == 1) return 0;
     const int64_t row_blocks = (M + qa::kRows - 1) / qa::kRows;
-    return (size_t)round_up(row_blocks * 4, 256) + (size_t)row_blocks * sp * qa::kRows * rank * 4;
+    return quant_counter_bytes(row_blocks) + (size_t)row_blocks * sp * qa::kRows * rank * 4;
 }
 
 // Clusters of `c` quantizer CTAs that can be resident at once on the current
@@ -412,8 +415,11 @@ svdq_status quantize_act_launch(int prec, const void* x, int64_t M, int64_t K, c
     a.cluster = plan.cluster;
     a.counters = reinterpret_cast<unsigned int*>(workspace);
     a.partials = workspace ? reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(workspace) +
-                                                       round_up(row_blocks * 4, 256))
+                                                       quant_counter_bytes(row_blocks))
                            : nullptr;
+    // the splits of a row block wait for one another only when the whole grid
+    // (one CTA per SM) is resident at once
+    a.coop = (plan.cluster == 1 && plan.splits > 1 && (int64_t)plan.splits * row_blocks <= num_sms()) ? 1 : 0;
     // stage: x tile, hi and lo L_down_t tiles, the chunk's 1/lambda; 1 KB aligned (128-byte swizzle)
     a.invl_off = (uint32_t)qa::kXBytes + (uint32_t)rank * 256u;
     a.stage_bytes = (uint32_t)round_up((int64_t)a.invl_off + qa::kInvlBytes, 1024);
@@ -916,7 +922,7 @@ svdq_status svdq_quantize_act_noalloc(svdq_precision p, int group_size, const vo
         SVDQ_TRY(noalloc_workspace_address(&ws));
         // the array keeps the previous call's contents: its counters must start at zero
         const int64_t row_blocks = (M + qa::kRows - 1) / qa::kRows;
-        if (cudaMemsetAsync(ws, 0, (size_t)round_up(row_blocks * 4, 256), reinterpret_cast<cudaStream_t>(stream)) !=
+        if (cudaMemsetAsync(ws, 0, quant_counter_bytes(row_blocks), reinterpret_cast<cudaStream_t>(stream)) !=
             cudaSuccess)
             return cuda_fail("cudaMemsetAsync(no-alloc workspace counters)");
     }

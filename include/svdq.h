@@ -153,7 +153,11 @@ svdq_status svdq_replicate_weight_scales(void* w_scales, int64_t N, int64_t K, s
  * fits one cluster (at most 8 CTAs) and all row blocks' clusters can be
  * resident at once; otherwise (on a B200, the M = 4608 layers of a 3072-wide
  * DiT among them) they add them through this workspace: fp32 partial sums
- * plus one counter per 128-row block.  The size returned covers that case;
+ * plus two counters per 128-row block.  When the whole grid is resident at
+ * once (one CTA per SM, no more CTAs than SMs) every CTA of the split adds a
+ * slice of the block's rows once all partials are written (a bounded wait
+ * on a counter; SVDQ_ERR_TIMEOUT at the wait limit); otherwise the last CTA
+ * to write its partial adds them all.  The size returned covers either case;
  * a call that runs in cluster mode leaves the workspace untouched.
  * Pure host function; errors as svdq_buffer_sizes. */
 svdq_status svdq_quantize_act_workspace_bytes(svdq_precision precision, int64_t M, int64_t K, int rank,

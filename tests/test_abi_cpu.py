@@ -165,8 +165,9 @@ def test_force_quant_plan_hook(L):
 
 
 def test_quantize_act_workspace_bytes(L):
-    # QKV shape: 36 row blocks x 4 K-splits x 128 rows x rank 32 fp32, plus a 256-byte counter block
-    assert L.svdq_quantize_act_workspace_bytes("nvfp4", 4608, 3072, 32) == 256 + 36 * 4 * 128 * 32 * 4
+    # QKV shape: 36 row blocks x 4 K-splits x 128 rows x rank 32 fp32, plus two counters per row block
+    # (36 x 8 bytes, rounded up to 512)
+    assert L.svdq_quantize_act_workspace_bytes("nvfp4", 4608, 3072, 32) == 512 + 36 * 4 * 128 * 32 * 4
     # 144 row blocks fill the GPU without a K split: no workspace
     assert L.svdq_quantize_act_workspace_bytes("nvfp4", 18432, 3072, 32) == 0
     assert L.svdq_quantize_act_workspace_bytes("int4", 4608, 3072, 0) == 0
