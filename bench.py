@@ -237,7 +237,7 @@ class ClockSampler:
             reasons = sorted({name for _, _, bits in rows for name, bit in self.REASON_BITS if bits & bit})
             return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": self.max_mhz,
                     "reasons": reasons, "samples": len(rows), "power_w_max": max(r[1] for r in rows),
-                    "source": "NVML every 1 ms during the timed region"}
+                    "source": "NVML every 1 ms during the timed graphs"}
         sm, smax, power, reasons = [], [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for _, ln in self.lines:
@@ -790,8 +790,12 @@ def run_cuda(args) -> dict | None:
     time.sleep(0.05)
     if world > 1:
         dist.barrier()
-    t = time_graphs(sh, gs, args.steps, flush, sampler)
+    # clocks are taken over all the timed graphs (back to back, then one step
+    # per flush): the step graph alone lasts only a few milliseconds
+    sampler.begin()
+    t = time_graphs(sh, gs, args.steps, flush)
     t_fl = time_graphs_flushed(sh, gs1, flushed_steps, flush)
+    sampler.end()
     if world > 1:
         dist.barrier()
     clocks = sampler.stop()
