@@ -696,6 +696,35 @@ def time_graphs(shape, gs, steps, flush, sampler=None):
     return res
 
 
+def time_sustained(shape, flush, steps: int) -> dict:
+    """The headline step for long enough (~40 ms back to back) that the SM
+    clock settles under the board's power cap; the headline's `--steps` steps
+    are a few milliseconds, most of them before it does."""
+    import torch
+
+    st = shape.stream
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=st):
+        for i in range(steps):
+            shape.quant(k=i % shape.sets)
+            shape.gemm(k=i % shape.sets)
+    g.replay()
+    with torch.cuda.stream(st):
+        flush.fill_(5)
+    torch.cuda.synchronize(shape.dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(st):
+        e0.record(st)
+        g.replay()
+        e1.record(st)
+    torch.cuda.synchronize(shape.dev)
+    t = e0.elapsed_time(e1) / steps / 1e3
+    del g
+    return {"workload": workload_config(shape.case, False, 1)["workload"], "steps": steps,
+            "step_us": round(t * 1e6, 2), "value": round(shape.case.flops / t / 1e12, 2), "unit": UNIT,
+            "timing": f"{steps} steps back to back in one CUDA graph, rotating input sets as the headline"}
+
+
 def time_graphs_flushed(shape, gs1, steps, flush):
     """The same per step with a 256 MiB L2 flush before every single-step
     replay (outside the events).  Each event pair then also holds the ~6 us a
@@ -890,6 +919,7 @@ def run_cuda(args) -> dict | None:
         torch.cuda.empty_cache()
         extra["svd_split_qkv"] = time_svd_split(dev, stream, flush, 3)
         torch.cuda.empty_cache()
+        extra[f"{case.name}_sustained"] = time_sustained(sh, flush, 400)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
