@@ -346,7 +346,7 @@ QuantPlan quant_plan(int64_t M, int64_t K, int rank) {
     const int sp = quant_splits(M, K);
     if (rank == 0 || sp == 1) return {sp, 1};
     const int mode = g_quant_plan_mode.load();
-    if (mode == 1) return {sp, 1};
+    if (mode == 1 || mode == 3) return {sp, 1};
     if (mode == 2) return {std::min(sp, qa::kMaxCluster), std::min(sp, qa::kMaxCluster)};
     const int64_t row_blocks = (M + qa::kRows - 1) / qa::kRows;
     if (sp <= qa::kMaxCluster && quant_max_clusters(sp) >= row_blocks) return {sp, sp};
@@ -419,7 +419,10 @@ svdq_status quantize_act_launch(int prec, const void* x, int64_t M, int64_t K, c
                            : nullptr;
     // the splits of a row block wait for one another only when the whole grid
     // (one CTA per SM) is resident at once
-    a.coop = (plan.cluster == 1 && plan.splits > 1 && (int64_t)plan.splits * row_blocks <= num_sms()) ? 1 : 0;
+    a.coop = (plan.cluster == 1 && plan.splits > 1 && (int64_t)plan.splits * row_blocks <= num_sms() &&
+              g_quant_plan_mode.load() != 3)
+                 ? 1
+                 : 0;
     // stage: x tile, hi and lo L_down_t tiles, the chunk's 1/lambda; 1 KB aligned (128-byte swizzle)
     a.invl_off = (uint32_t)qa::kXBytes + (uint32_t)rank * 256u;
     a.stage_bytes = (uint32_t)round_up((int64_t)a.invl_off + qa::kInvlBytes, 1024);
@@ -1257,8 +1260,9 @@ svdq_status svdq_debug_force_gemm_tiles(int mode) {
 }
 
 svdq_status svdq_debug_force_quant_plan(int mode) {
-    if (mode < 0 || mode > 2) {
-        snprintf(g_last_error, sizeof(g_last_error), "svdq_debug_force_quant_plan: mode %d is not 0, 1 or 2", mode);
+    if (mode < 0 || mode > 3) {
+        snprintf(g_last_error, sizeof(g_last_error), "svdq_debug_force_quant_plan: mode %d is not 0, 1, 2 or 3",
+                 mode);
         return SVDQ_ERR_INVALID_ARG;
     }
     g_quant_plan_mode.store(mode);

@@ -388,9 +388,12 @@ svdq_status svdq_device_status(int clear, int* site);
 svdq_status svdq_debug_set_wait_limit_ns(uint64_t ns);
 /* svdq_debug_force_quant_plan: how svdq_quantize_act adds the rank-r partials
  *    of a K split: 0 = automatic, 1 = always through the workspace (global
- *    memory, see svdq_quantize_act), 2 = always in one thread-block cluster
- *    through distributed shared memory.  Results are the same; tests use it to
- *    run both.  Any other value is SVDQ_ERR_INVALID_ARG. */
+ *    memory, see svdq_quantize_act_workspace_bytes; every split adds a slice
+ *    when the grid is resident at once), 2 = always in one thread-block
+ *    cluster through distributed shared memory, 3 = through the workspace
+ *    with the last CTA of a row block adding all of its rows (what a device
+ *    with fewer SMs than the grid's CTAs gets).  Results are the same; tests
+ *    use it to run every path.  Any other value is SVDQ_ERR_INVALID_ARG. */
 svdq_status svdq_debug_force_quant_plan(int mode);
 svdq_status svdq_debug_timeout_probe(svdq_stream_t stream);
 void svdq_debug_override_capability(int major, int minor);

@@ -154,14 +154,14 @@ def test_force_gemm_tiles_hook(L):
 
 
 def test_force_quant_plan_hook(L):
-    """Modes 0-2 are accepted (no device needed); anything else is rejected with a message."""
-    for mode in (1, 2, 0):
+    """Modes 0-3 are accepted (no device needed); anything else is rejected with a message."""
+    for mode in (1, 2, 3, 0):
         L.svdq_debug_force_quant_plan(mode)
-    for bad in (-1, 3):
+    for bad in (-1, 4):
         with pytest.raises(L.SvdqError) as e:
             L.svdq_debug_force_quant_plan(bad)
         assert e.value.status == L.SVDQ_ERR_INVALID_ARG
-        assert "not 0, 1 or 2" in L.lib.svdq_last_error().decode()
+        assert "not 0, 1, 2 or 3" in L.lib.svdq_last_error().decode()
 
 
 def test_quantize_act_workspace_bytes(L):

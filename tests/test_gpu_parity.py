@@ -60,9 +60,10 @@ def test_small_cases_each_gemm_kernel(case, mode):
         _lib.svdq_debug_force_gemm_tiles(0)
 
 
-# the two ways the quantizer adds the rank-r partials of a K split: through
-# the workspace (global memory) and inside one thread-block cluster
-# (distributed shared memory); a ragged tail, the largest cluster, rank 128
+# the ways the quantizer adds the rank-r partials of a K split: through the
+# workspace (global memory; every split adds a slice of rows, or the last CTA
+# adds all of them) and inside one thread-block cluster (distributed shared
+# memory); a ragged tail, the largest cluster, rank 128
 QUANT_PLAN_CASES = [
     W.scaled(W.QKV, M=300, K=1024, N=512, rank=64, name="qp_ragged_r64"),
     W.scaled(W.QKV, M=128, K=3072, N=256, rank=32, name="qp_one_block_k3072"),
@@ -71,7 +72,7 @@ QUANT_PLAN_CASES = [
 ]
 
 
-@pytest.mark.parametrize("mode", [1, 2], ids=["workspace", "cluster"])
+@pytest.mark.parametrize("mode", [1, 2, 3], ids=["workspace", "cluster", "workspace_last_cta"])
 @pytest.mark.parametrize("case", QUANT_PLAN_CASES, ids=lambda c: c.name)
 def test_quantizer_split_modes(case, mode):
     from bit_w4a4_quantized_token_b200 import _lib
