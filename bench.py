@@ -579,21 +579,32 @@ def time_gelu_mlp(dev, stream, flush, steps: int) -> dict:
     def fc2_unfused():
         layer.gemm(qu, p2, y2, stream=stream)
 
+    def fc1_gelu():   # fc1 with only the GELU in its epilogue, storing h
+        _lib.svdq_gemm_w4a4_gelu("nvfp4", 16, q1.x_codes, q1.x_scales, q1.x_tensor_scale, M, p1.w_codes, p1.w_scales,
+                                 p1.w_tensor_scale, Hd, c1.K, q1.lowrank_act, p1.L_up_t, c1.rank, p1.bias, 0, h,
+                                 stream=stream)
+
     t_f = _graph_time([s1.quant, fused_fc1, fc2_fused], stream, dev, flush, steps)
     t_u = _graph_time([s1.quant, fc1_plain, gelu, quant2, fc2_unfused], stream, dev, flush, steps)
+    t_g = _graph_time([s1.quant, fc1_gelu, quant2, fc2_unfused], stream, dev, flush, steps)
     t_f1 = _graph_time([fused_fc1], stream, dev, flush, steps)
     t_p1 = _graph_time([fc1_plain], stream, dev, flush, steps)
+    t_g1 = _graph_time([fc1_gelu], stream, dev, flush, steps)
     st, site = _lib.svdq_device_status(clear=True)
     if st != 0:
         raise RuntimeError(f"device status {st} at site {site} in the GELU MLP leg")
     flops = c1.flops + c2.flops
     return {"workload": "DiT MLP 3072 -> 12288 -> GELU -> 3072, rank 32 both layers, M=4608",
-            "step_us": {"fused": round(t_f * 1e6, 2), "unfused": round(t_u * 1e6, 2)},
+            "step_us": {"fused": round(t_f * 1e6, 2), "unfused": round(t_u * 1e6, 2),
+                        "gelu_epilogue": round(t_g * 1e6, 2)},
             "speedup": round(t_u / t_f, 3),
-            "fc1_us": {"gelu_quant_epilogue": round(t_f1 * 1e6, 2), "plain_epilogue": round(t_p1 * 1e6, 2)},
+            "speedup_gelu_epilogue": round(t_u / t_g, 3),
+            "fc1_us": {"gelu_quant_epilogue": round(t_f1 * 1e6, 2), "plain_epilogue": round(t_p1 * 1e6, 2),
+                       "gelu_epilogue": round(t_g1 * 1e6, 2)},
             "value": round(flops / t_f / 1e12, 2), "unit": UNIT,
             "fused_step": "quantize_act(fc1) + gemm_w4a4_gelu_quant(fc1) + gemm_w4a4(fc2)",
             "unfused_step": "quantize_act(fc1) + gemm_w4a4(fc1) + gelu + quantize_act(fc2) + gemm_w4a4(fc2)",
+            "gelu_epilogue_step": "quantize_act(fc1) + gemm_w4a4_gelu(fc1) + quantize_act(fc2) + gemm_w4a4(fc2)",
             "timing": FLUSHED_TIMING}
 
 

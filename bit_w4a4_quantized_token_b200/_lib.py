@@ -32,7 +32,7 @@ EXPORTS = (
     "svdq_replicate_weight_scales",
     "svdq_quantize_act_workspace_bytes", "svdq_quantize_act", "svdq_quantize_act_noalloc", "svdq_gemm_w4a4",
     "svdq_gemm_w4a4_qkv_norm_rope", "svdq_qkv_norm_rope", "svdq_gelu_mlp_workspace_bytes",
-    "svdq_gemm_w4a4_gelu_quant", "svdq_gelu", "svdq_gemm_w4a16", "svdq_svd_split_workspace_bytes",
+    "svdq_gemm_w4a4_gelu_quant", "svdq_gemm_w4a4_gelu", "svdq_gelu", "svdq_gemm_w4a16", "svdq_svd_split_workspace_bytes",
     "svdq_svd_split",
     "svdq_device_status",
     "svdq_debug_set_wait_limit_ns", "svdq_debug_timeout_probe", "svdq_debug_override_capability",
@@ -91,6 +91,8 @@ def _load():
     lib.svdq_gemm_w4a4_gelu_quant.argtypes = [I, I, P, P, P, I64, P, P, P, I64, I64, P, P, I, P, I, P, P, I, P, P, P,
                                               P, P, P, ctypes.c_size_t, P]
     lib.svdq_gemm_w4a4_gelu_quant.restype = I
+    lib.svdq_gemm_w4a4_gelu.argtypes = [I, I, P, P, P, I64, P, P, P, I64, I64, P, P, I, P, I, P, P]
+    lib.svdq_gemm_w4a4_gelu.restype = I
     lib.svdq_gelu.argtypes = [P, P, I64, I, P]
     lib.svdq_gelu.restype = I
     lib.svdq_gemm_w4a16.argtypes = [P, I64, P, P, I64, I64, P, P, P]
@@ -247,6 +249,14 @@ def svdq_gemm_w4a4_gelu_quant(precision, group_size, x_codes, x_scales, x_tensor
         int(rank), _ptr(bias), int(gelu_approx), _ptr(next_inv_lambda), _ptr(next_L_down_t), int(next_rank),
         _ptr(next_x_tensor_scale), _ptr(next_w_tensor_scale), _ptr(next_x_codes), _ptr(next_x_scales),
         _ptr(next_lowrank_act), _ptr(workspace), int(workspace_bytes), _stream(stream)), "svdq_gemm_w4a4_gelu_quant")
+
+
+def svdq_gemm_w4a4_gelu(precision, group_size, x_codes, x_scales, x_tensor_scale, M, w_codes, w_scales,
+                        w_tensor_scale, N, K, lowrank_act, L_up_t, rank, bias, gelu_approx, y, stream=None) -> None:
+    _check(lib.svdq_gemm_w4a4_gelu(
+        _prec(precision), int(group_size), _ptr(x_codes), _ptr(x_scales), _ptr(x_tensor_scale), int(M),
+        _ptr(w_codes), _ptr(w_scales), _ptr(w_tensor_scale), int(N), int(K), _ptr(lowrank_act), _ptr(L_up_t),
+        int(rank), _ptr(bias), int(gelu_approx), _ptr(y), _stream(stream)), "svdq_gemm_w4a4_gelu")
 
 
 def svdq_gelu(x, y, n, approx=0, stream=None) -> None:

@@ -382,6 +382,40 @@ __device__ __forceinline__ void gp_gelu_epilogue(const uint32_t (&acc)[NC], cons
 // 128 accumulators, as 16 packed words.  The bias pair of the warp's columns
 // 2j, 2j + 1 (word j of its bias) sits in lane j % 32, entry j / 32 of qb
 // (zero past N), fetched before the accumulator was ready.
+// The GELU epilogue's store-only form: this thread's row, columns nbase ..
+// nbase + NC - 1 of h = bf16(GELU(bf16(S acc + b))) (the y of the plain
+// epilogue, then the same table GELU as the fused path and the unfused pass)
+// written to y, 16 bytes at a time.
+template <int NC>
+__device__ __forceinline__ void gp_gelu_store(const uint32_t (&acc)[NC], const GemmArgs& a, float S, int64_t grow,
+                                              int nbase, const uint16_t* gelu_tab) {
+    if (grow >= a.M) return;
+    __nv_bfloat16* yrow = a.y + grow * (int64_t)a.N + nbase;
+#pragma unroll
+    for (int c = 0; c < NC / 16; ++c) {
+        const int n = nbase + 16 * c;
+        uint32_t bw[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+        if (a.bias) {
+            const uint4 w0 = __ldg(reinterpret_cast<const uint4*>(a.bias + n));
+            const uint4 w1 = __ldg(reinterpret_cast<const uint4*>(a.bias + n) + 1);
+            bw[0] = w0.x, bw[1] = w0.y, bw[2] = w0.z, bw[3] = w0.w;
+            bw[4] = w1.x, bw[5] = w1.y, bw[6] = w1.z, bw[7] = w1.w;
+        }
+        uint32_t hb[8];
+#pragma unroll
+        for (int p = 0; p < 8; ++p) {
+            const float o0 = fmaf(__uint_as_float(acc[16 * c + 2 * p]), S, bf16lo_to_f32(bw[p]));
+            const float o1 = fmaf(__uint_as_float(acc[16 * c + 2 * p + 1]), S, bf16hi_to_f32(bw[p]));
+            const __nv_bfloat162 y2 = __floats2bfloat162_rn(o0, o1);
+            const uint32_t yb = *reinterpret_cast<const uint32_t*>(&y2);
+            hb[p] = gelu_bf16_bits(yb & 0xFFFFu, gelu_tab) | (gelu_bf16_bits(yb >> 16, gelu_tab) << 16);
+        }
+        uint4* dst = reinterpret_cast<uint4*>(yrow + 16 * c);
+        dst[0] = make_uint4(hb[0], hb[1], hb[2], hb[3]);
+        dst[1] = make_uint4(hb[4], hb[5], hb[6], hb[7]);
+    }
+}
+
 __device__ __forceinline__ void gp_pack32(const uint32_t (&acc)[128], int c2, const uint32_t (&qb)[2], float S,
                                           uint32_t (&pk)[16]) {
 #pragma unroll
@@ -661,7 +695,7 @@ __global__ void __launch_bounds__(gp_threads<kEpi>(), 1)
             reinterpret_cast<const uint16_t*>(gelu_base + (size_t)kEpiWarpsGelu * kGeluScratch);
         float* gelu_inv = reinterpret_cast<float*>(gelu_base + (size_t)kEpiWarpsGelu * kGeluScratch + kGeluTabBytes);
         if (kEpi == kEpiGelu) {
-            const float S2 = *a.nx_x_scale;
+            const float S2 = a.gelu_store ? 1.0f : *a.nx_x_scale;   // unused by the store-only form
             gelu_six_s2 = __fmul_rn(6.0f, S2);
             gelu_scr = smem_u32(gelu_base);
             // reciprocals of the 128 decoded group scales e * S2, as the
@@ -760,10 +794,14 @@ __global__ void __launch_bounds__(gp_threads<kEpi>(), 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
                 // warp-uniform: with N % 128 == 0 a warp's columns are all in or all out
-                if (gbase < a.N)
-                    gp_gelu_epilogue<64>(acc, a, S, gelu_six_s2, gelu_inv, grow, gbase,
-                                         gelu_scr + (uint32_t)(warp - kEpiWarp0) * (uint32_t)kGeluScratch,
-                                         gelu_tab, lane);
+                if (gbase < a.N) {
+                    if (a.gelu_store)
+                        gp_gelu_store<64>(acc, a, S, grow, gbase, gelu_tab);
+                    else
+                        gp_gelu_epilogue<64>(acc, a, S, gelu_six_s2, gelu_inv, grow, gbase,
+                                             gelu_scr + (uint32_t)(warp - kEpiWarp0) * (uint32_t)kGeluScratch,
+                                             gelu_tab, lane);
+                }
                 continue;
             }
             uint32_t acc[128];

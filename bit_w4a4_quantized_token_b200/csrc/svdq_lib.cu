@@ -568,6 +568,7 @@ struct QkvEpilogue {
 // The fused GELU + next-layer activation epilogue's arguments (next_x_scale ==
 // nullptr: not used).
 struct GeluEpilogue {
+    bool store_y = false;   // store h = bf16(GELU(y)) to y; the next-layer fields below are then unused
     int approx = 0;
     const float* next_inv_lambda = nullptr;
     const void* next_L_down_t = nullptr;
@@ -626,7 +627,10 @@ svdq_status gemm_nvfp4_pair(const void* x_codes, const void* x_scales, const flo
         a.q_cols = qkv.heads * 128;
         a.qk_cols = 2 * qkv.heads * 128;
     }
-    if (gelu.next_x_scale) {
+    if (gelu.store_y) {
+        a.gelu_approx = gelu.approx;
+        a.gelu_store = 1;
+    } else if (gelu.next_x_scale) {
         a.gelu_approx = gelu.approx;
         a.nx_inv_lambda = gelu.next_inv_lambda;
         a.nx_ldt = reinterpret_cast<const __nv_bfloat16*>(gelu.next_L_down_t);
@@ -646,7 +650,7 @@ svdq_status gemm_nvfp4_pair(const void* x_codes, const void* x_scales, const flo
     // the activation quantizer, which releases its dependents early
     const dim3 grid(2 * (unsigned)clusters), block(gp_threads<kEpiPlain>());   // the QKV variant's too
     cudaError_t e;
-    if (gelu.next_x_scale)
+    if (gelu.next_x_scale || gelu.store_y)
         e = launch_ex(gemm_nvfp4_pair_kernel<kEpiGelu>, grid, dim3(gp::kThreadsGelu), gp::SMEM_BYTES_GELU, st, 2u,
                       tm_xc, tm_wc, tm_sfa, tm_sfb, tm_L, tm_Lup, tm_xc, a);
     else {
@@ -1054,6 +1058,39 @@ svdq_status svdq_gelu_mlp_workspace_bytes(int64_t M, int next_rank, size_t* byte
     if (next_rank > 32 || M < 1 || M >= (int64_t(1) << 31)) return SVDQ_ERR_UNSUPPORTED_SHAPE;
     *bytes = (size_t)M * (size_t)next_rank * sizeof(float);
     return SVDQ_OK;
+}
+
+svdq_status svdq_gemm_w4a4_gelu(svdq_precision p, int group_size, const void* x_codes, const void* x_scales,
+                                const float* x_tensor_scale, int64_t M, const void* w_codes, const void* w_scales,
+                                const float* w_tensor_scale, int64_t N, int64_t K, const void* lowrank_act,
+                                const void* L_up_t, int rank, const void* bias, int gelu_approx, void* y,
+                                svdq_stream_t stream) {
+    SVDQ_TRY(check_precision(p, group_size));
+    if (p != SVDQ_NVFP4) return SVDQ_ERR_INVALID_ARG;   // the GELU epilogue belongs to the nvfp4 GEMM
+    SVDQ_TRY(check_rank(rank));
+    if (gelu_approx != 0 && gelu_approx != 1) return SVDQ_ERR_INVALID_ARG;
+    SVDQ_TRY(check_dims(M, K));
+    SVDQ_TRY(check_dims(N, K));
+    if (N % 128 != 0) return SVDQ_ERR_UNSUPPORTED_SHAPE;   // whole 64-column pieces per epilogue warp
+    SVDQ_TRY(check_ptr(x_codes));
+    SVDQ_TRY(check_ptr(x_scales));
+    SVDQ_TRY(check_ptr(w_codes));
+    SVDQ_TRY(check_ptr(w_scales));
+    SVDQ_TRY(check_ptr(x_tensor_scale));
+    SVDQ_TRY(check_ptr(w_tensor_scale));
+    SVDQ_TRY(check_opt_ptr(bias));
+    SVDQ_TRY(check_ptr(y));
+    if (rank > 0) {
+        SVDQ_TRY(check_ptr(lowrank_act));
+        SVDQ_TRY(check_ptr(L_up_t));
+    }
+    SVDQ_TRY(check_device());
+    GeluEpilogue g;
+    g.store_y = true;
+    g.approx = gelu_approx;
+    return gemm_nvfp4_pair(x_codes, x_scales, x_tensor_scale, M, w_codes, w_scales, w_tensor_scale, N, K,
+                           lowrank_act, L_up_t, rank, bias, y, reinterpret_cast<cudaStream_t>(stream), QkvEpilogue(),
+                           g);
 }
 
 svdq_status svdq_gemm_w4a4_gelu_quant(svdq_precision p, int group_size, const void* x_codes, const void* x_scales,

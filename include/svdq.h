@@ -316,6 +316,21 @@ svdq_status svdq_gemm_w4a4_gelu_quant(svdq_precision precision, int group_size,
                                       void* next_lowrank_act, void* workspace, size_t workspace_bytes,
                                       svdq_stream_t stream);
 
+/* fc1 of the same MLP with only the GELU in its epilogue (a partial fusion,
+ * no counterpart on the pages): y = bf16(GELU(bf16(fc1 linear output))),
+ * bit for bit svdq_gelu applied to svdq_gemm_w4a4's y, written to y [M, N]
+ * bf16 (device, 16-byte aligned); fc2 then runs svdq_quantize_act on it and
+ * svdq_gemm_w4a4.  Arguments as svdq_gemm_w4a4, plus gelu_approx as in
+ * svdq_gemm_w4a4_gelu_quant.  nvfp4 only.  One kernel on `stream`.  Errors:
+ * as svdq_gemm_w4a4; INVALID_ARG for int4 or a bad gelu_approx;
+ * UNSUPPORTED_SHAPE when N % 128 != 0. */
+svdq_status svdq_gemm_w4a4_gelu(svdq_precision precision, int group_size,
+                                const void* x_codes, const void* x_scales, const float* x_tensor_scale,
+                                int64_t M, const void* w_codes, const void* w_scales,
+                                const float* w_tensor_scale, int64_t N, int64_t K,
+                                const void* lowrank_act, const void* L_up_t, int rank, const void* bias,
+                                int gelu_approx, void* y, svdq_stream_t stream);
+
 /* The unfused activation pass of the same MLP: y[i] = bf16(GELU(x[i])) over n
  * finite bf16 elements (device pointers, 16-byte aligned; y may equal x);
  * the same bf16 -> bf16 function the fused epilogue applies, so both paths

@@ -18,7 +18,9 @@ epilogue applies GELU and performs fc2's activation step itself.  Checks:
   correct fp32 summation orders round differently (the codes agree on >= 99 %
   of the elements), so there only the 1 %-of-rms bound holds on every element
   and the 1-ulp agreement is asked of >= 99 % of them;
-* the workspace of partial sums is left zeroed.
+* the workspace of partial sums is left zeroed;
+* fc1 with only the GELU in its epilogue (svdq_gemm_w4a4_gelu) stores the
+  GELU pass's h on fc1's y, bit for bit.
 """
 import numpy as np
 import pytest
@@ -84,8 +86,13 @@ def _run(M, D, Hd, r1, r2, approx, rows=None, cal_rows=None):
     _lib.svdq_gelu(y1, h, M * Hd, approx)
     qu = layer.quantize_act(h, p2, x_tensor_scale=S2)
     y2u = layer.gemm(qu, p2)
+    # the partial fusion: fc1's epilogue applies only the GELU and stores h
+    hs = torch.empty_like(y1)
+    _lib.svdq_gemm_w4a4_gelu("nvfp4", 16, q1.x_codes, q1.x_scales, q1.x_tensor_scale, M, p1.w_codes, p1.w_scales,
+                             p1.w_tensor_scale, Hd, D, q1.lowrank_act, p1.L_up_t, r1, p1.bias, approx, hs)
     torch.cuda.synchronize()
     assert float(ws.abs().max()) == 0.0, "workspace not left zeroed"
+    assert torch.equal(hs, h), "the GELU epilogue's h differs from the GELU pass on fc1's y"
     r1o, ho, r2o = O.gelu_mlp(x_bits, fc1, fc2, S1, S2, approx, rows=rows)
     # fc2 alone on the GPU's h (the unfused pass's bits; the fused path hands fc2 the same codes)
     h_rows = u16(h) if rows is None else u16(h)[np.asarray(rows)]
@@ -197,4 +204,21 @@ def test_fused_mlp_argument_checks():
                         (dict(next_x_tensor_scale=None), _lib.SVDQ_ERR_INVALID_ARG)):
         with pytest.raises(_lib.SvdqError) as e:
             _lib.svdq_gemm_w4a4_gelu_quant(**dict(args, **bad))
+        assert e.value.status == status, bad
+
+
+def test_gelu_epilogue_argument_checks():
+    from bit_w4a4_quantized_token_b200 import _lib
+
+    fake = 1 << 20
+    args = dict(precision="nvfp4", group_size=16, x_codes=fake, x_scales=fake, x_tensor_scale=fake, M=64,
+                w_codes=fake, w_scales=fake, w_tensor_scale=fake, N=512, K=256, lowrank_act=fake, L_up_t=fake,
+                rank=32, bias=None, gelu_approx=0, y=fake)
+    for bad, status in ((dict(N=576), _lib.SVDQ_ERR_UNSUPPORTED_SHAPE),
+                        (dict(gelu_approx=2), _lib.SVDQ_ERR_INVALID_ARG),
+                        (dict(precision="int4", group_size=64), _lib.SVDQ_ERR_INVALID_ARG),
+                        (dict(y=None), _lib.SVDQ_ERR_INVALID_ARG),
+                        (dict(y=fake + 2), _lib.SVDQ_ERR_INVALID_ARG)):
+        with pytest.raises(_lib.SvdqError) as e:
+            _lib.svdq_gemm_w4a4_gelu(**dict(args, **bad))
         assert e.value.status == status, bad
