@@ -76,7 +76,6 @@ struct GemmArgs {
     uint8_t* nx_scales;              // their E4M3 group scales, tensor-core layout, K = N
     float* nx_acc;                   // [M, nx_rank] fp32 sums of h (L_down / lambda), zero on entry
     int nx_rows_pad;                 // rows of nx_scales: M rounded up to 128
-    int gelu_store;                  // kEpiGelu with 1: store h = bf16(GELU(y)) to y instead (no next-layer step)
 };
 
 enum : uint32_t { kSiteGmEmpty = 16, kSiteGmFull = 17, kSiteGmAcc = 18, kSiteGmDrain = 19, kSiteGmAccEmpty = 20 };

@@ -133,7 +133,9 @@ static_assert(SMEM_BYTES_GELU <= 227 * 1024, "GELU epilogue buffers do not fit i
 
 // Epilogue variants of the pair kernel (separate instantiations, so that the
 // plain kernel keeps its registers).
-enum : int { kEpiPlain = 0, kEpiQkv = 1, kEpiGelu = 2 };
+// kEpiGeluStore: the GELU epilogue's store-only form (h = bf16(GELU(y)) to y).
+enum : int { kEpiPlain = 0, kEpiQkv = 1, kEpiGelu = 2, kEpiGeluStore = 3 };
+__host__ __device__ constexpr bool gp_is_gelu(int e) { return e == kEpiGelu || e == kEpiGeluStore; }
 
 // Bytes of the GEMM-ready copy of the weight scales of an N x K weight:
 // 16 KB per (256-row tile, 256 columns of K), whole tiles.
@@ -179,7 +181,7 @@ __device__ __forceinline__ uint64_t desc_sfb_kstep(uint32_t addr) {
 // faster for the plain one.
 template <int kEpi>
 __host__ __device__ constexpr int gp_epi_warps() {
-    return kEpi == kEpiGelu ? gp::kEpiWarpsGelu : gp::kEpiWarps;
+    return gp_is_gelu(kEpi) ? gp::kEpiWarpsGelu : gp::kEpiWarps;
 }
 template <int kEpi>
 __host__ __device__ constexpr int gp_threads() {
@@ -382,15 +384,16 @@ __device__ __forceinline__ void gp_gelu_epilogue(const uint32_t (&acc)[NC], cons
 // 128 accumulators, as 16 packed words.  The bias pair of the warp's columns
 // 2j, 2j + 1 (word j of its bias) sits in lane j % 32, entry j / 32 of qb
 // (zero past N), fetched before the accumulator was ready.
-// The GELU epilogue's store-only form: this thread's row, columns nbase ..
-// nbase + NC - 1 of h = bf16(GELU(bf16(S acc + b))) (the y of the plain
-// epilogue, then the same table GELU as the fused path and the unfused pass)
-// written to y, 16 bytes at a time.
+// The GELU epilogue's store-only form: columns nbase .. nbase + NC - 1 of
+// h = bf16(GELU(bf16(S acc + b))) (the y of the plain epilogue, then the same
+// table GELU as the fused path and the unfused pass) for the warp's 32 rows,
+// leaving through the warp's 1 KB of scratch as TMA stores of 32 x 16 boxes
+// (row-wise 16-byte stores by every thread took 32 us more over fc1 of the
+// DiT MLP).
 template <int NC>
-__device__ __forceinline__ void gp_gelu_store(const uint32_t (&acc)[NC], const GemmArgs& a, float S, int64_t grow,
-                                              int nbase, const uint16_t* gelu_tab) {
-    if (grow >= a.M) return;
-    __nv_bfloat16* yrow = a.y + grow * (int64_t)a.N + nbase;
+__device__ __forceinline__ void gp_gelu_store(const uint32_t (&acc)[NC], const GemmArgs& a, float S, int nbase,
+                                              const uint16_t* gelu_tab, uint32_t buf, uint32_t lane,
+                                              const CUtensorMap* tm_y, int row0) {
 #pragma unroll
     for (int c = 0; c < NC / 16; ++c) {
         const int n = nbase + 16 * c;
@@ -410,9 +413,16 @@ __device__ __forceinline__ void gp_gelu_store(const uint32_t (&acc)[NC], const G
             const uint32_t yb = *reinterpret_cast<const uint32_t*>(&y2);
             hb[p] = gelu_bf16_bits(yb & 0xFFFFu, gelu_tab) | (gelu_bf16_bits(yb >> 16, gelu_tab) << 16);
         }
-        uint4* dst = reinterpret_cast<uint4*>(yrow + 16 * c);
-        dst[0] = make_uint4(hb[0], hb[1], hb[2], hb[3]);
-        dst[1] = make_uint4(hb[4], hb[5], hb[6], hb[7]);
+        if (lane == 0) bulk_wait_group_read<0>();   // the previous box has left the buffer
+        __syncwarp();
+        st_shared_v4(buf + 32u * lane, hb[0], hb[1], hb[2], hb[3]);
+        st_shared_v4(buf + 32u * lane + 16u, hb[4], hb[5], hb[6], hb[7]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && row0 < a.M) {   // rows past M inside a box are clipped by the tensor map
+            tma_store_2d(tm_y, buf, n, row0);
+            bulk_commit_group();
+        }
     }
 }
 
@@ -524,7 +534,7 @@ __global__ void __launch_bounds__(gp_threads<kEpi>(), 1)
         tmem_alloc_pair(tmem_slot, TMEM_COLS);
         tmem_relinquish_pair();
     }
-    if (kEpi == kEpiGelu)     // the bf16 GELU table (gelu_mlp.cuh), once per CTA
+    if (gp_is_gelu(kEpi))     // the bf16 GELU table (gelu_mlp.cuh), once per CTA
         gelu_table_fill(reinterpret_cast<uint16_t*>(smem + (size_t)kStages * STAGE_BYTES + 256 +
                                                     (size_t)kEpiWarpsGelu * kGeluScratch),
                         (int)threadIdx.x, gp_threads<kEpi>(), a.gelu_approx);
@@ -694,8 +704,8 @@ __global__ void __launch_bounds__(gp_threads<kEpi>(), 1)
         const uint16_t* gelu_tab =
             reinterpret_cast<const uint16_t*>(gelu_base + (size_t)kEpiWarpsGelu * kGeluScratch);
         float* gelu_inv = reinterpret_cast<float*>(gelu_base + (size_t)kEpiWarpsGelu * kGeluScratch + kGeluTabBytes);
-        if (kEpi == kEpiGelu) {
-            const float S2 = a.gelu_store ? 1.0f : *a.nx_x_scale;   // unused by the store-only form
+        if (gp_is_gelu(kEpi)) {
+            const float S2 = kEpi == kEpiGeluStore ? 1.0f : *a.nx_x_scale;   // unused by the store-only form
             gelu_six_s2 = __fmul_rn(6.0f, S2);
             gelu_scr = smem_u32(gelu_base);
             // reciprocals of the 128 decoded group scales e * S2, as the
@@ -721,7 +731,7 @@ __global__ void __launch_bounds__(gp_threads<kEpi>(), 1)
             // sin), and a Q or K head's RMSNorm weights go with the bias
             uint32_t qbias[2] = {0u, 0u}, qgam[2] = {0u, 0u};
             const bool qk_head = kEpi == kEpiQkv && nbase < a.qk_cols;
-            if (kEpi != kEpiGelu && a.bias) {
+            if (!gp_is_gelu(kEpi) && a.bias) {
 #pragma unroll
                 for (int i = 0; i < 2; ++i) {
                     const int col = nbase + 2 * (32 * i + (int)lane);
@@ -780,7 +790,7 @@ __global__ void __launch_bounds__(gp_threads<kEpi>(), 1)
                 break;
             }
             tc_fence_after();
-            if (kEpi == kEpiGelu) {
+            if (gp_is_gelu(kEpi)) {
                 // four warps per lane quadrant: this warp's 64 columns
                 const int part = (int)(warp - kEpiWarp0) >> 2;
                 const int gbase = n_tile * BN + 64 * part;
@@ -795,8 +805,10 @@ __global__ void __launch_bounds__(gp_threads<kEpi>(), 1)
                 if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
                 // warp-uniform: with N % 128 == 0 a warp's columns are all in or all out
                 if (gbase < a.N) {
-                    if (a.gelu_store)
-                        gp_gelu_store<64>(acc, a, S, grow, gbase, gelu_tab);
+                    if (kEpi == kEpiGeluStore)
+                        gp_gelu_store<64>(acc, a, S, gbase, gelu_tab,
+                                          gelu_scr + (uint32_t)(warp - kEpiWarp0) * (uint32_t)kGeluScratch, lane,
+                                          &tm_y, (int)(grow - (int64_t)lane));
                     else
                         gp_gelu_epilogue<64>(acc, a, S, gelu_six_s2, gelu_inv, grow, gbase,
                                              gelu_scr + (uint32_t)(warp - kEpiWarp0) * (uint32_t)kGeluScratch,

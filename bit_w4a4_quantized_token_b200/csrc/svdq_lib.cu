@@ -130,6 +130,8 @@ svdq_status check_device() {
             cudaFuncSetAttribute(gemm_nvfp4_pair_kernel<kEpiQkv>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)gp::SMEM_BYTES_PLAIN) != cudaSuccess ||
             cudaFuncSetAttribute(gemm_nvfp4_pair_kernel<kEpiGelu>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)gp::SMEM_BYTES_GELU) != cudaSuccess ||
+            cudaFuncSetAttribute(gemm_nvfp4_pair_kernel<kEpiGeluStore>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)gp::SMEM_BYTES_GELU) != cudaSuccess)
             return cuda_fail("setting kernel shared-memory limits");
         g_device_ready[dev] = true;
@@ -629,7 +631,6 @@ svdq_status gemm_nvfp4_pair(const void* x_codes, const void* x_scales, const flo
     }
     if (gelu.store_y) {
         a.gelu_approx = gelu.approx;
-        a.gelu_store = 1;
     } else if (gelu.next_x_scale) {
         a.gelu_approx = gelu.approx;
         a.nx_inv_lambda = gelu.next_inv_lambda;
@@ -650,7 +651,15 @@ svdq_status gemm_nvfp4_pair(const void* x_codes, const void* x_scales, const flo
     // the activation quantizer, which releases its dependents early
     const dim3 grid(2 * (unsigned)clusters), block(gp_threads<kEpiPlain>());   // the QKV variant's too
     cudaError_t e;
-    if (gelu.next_x_scale || gelu.store_y)
+    if (gelu.store_y) {
+        // h leaves through TMA stores of 32-row x 16-column boxes
+        CUtensorMap tm_h;
+        if (!make_map(&tm_h, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, (uint64_t)N, (uint64_t)M, (uint64_t)N * 2, 16, 32,
+                      CU_TENSOR_MAP_SWIZZLE_NONE))
+            return SVDQ_ERR_CUDA;
+        e = launch_ex(gemm_nvfp4_pair_kernel<kEpiGeluStore>, grid, dim3(gp::kThreadsGelu), gp::SMEM_BYTES_GELU, st,
+                      2u, tm_xc, tm_wc, tm_sfa, tm_sfb, tm_L, tm_Lup, tm_h, a);
+    } else if (gelu.next_x_scale)
         e = launch_ex(gemm_nvfp4_pair_kernel<kEpiGelu>, grid, dim3(gp::kThreadsGelu), gp::SMEM_BYTES_GELU, st, 2u,
                       tm_xc, tm_wc, tm_sfa, tm_sfb, tm_L, tm_Lup, tm_xc, a);
     else {
