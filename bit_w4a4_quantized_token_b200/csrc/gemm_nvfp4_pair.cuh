@@ -238,13 +238,13 @@ __device__ __forceinline__ void gp_issue_stage(uint32_t acc, uint64_t da, uint64
 template <int NC>
 __device__ __forceinline__ void gp_gelu_epilogue(const uint32_t (&acc)[NC], const GemmArgs& a, float S,
                                                  float six_s2, const float* inv_tab, int64_t grow, int nbase,
-                                                 uint32_t scr, const uint16_t* gelu_tab, uint32_t lane) {
+                                                 uint32_t scr, const uint16_t* gelu_tab, uint32_t lane,
+                                                 const CUtensorMap* tm_codes) {
     static_assert(NC % 64 == 0, "a warp covers whole groups of four scale bytes");
     const bool row_ok = grow < a.M;
-    const int64_t half_k = (int64_t)a.N / 2;
     const int64_t kg4n = a.N / 64;
     uint32_t hpk[NC / 2];
-    uint32_t cw[4] = {0u, 0u, 0u, 0u};
+    uint32_t cw[NC / 8];   // this row's codes of the NC columns (4 bits each)
     uint32_t sword = 0u;
 #pragma unroll
     for (int c = 0; c < NC / 16; ++c) {
@@ -287,16 +287,11 @@ __device__ __forceinline__ void gp_gelu_epilogue(const uint32_t (&acc)[NC], cons
         float qv[8];
 #pragma unroll
         for (int i = 0; i < 8; i += 2) fmul2_rn(v[i], v[i + 1], inv, inv, qv[i], qv[i + 1]);
-        cw[2 * (c & 1)] = cvt_e2m1x8(qv);
+        cw[2 * c] = cvt_e2m1x8(qv);
 #pragma unroll
         for (int i = 0; i < 8; i += 2) fmul2_rn(v[8 + i], v[9 + i], inv, inv, qv[i], qv[i + 1]);
-        cw[2 * (c & 1) + 1] = cvt_e2m1x8(qv);
+        cw[2 * c + 1] = cvt_e2m1x8(qv);
         sword |= eb << (8 * (c & 3));
-        if (c & 1) {
-            if (row_ok)
-                *reinterpret_cast<uint4*>(a.nx_codes + grow * half_k + (n - 16) / 2) =
-                    make_uint4(cw[0], cw[1], cw[2], cw[3]);
-        }
         if ((c & 3) == 3) {
             const int64_t g0 = (n - 48) / 16;   // the first of these four groups (a multiple of 4)
             if (grow < a.nx_rows_pad)
@@ -304,6 +299,20 @@ __device__ __forceinline__ void gp_gelu_epilogue(const uint32_t (&acc)[NC], cons
             sword = 0u;
         }
     }
+    // the warp's 32 rows x NC / 2 bytes of codes leave through its scratch as
+    // one TMA store (row-wise 16-byte stores by every thread were slower)
+    static_assert(NC == 64, "one 32-byte code row per thread fills the 1 KB scratch");
+    const int64_t row0 = grow - (int64_t)lane;   // the warp's first row
+    st_shared_v4(scr + 32u * lane, cw[0], cw[1], cw[2], cw[3]);
+    st_shared_v4(scr + 32u * lane + 16u, cw[4], cw[5], cw[6], cw[7]);
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0 && row0 < a.M) {   // rows past M inside the box are clipped by the tensor map
+        tma_store_2d(tm_codes, scr, nbase / 2, (int)row0);
+        bulk_commit_group();
+    }
+    if (lane == 0) bulk_wait_group_read<0>();   // the scratch is reused below
+    __syncwarp();
     if (a.nx_rank == 0) return;
     // ---- rank-r down-projection of the next layer over these NC columns
     const int g = (int)(lane >> 2), t = (int)(lane & 3);
@@ -362,7 +371,6 @@ __device__ __forceinline__ void gp_gelu_epilogue(const uint32_t (&acc)[NC], cons
         }
         __syncwarp();
     }
-    const int64_t row0 = grow - (int64_t)lane;   // the warp's first row
 #pragma unroll
     for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
@@ -812,7 +820,7 @@ __global__ void __launch_bounds__(gp_threads<kEpi>(), 1)
                     else
                         gp_gelu_epilogue<64>(acc, a, S, gelu_six_s2, gelu_inv, grow, gbase,
                                              gelu_scr + (uint32_t)(warp - kEpiWarp0) * (uint32_t)kGeluScratch,
-                                             gelu_tab, lane);
+                                             gelu_tab, lane, &tm_y);
                 }
                 continue;
             }
@@ -885,8 +893,8 @@ __global__ void __launch_bounds__(gp_threads<kEpi>(), 1)
         }
     }
 
-    if (kEpi != kEpiGelu && warp >= (uint32_t)kEpiWarp0 && lane == 0)
-        bulk_wait_group<0>();   // this warp's y stores are done with shared memory and written
+    if (warp >= (uint32_t)kEpiWarp0 && lane == 0)
+        bulk_wait_group<0>();   // this warp's TMA stores are done with shared memory and written
     __syncthreads();
     if (s_failed && rank == 0 && warp == 0 && lane == 0) {
         // after a timeout, let the loads already issued land before either CTA

@@ -659,9 +659,15 @@ svdq_status gemm_nvfp4_pair(const void* x_codes, const void* x_scales, const flo
             return SVDQ_ERR_CUDA;
         e = launch_ex(gemm_nvfp4_pair_kernel<kEpiGeluStore>, grid, dim3(gp::kThreadsGelu), gp::SMEM_BYTES_GELU, st,
                       2u, tm_xc, tm_wc, tm_sfa, tm_sfb, tm_L, tm_Lup, tm_h, a);
-    } else if (gelu.next_x_scale)
+    } else if (gelu.next_x_scale) {
+        // fc2's codes leave through TMA stores of 32-row x 32-byte boxes
+        CUtensorMap tm_codes;
+        if (!make_map(&tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, gelu.next_codes, (uint64_t)N / 2, (uint64_t)M,
+                      (uint64_t)N / 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE))
+            return SVDQ_ERR_CUDA;
         e = launch_ex(gemm_nvfp4_pair_kernel<kEpiGelu>, grid, dim3(gp::kThreadsGelu), gp::SMEM_BYTES_GELU, st, 2u,
-                      tm_xc, tm_wc, tm_sfa, tm_sfb, tm_L, tm_Lup, tm_xc, a);
+                      tm_xc, tm_wc, tm_sfa, tm_sfb, tm_L, tm_Lup, tm_codes, a);
+    }
     else {
         // y leaves through TMA stores of 32 x 32 boxes (64-byte swizzle)
         CUtensorMap tm_y;
